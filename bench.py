@@ -1,0 +1,498 @@
+#!/usr/bin/env python
+"""MoE dispatch + combine on B200: tokens/s and achieved HBM GB/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload train8k]
+    python bench.py --impl reference ...      # the CPU oracle, timed on host cores
+
+One step is the whole hot path over one batch: layout (count, scan, assign)
+-> dispatch (permute into the expert-major pool; FP8 quantisation for the FP8
+workloads; tile_ready publication plus a consumer on a second stream for the
+streaming workload) -> combine (weighted top-k reduction back to token order),
+with identity experts (combine reads the dispatched pool; FP8 workloads read a
+seeded bf16 pool).  Inputs are resident in HBM before timing; the L2 is flushed
+(a 2 x L2 write) before every timed step and the flush is outside the events.
+
+Multi-GPU (torchrun): every rank runs the same workload on its own token shard
+(its own seed), with no collective on the data path (weak scaling); the step
+time is the maximum over ranks.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+from dataclasses import replace
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "dispatch+combine tokens/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------------ helpers
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="train8k", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-flush", action="store_true", help="skip the L2 flush (reported in config)")
+    ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--consumer-ctas", type=int, default=16)
+    return ap.parse_args(argv)
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def shard_workload(w: W.Workload, rank: int) -> W.Workload:
+    """Each rank's token shard: same shapes, its own seed (rank 0 keeps the workload's seed)."""
+    return replace(w, seed=w.seed + 100_000 * rank)
+
+
+def algorithmic_bytes(w: W.Workload) -> dict:
+    """Bytes the path must move at minimum; padding rows are never counted.
+
+    dispatch: read x once (T*H*2) + write N_a payload rows (N_a*H*b_p) + scales
+              (N_a*H/128*b_s) + read src_pool_row (4*N_a)
+    combine:  read N_a rows of y (N_a*H*2) + write out (T*H*2) + read
+              src_pool_row and topk_weight (8*N_a)
+    layout:   read topk_idx (4*N_a) + write src_pool_row, pool_recv_token,
+              pool_recv_slot (12*N_a)
+    """
+    Na, T, H = w.n_assign, w.T, w.H
+    bp = 2 if w.payload == "bf16" else 1
+    bs = {"none": 0, "f32": 4, "f32_pow2": 4, "ue8m0": 1}[w.scale]
+    groups = H // 128 if w.payload == "fp8" else 0
+    layout = 16 * Na
+    dispatch = T * H * 2 + Na * H * bp + Na * groups * bs + 4 * Na
+    combine = Na * H * 2 + T * H * 2 + 8 * Na
+    consumer = 2 * Na * H * bp if w.streaming else 0
+    return {"layout": layout, "dispatch": dispatch, "combine": combine,
+            "total": layout + dispatch + combine, "consumer": consumer}
+
+
+def load_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "combine_route_layout_02_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            table = json.load(f)
+    except Exception:
+        return None
+    ent = table.get(workload, {}).get(kernel)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = [("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown")]
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+            phys = device_index
+            if visible:
+                ids = [v for v in visible.split(",") if v.strip()]
+                if device_index < len(ids) and ids[device_index].strip().isdigit():
+                    phys = int(ids[device_index])
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(phys)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            self._ok = False
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, const in self.REASONS:
+                    if bits & getattr(nv, const, 0):
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._ok:
+            self._t.join()
+
+    def summary(self) -> dict:
+        if not self._ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples), "source": "nvml unavailable" if not self._ok else "nvml"}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml"}
+
+
+def reduce_max(values, world: int, device=None):
+    """Element-wise max over ranks (timing only; not a data-path collective)."""
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------ cpu oracle
+
+def oracle_step(w: W.Workload, d: dict, y_pool=None):
+    """One step of the plain oracle: layout -> dispatch -> combine."""
+    import oracle
+    lay = oracle.layout(d["topk_idx"].numpy(), w.E, w.R, w.B)
+    if w.payload == "bf16":
+        recv = oracle.dispatch_bf16(d["x"], lay)
+        y = recv
+    else:
+        oracle.dispatch_fp8(d["x"], lay, w.scale)
+        y = y_pool
+    return oracle.combine(y, d["topk_weight"].numpy(), lay)
+
+
+def oracle_y_pool(w: W.Workload, rows: int):
+    import numpy as np
+    import oracle
+    table = oracle.as_u16(W.random_x(61, w.H, seed=w.seed + 7))
+    return np.take(table, np.arange(max(rows, 1)) % 61, axis=0)
+
+
+def sample_inputs(w: W.Workload, d: dict, T: int):
+    ws = replace(w, T=T)
+    return ws, {"x": d["x"][:T].contiguous(), "topk_idx": d["topk_idx"][:T].contiguous(),
+                "topk_weight": d["topk_weight"][:T].contiguous()}
+
+
+def cpu_baseline(w: W.Workload, d: dict, budget_s: float) -> dict:
+    """The oracle as it stands (single-threaded C), timed on a bounded sample."""
+    import oracle
+    y = None
+    if w.payload != "bf16":
+        y = oracle_y_pool(w, oracle.capacity_rows(w.n_assign, w.E, w.B))
+    t0 = time.perf_counter()
+    oracle_step(w, d, y)
+    first = time.perf_counter() - t0
+    reps, total = 1, first
+    while total + first <= budget_s:
+        t0 = time.perf_counter()
+        oracle_step(w, d, y)
+        total += time.perf_counter() - t0
+        reps += 1
+    per = total / reps
+    return {"value": w.T / per, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"full {w.name} step (T={w.T}) x {reps}, single-threaded C oracle, "
+                      f"{per * 1e3:.1f} ms per step",
+            "ms_per_step": per * 1e3}
+
+
+# ------------------------------------------------------------- our arm
+
+def run_ours(args, rank: int, world: int, local: int) -> dict | None:
+    import torch
+    import combine_route_layout_02_b200 as sep
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = W.WORKLOADS[args.workload]
+    wr = shard_workload(w, rank)
+    d = W.make_inputs(wr)
+    x = d["x"].to(dev)
+    idx = d["topk_idx"].to(dev)
+    wt = d["topk_weight"].to(dev)
+    T, H = w.T, w.H
+
+    h = sep.sep_handle_create(T, w.k, w.E, w.R, w.B)
+    info = h.info()
+    rows = info.max_pool_rows
+    recv, scales = sep.alloc_pool(h, H, w.payload, w.scale, rows=rows)
+    if w.payload == "bf16":
+        y = recv
+    else:
+        import numpy as np
+        table = W.random_x(61, H, seed=w.seed + 7).to(dev)
+        y = table[torch.arange(rows, device=dev) % 61].contiguous()
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    main = torch.cuda.current_stream()
+    side = torch.cuda.Stream() if w.streaming else None
+    tile_ready = torch.zeros(info.max_tiles, dtype=torch.int32, device=dev) if w.streaming else None
+    dst = torch.empty_like(recv) if w.streaming else None
+    status = torch.zeros(2, dtype=torch.int32, device=dev) if w.streaming else None
+    seq = [0]
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = None if args.no_flush else torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+
+    def step(ev=None, xs=x, idxs=idx, wts=wt):
+        if ev is not None:
+            ev[0].record(main)
+        sep.sep_layout(idxs, w.E, w.R, w.B, handle=h)
+        epoch = h.epoch
+        if ev is not None:
+            ev[1].record(main)
+        if w.streaming:
+            seq[0] += 1
+            side.wait_stream(main)
+            sep.sep_consume_tiles(h, recv, tile_ready, seq[0], dst, status, num_ctas=args.consumer_ctas,
+                                  stream=side)
+            sep.sep_dispatch(h, xs, recv, tile_ready=tile_ready, dispatch_seq=seq[0])
+        else:
+            sep.sep_dispatch(h, xs, recv, payload=w.payload, scale=w.scale, recv_scales=scales)
+        if ev is not None:
+            ev[2].record(main)
+        sep.sep_combine(h, y, wts, out, layout_epoch=epoch)
+        if ev is not None:
+            ev[3].record(main)
+        if w.streaming:
+            main.wait_stream(side)
+            if ev is not None:
+                ev[4].record(main)
+
+    for _ in range(args.warmup):
+        if flush is not None:
+            flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if w.streaming:
+        assert status.cpu().tolist() == [0, 0], f"consumer status {status.cpu().tolist()}"
+
+    nev = 5 if w.streaming else 4
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    with sampler:
+        for i in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            step(events[i])
+        torch.cuda.synchronize()
+    barrier(world)
+    if w.streaming:
+        assert status.cpu().tolist() == [0, 0], f"consumer status {status.cpu().tolist()}"
+
+    lay_ms = [e[0].elapsed_time(e[1]) for e in events]
+    dis_ms = [e[1].elapsed_time(e[2]) for e in events]
+    com_ms = [e[2].elapsed_time(e[3]) for e in events]
+    tot_ms = [e[0].elapsed_time(e[nev - 1]) for e in events]
+    mean = statistics.fmean
+    local_vals = [mean(tot_ms), mean(lay_ms), mean(dis_ms), mean(com_ms)]
+    step_ms, layout_ms, dispatch_ms, combine_ms = reduce_max(local_vals, world, dev)
+
+    # end to end through the C ABI: pinned host inputs in, combined output back out
+    x_h, idx_h, wt_h = d["x"].pin_memory(), d["topk_idx"].pin_memory(), d["topk_weight"].pin_memory()
+    out_h = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+    x_d, idx_d, wt_d = torch.empty_like(x), torch.empty_like(idx), torch.empty_like(wt)
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        idx_d.copy_(idx_h, non_blocking=True)
+        wt_d.copy_(wt_h, non_blocking=True)
+        step(None, x_d, idx_d, wt_d)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.e2e_steps)]
+    barrier(world)
+    for i in range(args.e2e_steps):
+        if flush is not None:
+            flush.zero_()
+        e2e_ev[i][0].record(main)
+        e2e_step()
+        e2e_ev[i][1].record(main)
+    torch.cuda.synchronize()
+    barrier(world)
+    (e2e_ms,) = reduce_max([mean([a.elapsed_time(b) for a, b in e2e_ev])], world, dev)
+    h2d = x_h.numel() * 2 + idx_h.numel() * idx_h.element_size() + wt_h.numel() * 4
+    d2h = out_h.numel() * 2
+    sep.sep_handle_free(h)
+
+    ab = algorithmic_bytes(w)
+    peaks = load_peaks()
+    kern = {"dispatch": (dispatch_ms, ab["dispatch"]), "combine": (combine_ms, ab["combine"])}
+    dom = max(kern, key=lambda k: kern[k][0])
+    dom_ms, dom_bytes = kern[dom]
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    step_gbs = ab["total"] / (step_ms * 1e-3) / 1e9
+    launches_per_step = 3 + 1 + 1 + (1 if w.streaming else 0)
+    traffic = profiled_traffic(w.name, dom)
+
+    res = {
+        "metric": METRIC,
+        "value": world * T / (step_ms * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.payload == "bf16" else "fp8-e4m3 dispatch, bf16 combine",
+        "data": "synthetic",
+        "config": {"workload": w.name, "T": T, "H": H, "E": w.E, "owners": w.R, "top_k": w.k,
+                   "block_m": w.B, "payload": w.payload, "scale": w.scale,
+                   "experts": "identity (combine reads the dispatched pool)" if w.payload == "bf16"
+                   else "identity-shaped (combine reads a seeded bf16 pool)",
+                   "streaming": w.streaming, "parallelism": f"{world} independent token shards",
+                   "l2": "not flushed" if args.no_flush else f"flushed before every timed step ({2 * l2 >> 20} MB write, outside the events)",
+                   "sm_count": n_sms, "timing": "CUDA events per step on the launching stream, mean of steps, max over ranks"},
+        "achieved_gbs": step_gbs,
+        "pct_of_peak": 100.0 * step_gbs / peaks["hbm_gbs"],
+        "phases_us": {"layout": layout_ms * 1e3, "dispatch": dispatch_ms * 1e3, "combine": combine_ms * 1e3},
+        "phase_gbs": {"layout": ab["layout"] / (layout_ms * 1e-3) / 1e9,
+                      "dispatch": ab["dispatch"] / (dispatch_ms * 1e-3) / 1e9,
+                      "combine": ab["combine"] / (combine_ms * 1e-3) / 1e9},
+        "algorithmic_bytes": ab,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "peak_source": peaks["source"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": traffic},
+        "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(wr, d, args.cpu_budget)
+    return res if rank == 0 else None
+
+
+# ------------------------------------------------------- reference arm
+
+def run_reference(args, rank: int) -> dict | None:
+    """The CPU oracle as it stands, on the host cores, on a bounded sample."""
+    if rank != 0:
+        return None
+    w = W.WORKLOADS[args.workload]
+    d = W.make_inputs(w)
+    import oracle
+    y_full = None
+    if w.payload != "bf16":
+        y_full = oracle_y_pool(w, oracle.capacity_rows(w.n_assign, w.E, w.B))
+    # size the per-step sample so that warm-up + timed steps take about two minutes
+    t0 = time.perf_counter()
+    oracle_step(*sample_inputs(w, d, min(w.T, 256)), y_full)
+    per_tok = (time.perf_counter() - t0) / min(w.T, 256)
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    Ts = int(max(16, min(w.T, budget / max(per_tok, 1e-9))))
+    ws, ds = sample_inputs(w, d, Ts)
+    for _ in range(args.warmup):
+        oracle_step(ws, ds, y_full)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_step(ws, ds, y_full)
+        times.append(time.perf_counter() - t0)
+    per = statistics.fmean(times)
+    value = Ts / per
+    sample = f"first {Ts} of {w.T} tokens of {w.name} per step, single-threaded C oracle"
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if w.payload == "bf16" else "fp8-e4m3 dispatch, bf16 combine",
+        "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "H": w.H, "E": w.E, "owners": w.R, "top_k": w.k,
+                   "block_m": w.B, "payload": w.payload, "scale": w.scale, "sample_tokens": Ts},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main(argv=None) -> int:
+    args = parse_args(argv)
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        res = run_reference(args, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    try:
+        res = run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if res is not None:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

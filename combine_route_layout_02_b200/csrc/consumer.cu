@@ -1,0 +1,103 @@
+// Reference consumer of a streaming dispatch (StreamEP README, "Streaming
+// dispatch in one paragraph": a consumer kernel on another stream spins on
+// the acquire-load of tile_ready[tile] >= dispatch_seq and proceeds; padding
+// rows are predicated out by pool_recv_token >= 0).
+//
+// Persistent CTAs walk the tiles in the order a token-major dispatch finishes
+// them: tile i of every expert before tile i+1 of any.  Position n of that
+// order belongs to CTA n % gridDim.x.  Thread 0 waits (acquire load, bounded by
+// %globaltimer and a poll budget, with nanosleep back-off), the CTA barrier
+// passes the acquired view to the other threads, and the CTA copies the tile's
+// valid rows with L2-coherent loads.  When a wait gives up, status[0] becomes
+// SEP_ERR_TIMEOUT; every CTA then stops waiting and counts its remaining tiles
+// in status[1].  No wait is unbounded.
+#include "sep_internal.cuh"
+
+namespace sep {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kMaxExperts = 1024;
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *ptr)
+{
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint64_t global_time_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// 1 once tile_ready[tile] has reached seq; 0 if this or another CTA gave up.
+__device__ int wait_tile(const ConsumeParams &p, int tile)
+{
+    const uint64_t t0 = global_time_ns();
+    for (uint32_t polls = 0;; ++polls) {
+        if ((int32_t)(ld_acquire_gpu(p.tile_ready + tile) - p.seq) >= 0)
+            return 1;
+        if (*reinterpret_cast<volatile const uint32_t *>(p.abort_flag) != 0u)
+            return 0;
+        if (polls >= p.max_polls || global_time_ns() - t0 > p.timeout_ns) {
+            atomicCAS(p.abort_flag, 0u, (uint32_t)SEP_ERR_TIMEOUT);
+            return 0;
+        }
+        __nanosleep(256);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads) consume_tiles_kernel(ConsumeParams p)
+{
+    __shared__ int s_off[kMaxExperts + 1];
+    __shared__ int s_go;
+    for (int e = threadIdx.x; e <= p.E; e += blockDim.x)
+        s_off[e] = p.expert_pool_block_offset[e];
+    __syncthreads();
+    int max_tau = 0;
+    for (int e = 0; e < p.E; ++e)
+        max_tau = max(max_tau, s_off[e + 1] - s_off[e]);
+
+    const int64_t vecs = p.row_bytes / 16;
+    long long pos = 0;
+    for (int i = 0; i < max_tau; ++i) {
+        for (int e = 0; e < p.E; ++e) {
+            if (s_off[e + 1] - s_off[e] <= i)
+                continue;
+            if (pos++ % gridDim.x != blockIdx.x)
+                continue;
+            const int tile = s_off[e] + i;
+            if (threadIdx.x == 0)
+                s_go = wait_tile(p, tile);
+            __syncthreads();
+            if (s_go) {
+                const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+                for (int r = warp; r < p.B; r += kThreads / 32) {
+                    const int64_t row = (int64_t)tile * p.B + r;
+                    if (__ldg(p.pool_recv_token + row) < 0)
+                        continue;                        // padding: never read
+                    const uint4 *src = reinterpret_cast<const uint4 *>(p.src) + row * vecs;
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.dst) + row * vecs;
+                    for (int64_t v = lane; v < vecs; v += 32)
+                        dst[v] = __ldcg(src + v);
+                }
+            } else if (threadIdx.x == 0) {
+                atomicAdd(p.status + 1, 1u);
+            }
+            __syncthreads();
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_consume(const ConsumeParams &p, int num_ctas, cudaStream_t s)
+{
+    consume_tiles_kernel<<<num_ctas, kThreads, 0, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace sep

@@ -1,0 +1,274 @@
+// Dispatch permute: token rows into the expert-major pool.
+//
+// recv[src_pool_row[t, j]] = x[t] for every valid (t, j) (StreamEP README,
+// "Streaming dispatch in one paragraph": each landed (token, k) pair lands in
+// its pool slot; PR #769 "Description": the activation copy of the dispatch
+// epilogue).  Token-major: a warp reads its slice of x[t] once with 16-byte
+// loads and stores it to the token's k pool rows, so HBM sees the algorithmic
+// minimum (read T*H once, write N_a rows).  Padding rows are never touched.
+//
+// FP8 (DeepEP low-latency article, "FP8 and Quantization Support"; blog, "FP8
+// Dispatch 减少的是 payload"): a lane holds 16 channels, 8 lanes one 128-channel
+// group; amax by shuffles, one scale per group, codes from the hardware
+// e4m3x2 round-to-nearest-even satfinite conversion; each token is quantised
+// once and its codes written k times.
+//
+// Streaming (StreamEP README, same section): after its rows are stored, a
+// warp fences, then lane j atomically adds one arrival to the tile of row j
+// (acq_rel, gpu scope); the arrival that reaches the tile's target (valid rows
+// x warps per row) release-stores dispatch_seq into tile_ready[tile].
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "sep_internal.cuh"
+
+namespace sep {
+namespace {
+
+constexpr int kWarps = 8;
+
+__device__ __forceinline__ uint4 ld_stream(const uint4 *ptr)
+{
+    uint4 v;
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "l"(ptr));
+    return v;
+}
+
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned *ptr, unsigned v)
+{
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(ptr), "r"(v) : "memory");
+    return old;
+}
+
+__device__ __forceinline__ void st_release_gpu(unsigned *ptr, unsigned v)
+{
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+}
+
+// Publish the rows this warp just finished for token t (one arrival per row).
+__device__ __forceinline__ void publish_rows(const DispatchParams &p, int my_row, int lane)
+{
+    __threadfence();
+    __syncwarp();
+    if (lane < p.k && my_row >= 0) {
+        const int tile = my_row / p.B;
+        const unsigned need = (unsigned)p.pool_arrival_target[tile] * (unsigned)p.segs;
+        const unsigned old = atom_add_acq_rel_gpu(p.pool_arrival_count + tile, 1u);
+        if (old + 1u == need)
+            st_release_gpu(p.tile_ready + tile, p.seq);
+    }
+}
+
+// bf16: a work item is (token, segment of seg_len 16-byte vectors).
+template <int UNROLL, bool PUBLISH>
+__global__ void __launch_bounds__(kWarps * 32) dispatch_bf16_kernel(DispatchParams p)
+{
+    const int lane = threadIdx.x & 31;
+    const int V = p.H / 8;
+    const int64_t items = p.T * p.segs;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t it = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items; it += nwarps) {
+        const int64_t t = it / p.segs;
+        const int s = (int)(it - t * p.segs);
+        const int v_begin = s * p.seg_len;
+        const int v_end = min(V, v_begin + p.seg_len);
+        const int my_row = lane < p.k ? __ldg(p.src_pool_row + t * p.k + lane) : -1;
+        const uint4 *src = static_cast<const uint4 *>(p.x) + t * V;
+        for (int v0 = v_begin; v0 < v_end; v0 += 32 * UNROLL) {
+            uint4 buf[UNROLL];
+#pragma unroll
+            for (int u = 0; u < UNROLL; ++u) {
+                const int v = v0 + u * 32 + lane;
+                buf[u] = v < v_end ? ld_stream(src + v) : make_uint4(0, 0, 0, 0);
+            }
+            for (int j = 0; j < p.k; ++j) {
+                const int row = __shfl_sync(kFullMask, my_row, j);
+                if (row < 0)
+                    continue;                            // warp-uniform
+                uint4 *dst = static_cast<uint4 *>(p.recv) + (int64_t)row * V;
+#pragma unroll
+                for (int u = 0; u < UNROLL; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v < v_end)
+                        dst[v] = buf[u];
+                }
+            }
+        }
+        if (PUBLISH)
+            publish_rows(p, my_row, lane);
+    }
+}
+
+// Smallest E with 448 * 2^E >= amax (0 for amax == 0), clamped to [-127, 127].
+// amax = m * 2^x with m in [1, 2): 448 = 1.75 * 2^8, so E = x - 8 when
+// m <= 1.75 (mantissa field <= 0x600000) and x - 7 otherwise.  Every subnormal
+// amax is below 448 * 2^-134 and clamps to -127.
+__device__ __forceinline__ int ue8m0_exponent(float amax)
+{
+    const uint32_t u = __float_as_uint(amax);
+    if (u == 0u)
+        return 0;
+    const int ex = (int)(u >> 23);
+    if (ex == 0)
+        return -127;
+    const int e = ex - 127 - 8 + ((u & 0x7fffffu) > 0x600000u ? 1 : 0);
+    return e < -127 ? -127 : (e > 127 ? 127 : e);
+}
+
+// 2^e as fp32 for e in [-127, 127] (2^-127 is subnormal).
+__device__ __forceinline__ float exp2_int(int e)
+{
+    return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float *f)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+// fp8: a work item is (token, segment of seg_len 512-channel iterations).
+template <int SCALE, bool PUBLISH>
+__global__ void __launch_bounds__(kWarps * 32) dispatch_fp8_kernel(DispatchParams p)
+{
+    const int lane = threadIdx.x & 31;
+    const int H = p.H;
+    const int G = H / 128;
+    const int iters = (H + 511) / 512;
+    const int64_t items = p.T * p.segs;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t it = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items; it += nwarps) {
+        const int64_t t = it / p.segs;
+        const int s = (int)(it - t * p.segs);
+        const int i_begin = s * p.seg_len;
+        const int i_end = min(iters, i_begin + p.seg_len);
+        const int my_row = lane < p.k ? __ldg(p.src_pool_row + t * p.k + lane) : -1;
+        const __nv_bfloat16 *xrow = static_cast<const __nv_bfloat16 *>(p.x) + t * H;
+        for (int i = i_begin; i < i_end; ++i) {
+            const int c0 = i * 512 + lane * 16;          // H % 128 == 0: whole groups are in or out
+            const bool active = c0 < H;
+            float f[16];
+            if (active) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(xrow + c0);
+                bf16x8_to_f32(ld_stream(src), f);
+                bf16x8_to_f32(ld_stream(src + 1), f + 8);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 16; ++q)
+                    f[q] = 0.f;
+            }
+            float amax = 0.f;
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+                amax = fmaxf(amax, fabsf(f[q]));
+            amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 1));
+            amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 2));
+            amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 4));
+
+            float scale_f = 1.f, inv = 1.f;
+            int expo = 0;
+            if (SCALE == SEP_SCALE_F32) {
+                scale_f = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
+            } else {
+                expo = ue8m0_exponent(amax);
+                scale_f = exp2_int(expo);
+                inv = exp2_int(-expo);                    // exact: x * 2^-E == x / 2^E
+            }
+            uint32_t packed[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float a[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+                    a[r] = SCALE == SEP_SCALE_F32 ? __fdiv_rn(f[4 * q + r], scale_f)
+                                                  : __fmul_rn(f[4 * q + r], inv);
+                const __nv_fp8x2_storage_t lo =
+                    __nv_cvt_float2_to_fp8x2(make_float2(a[0], a[1]), __NV_SATFINITE, __NV_E4M3);
+                const __nv_fp8x2_storage_t hi =
+                    __nv_cvt_float2_to_fp8x2(make_float2(a[2], a[3]), __NV_SATFINITE, __NV_E4M3);
+                packed[q] = (uint32_t)lo | ((uint32_t)hi << 16);
+            }
+            const uint4 codes = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            const int g = c0 / 128;
+            for (int j = 0; j < p.k; ++j) {
+                const int row = __shfl_sync(kFullMask, my_row, j);
+                if (row < 0)
+                    continue;                            // warp-uniform
+                if (active) {
+                    uint8_t *dst = static_cast<uint8_t *>(p.recv) + (int64_t)row * H + c0;
+                    *reinterpret_cast<uint4 *>(dst) = codes;
+                    if ((lane & 7) == 0) {
+                        if (SCALE == SEP_SCALE_UE8M0)
+                            static_cast<uint8_t *>(p.recv_scales)[(int64_t)row * G + g] = (uint8_t)(expo + 127);
+                        else
+                            static_cast<float *>(p.recv_scales)[(int64_t)row * G + g] = scale_f;
+                    }
+                }
+            }
+        }
+        if (PUBLISH)
+            publish_rows(p, my_row, lane);
+    }
+}
+
+template <typename K>
+int blocks_for(K kernel, int64_t items, int num_sms)
+{
+    const int per_sm = occupancy_blocks_per_sm(reinterpret_cast<const void *>(kernel), kWarps * 32, 0);
+    const int64_t want = (items + kWarps - 1) / kWarps;
+    const int64_t cap = (int64_t)num_sms * per_sm;
+    return (int)(want < cap ? want : cap);
+}
+
+template <bool PUBLISH>
+cudaError_t launch_fp8(const DispatchParams &p, cudaStream_t s, int num_sms)
+{
+    const int64_t items = p.T * p.segs;
+    switch (p.scale) {
+    case SEP_SCALE_F32: {
+        auto k = dispatch_fp8_kernel<SEP_SCALE_F32, PUBLISH>;
+        k<<<blocks_for(k, items, num_sms), kWarps * 32, 0, s>>>(p);
+        break;
+    }
+    case SEP_SCALE_UE8M0: {
+        auto k = dispatch_fp8_kernel<SEP_SCALE_UE8M0, PUBLISH>;
+        k<<<blocks_for(k, items, num_sms), kWarps * 32, 0, s>>>(p);
+        break;
+    }
+    default: {
+        auto k = dispatch_fp8_kernel<SEP_SCALE_F32_POW2, PUBLISH>;
+        k<<<blocks_for(k, items, num_sms), kWarps * 32, 0, s>>>(p);
+        break;
+    }
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const DispatchParams &p, int payload, cudaStream_t s, int num_sms)
+{
+    const int64_t items = p.T * p.segs;
+    if (items == 0)
+        return cudaSuccess;
+    if (payload == SEP_PAYLOAD_BF16) {
+        if (p.tile_ready != nullptr) {
+            auto k = dispatch_bf16_kernel<4, true>;
+            k<<<blocks_for(k, items, num_sms), kWarps * 32, 0, s>>>(p);
+        } else {
+            auto k = dispatch_bf16_kernel<4, false>;
+            k<<<blocks_for(k, items, num_sms), kWarps * 32, 0, s>>>(p);
+        }
+        return cudaGetLastError();
+    }
+    return p.tile_ready != nullptr ? launch_fp8<true>(p, s, num_sms) : launch_fp8<false>(p, s, num_sms);
+}
+
+}  // namespace sep

@@ -1,0 +1,606 @@
+// Host side of the sep C ABI: argument validation, handle storage, launches.
+//
+// Every check happens on the host before anything is enqueued (PR #769,
+// "Description": unsupported modes are rejected up front), capacity is checked
+// against the worst case or the synced exact size so rows are never silently
+// dropped ("DeepEP MoE dispatch/combine" blog, "Imbalance 决定 buffer 与尾延迟"),
+// and a handle carries the epoch of its routing so a combine against a
+// re-laid-out handle is refused (blog, "EPHandle" and "集成时的数据契约").
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "sep_internal.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+sep_status fail(sep_status st, const char *fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+sep_status cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(SEP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr int64_t kMaxRows = (1LL << 31) - 1;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Worst-case pool rows for Na assignments: every used expert pads < B rows.
+int64_t worst_pool_rows(int64_t Na, int E, int B)
+{
+    const int64_t used = Na < E ? Na : E;
+    const int64_t rows = Na + used * (B - 1);
+    return (rows + B - 1) / B * B;
+}
+
+sep_status check_dims(int64_t T, int k, int E, int R, int B)
+{
+    if (T < 0)
+        return fail(SEP_ERR_INVALID_ARG, "num_tokens must be >= 0 (got %lld)", (long long)T);
+    if (k < 1 || k > 32)
+        return fail(SEP_ERR_INVALID_ARG, "top_k must be in 1..32 (got %d)", k);
+    if (E < 1 || E > 1024)
+        return fail(SEP_ERR_INVALID_ARG, "num_experts must be in 1..1024 (got %d)", E);
+    if (R < 1 || R > E || E % R != 0)
+        return fail(SEP_ERR_INVALID_ARG, "num_owners must divide num_experts (got %d, %d)", R, E);
+    if (B < 1 || B > 1024)
+        return fail(SEP_ERR_INVALID_ARG, "block_m must be in 1..1024 (got %d)", B);
+    if (T * k > kMaxRows || worst_pool_rows(T * k, E, B) > kMaxRows)
+        return fail(SEP_ERR_INVALID_ARG, "num_tokens * top_k too large for 32-bit pool rows");
+    return SEP_OK;
+}
+
+sep_status current_device(int *dev)
+{
+    const cudaError_t e = cudaGetDevice(dev);
+    return e == cudaSuccess ? SEP_OK : cuda_fail(e, "cudaGetDevice");
+}
+
+sep_status check_device(const sep_handle *h)
+{
+    int dev = -1;
+    sep_status st = current_device(&dev);
+    if (st != SEP_OK)
+        return st;
+    if (dev != h->device)
+        return fail(SEP_ERR_INVALID_ARG, "handle lives on device %d, current device is %d", h->device, dev);
+    return SEP_OK;
+}
+
+size_t carve(size_t *off, size_t bytes)
+{
+    const size_t at = *off;
+    *off = (at + bytes + 255) / 256 * 256;
+    return at;
+}
+
+sep_status create(int64_t T_cap, int k, int E, int R, int B, uint32_t flags, cudaStream_t s,
+                  sep_handle **out)
+{
+    sep_status st = check_dims(T_cap, k, E, R, B);
+    if (st != SEP_OK)
+        return st;
+    int dev = -1;
+    if ((st = current_device(&dev)) != SEP_OK)
+        return st;
+    sep_handle *h = new (std::nothrow) sep_handle();
+    if (h == nullptr)
+        return fail(SEP_ERR_CUDA, "out of host memory");
+    h->device = dev;
+    h->k = k;
+    h->E = E;
+    h->R = R;
+    h->B = B;
+    h->flags_cap = flags;
+    h->T_cap = T_cap;
+    h->Na_cap = T_cap * k;
+    h->P_cap = worst_pool_rows(h->Na_cap, E, B);
+    h->NT_cap = h->P_cap / B;
+    h->wchunk_cap = sep::layout_wchunk_capacity(h->Na_cap);
+    h->last_stream = s;
+
+    const int64_t P1 = h->P_cap > 0 ? h->P_cap : 1;
+    const int64_t NT1 = h->NT_cap > 0 ? h->NT_cap : 1;
+    const int64_t Na1 = h->Na_cap > 0 ? h->Na_cap : 1;
+    size_t off = 0;
+    const size_t o_sizes = carve(&off, 32);              // {P, NT} + bad_epoch, one copy to the host
+    const size_t o_ec = carve(&off, (size_t)E * 4);
+    const size_t o_oc = carve(&off, (size_t)R * 4);
+    const size_t o_otc = carve(&off, (size_t)R * 4);
+    const size_t o_off = carve(&off, (size_t)(E + 1) * 4);
+    const size_t o_roff = carve(&off, (size_t)(R + 1) * 4);
+    const size_t o_te = carve(&off, (size_t)NT1 * 4);
+    const size_t o_tg = carve(&off, (size_t)NT1 * 4);
+    const size_t o_ac = carve(&off, (size_t)NT1 * 4);
+    const size_t o_spr = carve(&off, (size_t)Na1 * 4);
+    const size_t o_tok = carve(&off, (size_t)P1 * 4);
+    const size_t o_slot = carve(&off, (size_t)P1 * 4);
+    const size_t o_hist = carve(&off, (size_t)h->wchunk_cap * E * 4);
+    const size_t o_base = carve(&off, (size_t)h->wchunk_cap * E * 4);
+    const size_t o_in = (flags & SEP_LAYOUT_TOKEN_IN_OWNER) ? carve(&off, (size_t)(T_cap > 0 ? T_cap : 1) * R) : 0;
+
+    cudaError_t e = cudaMallocAsync(&h->block, off, s);
+    if (e != cudaSuccess) {
+        delete h;
+        return cuda_fail(e, "cudaMallocAsync (handle storage)");
+    }
+    e = cudaMallocHost(reinterpret_cast<void **>(&h->host_mirror), 32);
+    if (e != cudaSuccess) {
+        cudaFreeAsync(h->block, s);
+        delete h;
+        return cuda_fail(e, "cudaMallocHost (handle mirror)");
+    }
+    char *b = static_cast<char *>(h->block);
+    h->sizes = reinterpret_cast<int64_t *>(b + o_sizes);
+    h->bad_epoch = reinterpret_cast<uint32_t *>(b + o_sizes + 16);
+    h->expert_counts = reinterpret_cast<int32_t *>(b + o_ec);
+    h->owner_counts = reinterpret_cast<int32_t *>(b + o_oc);
+    h->owner_token_counts = reinterpret_cast<int32_t *>(b + o_otc);
+    h->expert_pool_block_offset = reinterpret_cast<int32_t *>(b + o_off);
+    h->owner_pool_row_offset = reinterpret_cast<int32_t *>(b + o_roff);
+    h->tile_expert = reinterpret_cast<int32_t *>(b + o_te);
+    h->pool_arrival_target = reinterpret_cast<int32_t *>(b + o_tg);
+    h->pool_arrival_count = reinterpret_cast<uint32_t *>(b + o_ac);
+    h->src_pool_row = reinterpret_cast<int32_t *>(b + o_spr);
+    h->pool_recv_token = reinterpret_cast<int32_t *>(b + o_tok);
+    h->pool_recv_slot = reinterpret_cast<int32_t *>(b + o_slot);
+    h->wchunk_hist = reinterpret_cast<int32_t *>(b + o_hist);
+    h->wchunk_base = reinterpret_cast<int32_t *>(b + o_base);
+    h->is_token_in_rank = (flags & SEP_LAYOUT_TOKEN_IN_OWNER) ? reinterpret_cast<uint8_t *>(b + o_in) : nullptr;
+    e = cudaMemsetAsync(h->sizes, 0, 32, s);             // sizes and bad_epoch start at zero
+    if (e != cudaSuccess) {
+        cudaFreeAsync(h->block, s);
+        cudaFreeHost(h->host_mirror);
+        delete h;
+        return cuda_fail(e, "cudaMemsetAsync (handle)");
+    }
+    h->T = 0;
+    h->epoch = 0;
+    h->synced = 0;
+    h->P = h->NT = -1;
+    *out = h;
+    return SEP_OK;
+}
+
+// Rows a buffer must hold for the handle's current layout.
+int64_t needed_rows(const sep_handle *h)
+{
+    return h->synced ? h->P : worst_pool_rows(h->T * h->k, h->E, h->B);
+}
+
+}  // namespace
+
+namespace sep {
+
+int device_sm_count()
+{
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+int occupancy_blocks_per_sm(const void *kernel, int threads, size_t smem)
+{
+    struct Entry {
+        const void *kernel;
+        int threads;
+        int blocks;
+    };
+    static Entry cache[32];
+    static int used = 0;
+    for (int i = 0; i < used; ++i)
+        if (cache[i].kernel == kernel && cache[i].threads == threads)
+            return cache[i].blocks;
+    int b = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kernel, threads, smem) != cudaSuccess || b < 1)
+        b = 1;
+    if (used < 32)
+        cache[used++] = Entry{kernel, threads, b};
+    return b;
+}
+
+}  // namespace sep
+
+extern "C" {
+
+int sep_abi_version(void) { return SEP_ABI_VERSION; }
+
+const char *sep_last_error(void) { return g_err; }
+
+const char *sep_status_string(sep_status st)
+{
+    switch (st) {
+    case SEP_OK: return "SEP_OK";
+    case SEP_ERR_INVALID_ARG: return "SEP_ERR_INVALID_ARG";
+    case SEP_ERR_CAPACITY: return "SEP_ERR_CAPACITY";
+    case SEP_ERR_BAD_EXPERT_ID: return "SEP_ERR_BAD_EXPERT_ID";
+    case SEP_ERR_HANDLE_MISMATCH: return "SEP_ERR_HANDLE_MISMATCH";
+    case SEP_ERR_TIMEOUT: return "SEP_ERR_TIMEOUT";
+    case SEP_ERR_CUDA: return "SEP_ERR_CUDA";
+    }
+    return "SEP_ERR_UNKNOWN";
+}
+
+sep_status sep_handle_create(int64_t max_tokens, int top_k, int num_experts, int num_owners,
+                             int block_m, uint32_t flags, void *stream, sep_handle **handle)
+{
+    if (handle == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "handle out-pointer is NULL");
+    if (flags & ~(SEP_LAYOUT_SYNC_COUNTS | SEP_LAYOUT_TOKEN_IN_OWNER))
+        return fail(SEP_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+    return create(max_tokens, top_k, num_experts, num_owners, block_m, flags,
+                  static_cast<cudaStream_t>(stream), handle);
+}
+
+sep_status sep_layout(const void *topk_idx, int idx_bytes, int64_t num_tokens, int top_k,
+                      int num_experts, int num_owners, int block_m, uint32_t flags, void *stream,
+                      sep_handle **handle)
+{
+    if (handle == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "handle in/out pointer is NULL");
+    if (flags & ~(SEP_LAYOUT_SYNC_COUNTS | SEP_LAYOUT_TOKEN_IN_OWNER))
+        return fail(SEP_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+    if (idx_bytes != 4 && idx_bytes != 8)
+        return fail(SEP_ERR_INVALID_ARG, "idx_bytes must be 4 or 8 (got %d)", idx_bytes);
+    sep_status st = check_dims(num_tokens, top_k, num_experts, num_owners, block_m);
+    if (st != SEP_OK)
+        return st;
+    if (num_tokens > 0 && topk_idx == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "topk_idx is NULL");
+    if (topk_idx != nullptr && (reinterpret_cast<uintptr_t>(topk_idx) % idx_bytes) != 0)
+        return fail(SEP_ERR_INVALID_ARG, "topk_idx is not %d-byte aligned", idx_bytes);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    sep_handle *h = *handle;
+    if (h != nullptr) {
+        if ((st = check_device(h)) != SEP_OK)
+            return st;
+        if (h->k != top_k || h->E != num_experts || h->R != num_owners || h->B != block_m)
+            return fail(SEP_ERR_HANDLE_MISMATCH, "handle was made for k=%d E=%d R=%d B=%d", h->k, h->E, h->R, h->B);
+        if (num_tokens > h->T_cap)
+            return fail(SEP_ERR_HANDLE_MISMATCH, "handle holds at most %lld tokens (got %lld)",
+                        (long long)h->T_cap, (long long)num_tokens);
+        if ((flags & SEP_LAYOUT_TOKEN_IN_OWNER) && h->is_token_in_rank == nullptr)
+            return fail(SEP_ERR_HANDLE_MISMATCH, "handle was made without SEP_LAYOUT_TOKEN_IN_OWNER");
+    } else {
+        if ((st = create(num_tokens, top_k, num_experts, num_owners, block_m, flags, s, &h)) != SEP_OK)
+            return st;
+    }
+
+    h->T = num_tokens;
+    h->flags = flags;
+    h->arrivals_used = 0;                                // the assign kernel zeroes the counts
+    h->epoch += 1;
+    h->synced = 0;
+    h->P = h->NT = -1;
+    h->last_stream = s;
+
+    sep::LayoutParams p{};
+    p.topk_idx = topk_idx;
+    p.T = num_tokens;
+    p.k = top_k;
+    p.E = num_experts;
+    p.R = num_owners;
+    p.B = block_m;
+    p.Na = num_tokens * top_k;
+    p.rounds = sep::layout_rounds_for(p.Na);
+    p.num_wchunks = (int)sep::layout_wchunks_for(p.Na, p.rounds);
+    p.wchunk_hist = h->wchunk_hist;
+    p.wchunk_base = h->wchunk_base;
+    p.expert_counts = h->expert_counts;
+    p.owner_counts = h->owner_counts;
+    p.owner_token_counts = h->owner_token_counts;
+    p.is_token_in_rank = (flags & SEP_LAYOUT_TOKEN_IN_OWNER) ? h->is_token_in_rank : nullptr;
+    p.expert_pool_block_offset = h->expert_pool_block_offset;
+    p.owner_pool_row_offset = h->owner_pool_row_offset;
+    p.tile_expert = h->tile_expert;
+    p.pool_arrival_target = h->pool_arrival_target;
+    p.pool_arrival_count = h->pool_arrival_count;
+    p.src_pool_row = h->src_pool_row;
+    p.pool_recv_token = h->pool_recv_token;
+    p.pool_recv_slot = h->pool_recv_slot;
+    p.sizes = h->sizes;
+    p.bad_epoch = h->bad_epoch;
+    p.epoch = h->epoch;
+    if (p.num_wchunks > h->wchunk_cap)
+        return fail(SEP_ERR_CUDA, "internal: chunk table too small");
+    cudaError_t e = sep::launch_layout(p, idx_bytes, s);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "layout launch");
+    *handle = h;
+    if (flags & SEP_LAYOUT_SYNC_COUNTS)
+        return sep_handle_sync(h, stream);
+    return SEP_OK;
+}
+
+sep_status sep_handle_info(const sep_handle *h, sep_layout_info *info)
+{
+    if (h == nullptr || info == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "NULL handle or info");
+    std::memset(info, 0, sizeof *info);
+    info->num_tokens = h->T;
+    info->top_k = h->k;
+    info->num_experts = h->E;
+    info->num_owners = h->R;
+    info->block_m = h->B;
+    info->max_tokens = h->T_cap;
+    info->max_pool_rows = h->P_cap;
+    info->max_tiles = h->NT_cap;
+    info->num_pool_rows = h->synced ? h->P : -1;
+    info->num_tiles = h->synced ? h->NT : -1;
+    info->epoch = h->epoch;
+    info->flags = h->flags;
+    info->expert_counts = h->expert_counts;
+    info->owner_counts = h->owner_counts;
+    info->owner_token_counts = h->owner_token_counts;
+    info->is_token_in_rank = (h->flags & SEP_LAYOUT_TOKEN_IN_OWNER) ? h->is_token_in_rank : nullptr;
+    info->expert_pool_block_offset = h->expert_pool_block_offset;
+    info->owner_pool_row_offset = h->owner_pool_row_offset;
+    info->tile_expert = h->tile_expert;
+    info->pool_arrival_target = h->pool_arrival_target;
+    info->pool_arrival_count = h->pool_arrival_count;
+    info->src_pool_row = h->src_pool_row;
+    info->pool_recv_token = h->pool_recv_token;
+    info->pool_recv_slot = h->pool_recv_slot;
+    info->device_sizes = h->sizes;
+    return SEP_OK;
+}
+
+sep_status sep_handle_sync(sep_handle *h, void *stream)
+{
+    if (h == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "NULL handle");
+    sep_status st = check_device(h);
+    if (st != SEP_OK)
+        return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(h->host_mirror, h->sizes, 24, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaMemcpyAsync (sizes)");
+    if ((e = cudaStreamSynchronize(s)) != cudaSuccess)
+        return cuda_fail(e, "cudaStreamSynchronize");
+    h->P = h->host_mirror[0];
+    h->NT = h->host_mirror[1];
+    h->synced = 1;
+    uint32_t bad = 0;
+    std::memcpy(&bad, h->host_mirror + 2, sizeof bad);
+    if (bad != 0 && bad == h->epoch)
+        return fail(SEP_ERR_BAD_EXPERT_ID, "topk_idx holds an expert id >= num_experts (%d)", h->E);
+    return SEP_OK;
+}
+
+sep_status sep_dispatch(sep_handle *h, const void *x, int64_t hidden, int payload, int scale,
+                        void *recv_x, void *recv_scales, int64_t recv_capacity_rows,
+                        uint32_t *tile_ready, int64_t tile_ready_len, uint32_t dispatch_seq, void *stream)
+{
+    if (h == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "NULL handle");
+    sep_status st = check_device(h);
+    if (st != SEP_OK)
+        return st;
+    if (payload != SEP_PAYLOAD_BF16 && payload != SEP_PAYLOAD_FP8_E4M3)
+        return fail(SEP_ERR_INVALID_ARG, "unknown payload %d", payload);
+    const bool fp8 = payload == SEP_PAYLOAD_FP8_E4M3;
+    if (!fp8 && scale != SEP_SCALE_NONE)
+        return fail(SEP_ERR_INVALID_ARG, "bf16 payload takes SEP_SCALE_NONE");
+    if (fp8 && scale != SEP_SCALE_F32 && scale != SEP_SCALE_UE8M0 && scale != SEP_SCALE_F32_POW2)
+        return fail(SEP_ERR_INVALID_ARG, "FP8 payload needs a scale format (got %d)", scale);
+    if (hidden < 1 || hidden > 65536 || hidden % (fp8 ? 128 : 8) != 0)
+        return fail(SEP_ERR_INVALID_ARG, "hidden must be a multiple of %d in 1..65536 (got %lld)",
+                    fp8 ? 128 : 8, (long long)hidden);
+    if (h->T > 0 && (x == nullptr || recv_x == nullptr))
+        return fail(SEP_ERR_INVALID_ARG, "x or recv_x is NULL");
+    if (!aligned16(x) || !aligned16(recv_x))
+        return fail(SEP_ERR_INVALID_ARG, "x and recv_x must be 16-byte aligned");
+    if (fp8) {
+        if (h->T > 0 && recv_scales == nullptr)
+            return fail(SEP_ERR_INVALID_ARG, "recv_scales is NULL");
+        if (scale != SEP_SCALE_UE8M0 && (reinterpret_cast<uintptr_t>(recv_scales) & 3u))
+            return fail(SEP_ERR_INVALID_ARG, "fp32 recv_scales must be 4-byte aligned");
+    }
+    const int64_t need = needed_rows(h);
+    if (recv_capacity_rows < need)
+        return fail(SEP_ERR_CAPACITY, "recv_x holds %lld rows, the layout needs %lld%s",
+                    (long long)recv_capacity_rows, (long long)need,
+                    h->synced ? "" : " (worst case; sync the layout for the exact size)");
+    if (tile_ready != nullptr) {
+        if (dispatch_seq == 0)
+            return fail(SEP_ERR_INVALID_ARG, "dispatch_seq must be nonzero with tile_ready");
+        if ((reinterpret_cast<uintptr_t>(tile_ready) & 3u) != 0)
+            return fail(SEP_ERR_INVALID_ARG, "tile_ready must be 4-byte aligned");
+        if (tile_ready_len < need / h->B)
+            return fail(SEP_ERR_CAPACITY, "tile_ready holds %lld entries, the layout needs %lld",
+                        (long long)tile_ready_len, (long long)(need / h->B));
+        if (tile_ready == h->last_tile_ready && (int32_t)(dispatch_seq - h->last_seq) <= 0)
+            return fail(SEP_ERR_INVALID_ARG, "dispatch_seq %u does not advance past %u for this tile_ready",
+                        dispatch_seq, h->last_seq);
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    h->last_stream = s;
+    if (tile_ready != nullptr) {
+        h->last_tile_ready = tile_ready;
+        h->last_seq = dispatch_seq;
+    }
+    if (h->T == 0)
+        return SEP_OK;
+    if (tile_ready != nullptr) {
+        if (h->arrivals_used) {                          // a second streaming dispatch of this layout
+            cudaError_t e = cudaMemsetAsync(h->pool_arrival_count, 0, (size_t)(h->NT_cap > 0 ? h->NT_cap : 1) * 4, s);
+            if (e != cudaSuccess)
+                return cuda_fail(e, "cudaMemsetAsync (arrival counts)");
+        }
+        h->arrivals_used = 1;
+    }
+
+    const int num_sms = sep::device_sm_count();
+    sep::DispatchParams p{};
+    p.x = x;
+    p.T = h->T;
+    p.H = (int)hidden;
+    p.k = h->k;
+    p.B = h->B;
+    p.src_pool_row = h->src_pool_row;
+    p.recv = recv_x;
+    p.recv_scales = recv_scales;
+    p.scale = scale;
+    p.tile_ready = tile_ready;
+    p.pool_arrival_count = h->pool_arrival_count;
+    p.pool_arrival_target = h->pool_arrival_target;
+    p.seq = dispatch_seq;
+    // split a token row over several warps when there are too few tokens to fill the GPU
+    const int64_t units = fp8 ? (hidden + 511) / 512 : ((hidden / 8) + 31) / 32;   // warp-steps per row
+    const int64_t want_warps = (int64_t)num_sms * 32;
+    int64_t segs = (want_warps + h->T - 1) / h->T;
+    if (segs > units)
+        segs = units;
+    if (segs < 1)
+        segs = 1;
+    const int64_t steps = (units + segs - 1) / segs;
+    p.seg_len = (int)(fp8 ? steps : steps * 32);
+    p.segs = (int)((units + steps - 1) / steps);
+    cudaError_t e = sep::launch_dispatch(p, payload, s, num_sms);
+    return e == cudaSuccess ? SEP_OK : cuda_fail(e, "dispatch launch");
+}
+
+sep_status sep_combine(const sep_handle *h, uint32_t layout_epoch, const void *y_pool, int64_t hidden,
+                       int64_t y_capacity_rows, const float *topk_weight, void *out, void *stream)
+{
+    if (h == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "NULL handle");
+    sep_status st = check_device(h);
+    if (st != SEP_OK)
+        return st;
+    if (layout_epoch != h->epoch)
+        return fail(SEP_ERR_HANDLE_MISMATCH, "handle epoch is %u, caller's routing has epoch %u",
+                    h->epoch, layout_epoch);
+    if (hidden < 1 || hidden > 65536 || hidden % 8 != 0)
+        return fail(SEP_ERR_INVALID_ARG, "hidden must be a multiple of 8 in 1..65536 (got %lld)",
+                    (long long)hidden);
+    if (h->T > 0 && (y_pool == nullptr || topk_weight == nullptr || out == nullptr))
+        return fail(SEP_ERR_INVALID_ARG, "y_pool, topk_weight or out is NULL");
+    if (!aligned16(y_pool) || !aligned16(out))
+        return fail(SEP_ERR_INVALID_ARG, "y_pool and out must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(topk_weight) & 3u) != 0)
+        return fail(SEP_ERR_INVALID_ARG, "topk_weight must be 4-byte aligned");
+    const int64_t need = needed_rows(h);
+    if (y_capacity_rows < need)
+        return fail(SEP_ERR_CAPACITY, "y_pool holds %lld rows, the layout needs %lld",
+                    (long long)y_capacity_rows, (long long)need);
+    if (h->T == 0)
+        return SEP_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const_cast<sep_handle *>(h)->last_stream = s;
+
+    const int num_sms = sep::device_sm_count();
+    sep::CombineParams p{};
+    p.y = y_pool;
+    p.T = h->T;
+    p.H = (int)hidden;
+    p.k = h->k;
+    p.src_pool_row = h->src_pool_row;
+    p.w = topk_weight;
+    p.out = out;
+    const int64_t units = ((hidden / 8) + 31) / 32;
+    const int64_t want_warps = (int64_t)num_sms * 32;
+    int64_t segs = (want_warps + h->T - 1) / h->T;
+    if (segs > units)
+        segs = units;
+    if (segs < 1)
+        segs = 1;
+    const int64_t steps = (units + segs - 1) / segs;
+    p.seg_len = (int)(steps * 32);
+    p.segs = (int)((units + steps - 1) / steps);
+    cudaError_t e = sep::launch_combine(p, s, num_sms);
+    return e == cudaSuccess ? SEP_OK : cuda_fail(e, "combine launch");
+}
+
+sep_status sep_consume_tiles(const sep_handle *h, const void *recv_x, int64_t row_bytes,
+                             int64_t capacity_rows, const uint32_t *tile_ready, int64_t tile_ready_len,
+                             uint32_t dispatch_seq, void *dst, int num_ctas, uint64_t timeout_ns,
+                             uint32_t *status, void *stream)
+{
+    if (h == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "NULL handle");
+    sep_status st = check_device(h);
+    if (st != SEP_OK)
+        return st;
+    if (tile_ready == nullptr || status == nullptr || (h->T > 0 && (recv_x == nullptr || dst == nullptr)))
+        return fail(SEP_ERR_INVALID_ARG, "NULL tile_ready, status, recv_x or dst");
+    if (row_bytes < 16 || row_bytes % 16 != 0 || row_bytes > (1LL << 20))
+        return fail(SEP_ERR_INVALID_ARG, "row_bytes must be a multiple of 16 in 16..2^20");
+    if (!aligned16(recv_x) || !aligned16(dst))
+        return fail(SEP_ERR_INVALID_ARG, "recv_x and dst must be 16-byte aligned");
+    if (((reinterpret_cast<uintptr_t>(tile_ready) | reinterpret_cast<uintptr_t>(status)) & 3u) != 0)
+        return fail(SEP_ERR_INVALID_ARG, "tile_ready and status must be 4-byte aligned");
+    if (dispatch_seq == 0)
+        return fail(SEP_ERR_INVALID_ARG, "dispatch_seq must be nonzero");
+    if (num_ctas < 1 || num_ctas > 1024)
+        return fail(SEP_ERR_INVALID_ARG, "num_ctas must be in 1..1024");
+    const int64_t need = needed_rows(h);
+    if (capacity_rows < need)
+        return fail(SEP_ERR_CAPACITY, "recv_x/dst hold %lld rows, the layout needs %lld",
+                    (long long)capacity_rows, (long long)need);
+    if (tile_ready_len < need / h->B)
+        return fail(SEP_ERR_CAPACITY, "tile_ready holds %lld entries, the layout needs %lld",
+                    (long long)tile_ready_len, (long long)(need / h->B));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(status, 0, 2 * sizeof(uint32_t), s);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaMemsetAsync (status)");
+    if (h->T == 0)
+        return SEP_OK;
+    sep::ConsumeParams p{};
+    p.src = static_cast<const uint8_t *>(recv_x);
+    p.dst = static_cast<uint8_t *>(dst);
+    p.row_bytes = row_bytes;
+    p.E = h->E;
+    p.B = h->B;
+    p.expert_pool_block_offset = h->expert_pool_block_offset;
+    p.pool_recv_token = h->pool_recv_token;
+    p.tile_ready = tile_ready;
+    p.seq = dispatch_seq;
+    p.timeout_ns = timeout_ns ? timeout_ns : 1000000000ull;
+    const uint64_t polls = p.timeout_ns / 128 + 1024;
+    p.max_polls = polls > 0xffffffffull ? 0xffffffffu : (uint32_t)polls;
+    p.status = status;
+    p.abort_flag = status;
+    e = sep::launch_consume(p, num_ctas, s);
+    return e == cudaSuccess ? SEP_OK : cuda_fail(e, "consumer launch");
+}
+
+void sep_handle_free(sep_handle *h)
+{
+    if (h == nullptr)
+        return;
+    int prev = -1;
+    const bool switched = cudaGetDevice(&prev) == cudaSuccess && prev != h->device &&
+                          cudaSetDevice(h->device) == cudaSuccess;
+    if (h->block != nullptr)
+        cudaFreeAsync(h->block, h->last_stream);
+    if (h->host_mirror != nullptr)
+        cudaFreeHost(h->host_mirror);
+    if (switched)
+        cudaSetDevice(prev);
+    delete h;
+}
+
+}  // extern "C"

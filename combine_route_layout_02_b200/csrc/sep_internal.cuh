@@ -1,0 +1,142 @@
+// Internal declarations of the sep library (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sep.h"
+
+namespace sep {
+
+constexpr unsigned kFullMask = 0xffffffffu;
+
+// ----------------------------------------------------------------- layout
+
+// Per-warp chunks of the assignment stream: warp w of the count / assign
+// kernels owns assignments [w * 32 * rounds, (w + 1) * 32 * rounds).
+struct LayoutParams {
+    const void *topk_idx;
+    int64_t T;
+    int k, E, R, B;
+    int64_t Na;                      // T * k
+    int rounds;                      // 32-entry rounds per warp chunk
+    int num_wchunks;
+    int32_t *wchunk_hist;            // [E][num_wchunks] counts per (expert, chunk)
+    int32_t *wchunk_base;            // [E][num_wchunks] exclusive prefix over chunks
+    int32_t *expert_counts;          // [E]
+    int32_t *owner_counts;           // [R]
+    int32_t *owner_token_counts;     // [R]
+    uint8_t *is_token_in_rank;       // [T][R] or nullptr
+    int32_t *expert_pool_block_offset;  // [E+1]
+    int32_t *owner_pool_row_offset;  // [R+1]
+    int32_t *tile_expert;            // [NT_cap]
+    int32_t *pool_arrival_target;    // [NT_cap]
+    uint32_t *pool_arrival_count;    // [NT_cap]
+    int32_t *src_pool_row;           // [Na]
+    int32_t *pool_recv_token;        // [P_cap]
+    int32_t *pool_recv_slot;         // [P_cap]
+    int64_t *sizes;                  // [2] = {P, NT}
+    uint32_t *bad_epoch;             // last epoch that met an id >= E
+    uint32_t epoch;
+};
+
+int layout_rounds_for(int64_t Na);
+int64_t layout_wchunks_for(int64_t Na, int rounds);
+int64_t layout_wchunk_capacity(int64_t Na_cap);
+cudaError_t launch_layout(const LayoutParams &p, int idx_bytes, cudaStream_t s);
+
+// --------------------------------------------------------------- dispatch
+
+struct DispatchParams {
+    const void *x;                   // bf16 [T][H]
+    int64_t T;
+    int H, k, B;
+    const int32_t *src_pool_row;     // [T][k]
+    void *recv;                      // [rows][H] bf16 or e4m3
+    void *recv_scales;               // [rows][H/128] f32 or u8
+    int scale;                       // sep_scale
+    int segs;                        // warps sharing one token row
+    int seg_len;                     // per warp: 16-byte vectors (bf16) or 512-channel steps (fp8)
+    // streaming publication (tile_ready != nullptr)
+    uint32_t *tile_ready;
+    uint32_t *pool_arrival_count;
+    const int32_t *pool_arrival_target;
+    uint32_t seq;
+};
+
+cudaError_t launch_dispatch(const DispatchParams &p, int payload, cudaStream_t s, int num_sms);
+
+// ---------------------------------------------------------------- combine
+
+struct CombineParams {
+    const void *y;                   // bf16 [rows][H]
+    int64_t T;
+    int H, k;
+    const int32_t *src_pool_row;     // [T][k]
+    const float *w;                  // [T][k]
+    void *out;                       // bf16 [T][H]
+    int segs;                        // warps sharing one token row
+    int seg_len;                     // 16-byte vectors per warp
+};
+
+cudaError_t launch_combine(const CombineParams &p, cudaStream_t s, int num_sms);
+
+// --------------------------------------------------------------- consumer
+
+struct ConsumeParams {
+    const uint8_t *src;
+    uint8_t *dst;
+    int64_t row_bytes;
+    int E, B;
+    const int32_t *expert_pool_block_offset;   // [E+1]
+    const int32_t *pool_recv_token;
+    const uint32_t *tile_ready;
+    uint32_t seq;
+    uint64_t timeout_ns;
+    uint32_t max_polls;
+    uint32_t *status;                // [2]: code, tiles not copied
+    uint32_t *abort_flag;            // = &status[0]
+};
+
+cudaError_t launch_consume(const ConsumeParams &p, int num_ctas, cudaStream_t s);
+
+// ------------------------------------------------------------------ utils
+
+int device_sm_count();
+
+// Resident CTAs per SM for a kernel at a block size (cached per kernel).
+int occupancy_blocks_per_sm(const void *kernel, int threads, size_t smem);
+
+}  // namespace sep
+
+// Library-owned state behind the opaque handle.
+struct sep_handle {
+    int device;
+    int k, E, R, B;
+    uint32_t flags_cap;              // flags the storage was sized for
+    int64_t T_cap, Na_cap, P_cap, NT_cap, wchunk_cap;
+    // current layout
+    int64_t T;
+    uint32_t flags;
+    uint32_t epoch;
+    int synced;
+    int64_t P, NT;
+    // streaming-dispatch guard
+    const uint32_t *last_tile_ready;
+    uint32_t last_seq;
+    int arrivals_used;               // a streaming dispatch ran since the layout reset the counts
+    cudaStream_t last_stream;
+    // device storage: one block, carved
+    void *block;
+    int32_t *expert_counts, *owner_counts, *owner_token_counts;
+    int32_t *expert_pool_block_offset, *owner_pool_row_offset;
+    int32_t *tile_expert, *pool_arrival_target;
+    uint32_t *pool_arrival_count;
+    int32_t *src_pool_row, *pool_recv_token, *pool_recv_slot;
+    int32_t *wchunk_hist, *wchunk_base;
+    uint8_t *is_token_in_rank;
+    int64_t *sizes;
+    uint32_t *bad_epoch;
+    // pinned host mirror of {P, NT, bad_epoch}
+    int64_t *host_mirror;
+};

@@ -1,0 +1,247 @@
+"""Thin ctypes binding of the sep C ABI (include/sep.h).
+
+Argument marshalling only: every step of layout, dispatch and combine runs in
+the CUDA kernels of ``libsep.so``.  PyTorch supplies device memory and streams.
+Each function has the name of the C entry point it calls.  There is no CPU
+path: if the library cannot be loaded, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from dataclasses import dataclass
+
+import torch
+
+from . import build as _build
+
+SEP_OK, SEP_ERR_INVALID_ARG, SEP_ERR_CAPACITY, SEP_ERR_BAD_EXPERT_ID = 0, 1, 2, 3
+SEP_ERR_HANDLE_MISMATCH, SEP_ERR_TIMEOUT, SEP_ERR_CUDA = 4, 5, 6
+SEP_PAYLOAD_BF16, SEP_PAYLOAD_FP8_E4M3 = 0, 1
+SEP_SCALE_NONE, SEP_SCALE_F32, SEP_SCALE_UE8M0, SEP_SCALE_F32_POW2 = 0, 1, 2, 3
+SEP_LAYOUT_SYNC_COUNTS, SEP_LAYOUT_TOKEN_IN_OWNER = 0x1, 0x2
+
+PAYLOADS = {"bf16": SEP_PAYLOAD_BF16, "fp8": SEP_PAYLOAD_FP8_E4M3}
+SCALES = {"none": SEP_SCALE_NONE, "f32": SEP_SCALE_F32, "ue8m0": SEP_SCALE_UE8M0,
+          "f32_pow2": SEP_SCALE_F32_POW2}
+
+_P = ctypes.c_void_p
+_i32, _i64, _u32, _u64 = ctypes.c_int, ctypes.c_int64, ctypes.c_uint32, ctypes.c_uint64
+
+
+class LayoutInfo(ctypes.Structure):
+    """Mirror of sep_layout_info."""
+    _fields_ = [
+        ("num_tokens", _i64), ("top_k", ctypes.c_int32), ("num_experts", ctypes.c_int32),
+        ("num_owners", ctypes.c_int32), ("block_m", ctypes.c_int32), ("max_tokens", _i64),
+        ("max_pool_rows", _i64), ("max_tiles", _i64), ("num_pool_rows", _i64), ("num_tiles", _i64),
+        ("epoch", _u32), ("flags", _u32),
+        ("expert_counts", _P), ("owner_counts", _P), ("owner_token_counts", _P),
+        ("is_token_in_rank", _P), ("expert_pool_block_offset", _P), ("owner_pool_row_offset", _P),
+        ("tile_expert", _P), ("pool_arrival_target", _P), ("pool_arrival_count", _P),
+        ("src_pool_row", _P), ("pool_recv_token", _P), ("pool_recv_slot", _P), ("device_sizes", _P),
+    ]
+
+
+# (name, restype, argtypes) of every entry point declared in include/sep.h
+_SIGNATURES = [
+    ("sep_layout", _i32, [_P, _i32, _i64, _i32, _i32, _i32, _i32, _u32, _P, ctypes.POINTER(_P)]),
+    ("sep_handle_create", _i32, [_i64, _i32, _i32, _i32, _i32, _u32, _P, ctypes.POINTER(_P)]),
+    ("sep_handle_info", _i32, [_P, ctypes.POINTER(LayoutInfo)]),
+    ("sep_handle_sync", _i32, [_P, _P]),
+    ("sep_dispatch", _i32, [_P, _P, _i64, _i32, _i32, _P, _P, _i64, _P, _i64, _u32, _P]),
+    ("sep_combine", _i32, [_P, _u32, _P, _i64, _i64, _P, _P, _P]),
+    ("sep_consume_tiles", _i32, [_P, _P, _i64, _i64, _P, _i64, _u32, _P, _i32, _u64, _P, _P]),
+    ("sep_handle_free", None, [_P]),
+    ("sep_last_error", ctypes.c_char_p, []),
+    ("sep_status_string", ctypes.c_char_p, [_i32]),
+    ("sep_abi_version", _i32, []),
+]
+
+
+def _load() -> ctypes.CDLL:
+    path = _build.LIB
+    if not os.path.exists(path):
+        _build.build()
+    lib = ctypes.CDLL(path)
+    for name, res, args in _SIGNATURES:
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def declared_entry_points(header: str | None = None) -> list[str]:
+    """Entry-point names declared in include/sep.h."""
+    header = header or os.path.join(_build.INCLUDE, "sep.h")
+    text = open(header).read()
+    return sorted(set(re.findall(r"^SEP_API\s+[^;(]*?\b(sep_\w+)\s*\(", text, flags=re.M)))
+
+
+class SepError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = _lib.sep_last_error().decode(errors="replace")
+        name = _lib.sep_status_string(status).decode()
+        super().__init__(f"{where}: {name}: {msg}")
+        self.status = status
+
+
+def _check(status: int, where: str) -> None:
+    if status != SEP_OK:
+        raise SepError(status, where)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    if t is None:
+        return ctypes.c_void_p(None)
+    if not t.is_cuda:
+        raise ValueError("sep takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("sep takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+class _DeviceArray:
+    """A raw device array seen by torch through __cuda_array_interface__."""
+
+    def __init__(self, ptr: int, shape, typestr: str):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr,
+                                         "data": (ptr, True), "version": 3, "strides": None}
+
+
+@dataclass
+class Handle:
+    """Owns one sep_handle*; free it with sep_handle_free (or close())."""
+    ptr: ctypes.c_void_p
+
+    def info(self) -> LayoutInfo:
+        info = LayoutInfo()
+        _check(_lib.sep_handle_info(self.ptr, ctypes.byref(info)), "sep_handle_info")
+        return info
+
+    @property
+    def epoch(self) -> int:
+        return self.info().epoch
+
+    def view(self, name: str) -> torch.Tensor:
+        """Copy of one of the handle's device arrays (current layout only)."""
+        info = self.info()
+        T, k, E, R = info.num_tokens, info.top_k, info.num_experts, info.num_owners
+        shapes = {
+            "expert_counts": ((E,), "<i4"), "owner_counts": ((R,), "<i4"),
+            "owner_token_counts": ((R,), "<i4"), "is_token_in_rank": ((T, R), "|u1"),
+            "expert_pool_block_offset": ((E + 1,), "<i4"), "owner_pool_row_offset": ((R + 1,), "<i4"),
+            "tile_expert": ((info.max_tiles,), "<i4"), "pool_arrival_target": ((info.max_tiles,), "<i4"),
+            "pool_arrival_count": ((info.max_tiles,), "<i4"), "src_pool_row": ((T, k), "<i4"),
+            "pool_recv_token": ((info.max_pool_rows,), "<i4"),
+            "pool_recv_slot": ((info.max_pool_rows,), "<i4"), "device_sizes": ((2,), "<i8"),
+        }
+        shape, typestr = shapes[name]
+        ptr = getattr(info, name)
+        if ptr is None or 0 in shape:
+            dt = {"<i4": torch.int32, "|u1": torch.uint8, "<i8": torch.int64}[typestr]
+            return torch.zeros(shape, dtype=dt, device="cuda")
+        t = torch.as_tensor(_DeviceArray(ptr, shape, typestr), device="cuda")
+        return t.clone()
+
+    def close(self) -> None:
+        if self.ptr:
+            _lib.sep_handle_free(self.ptr)
+            self.ptr = ctypes.c_void_p(None)
+
+
+def sep_handle_create(max_tokens: int, top_k: int, num_experts: int, num_owners: int, block_m: int,
+                      flags: int = 0, stream=None) -> Handle:
+    out = ctypes.c_void_p(None)
+    _check(_lib.sep_handle_create(max_tokens, top_k, num_experts, num_owners, block_m, flags,
+                                  _stream(stream), ctypes.byref(out)), "sep_handle_create")
+    return Handle(out)
+
+
+def sep_layout(topk_idx: torch.Tensor, num_experts: int, num_owners: int, block_m: int,
+               flags: int = 0, handle: Handle | None = None, stream=None) -> Handle:
+    """Lay out a routing; reuses ``handle`` when given (its previous layout is invalidated)."""
+    if topk_idx.dtype not in (torch.int32, torch.int64) or topk_idx.dim() != 2:
+        raise ValueError("topk_idx must be a [T, k] int32 or int64 tensor")
+    T, k = topk_idx.shape
+    h = handle.ptr if handle is not None else ctypes.c_void_p(None)
+    _check(_lib.sep_layout(_ptr(topk_idx) if T else ctypes.c_void_p(None), topk_idx.element_size(),
+                           T, k, num_experts, num_owners, block_m, flags, _stream(stream),
+                           ctypes.byref(h)), "sep_layout")
+    if handle is not None:
+        handle.ptr = h
+        return handle
+    return Handle(h)
+
+
+def sep_handle_sync(handle: Handle, stream=None) -> None:
+    _check(_lib.sep_handle_sync(handle.ptr, _stream(stream)), "sep_handle_sync")
+
+
+def sep_dispatch(handle: Handle, x: torch.Tensor, recv_x: torch.Tensor, payload: str = "bf16",
+                 scale: str = "none", recv_scales: torch.Tensor | None = None,
+                 tile_ready: torch.Tensor | None = None, dispatch_seq: int = 0, stream=None) -> None:
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a [T, H] bf16 tensor")
+    _check(_lib.sep_dispatch(handle.ptr, _ptr(x), x.shape[1], PAYLOADS[payload], SCALES[scale],
+                             _ptr(recv_x), _ptr(recv_scales), recv_x.shape[0], _ptr(tile_ready),
+                             0 if tile_ready is None else tile_ready.numel(), dispatch_seq,
+                             _stream(stream)), "sep_dispatch")
+
+
+def sep_combine(handle: Handle, y_pool: torch.Tensor, topk_weight: torch.Tensor, out: torch.Tensor,
+                layout_epoch: int | None = None, stream=None) -> None:
+    if y_pool.dtype != torch.bfloat16 or out.dtype != torch.bfloat16 or topk_weight.dtype != torch.float32:
+        raise ValueError("y_pool/out must be bf16 and topk_weight fp32")
+    epoch = handle.epoch if layout_epoch is None else layout_epoch
+    _check(_lib.sep_combine(handle.ptr, epoch, _ptr(y_pool), y_pool.shape[1], y_pool.shape[0],
+                            _ptr(topk_weight), _ptr(out), _stream(stream)), "sep_combine")
+
+
+def sep_consume_tiles(handle: Handle, recv_x: torch.Tensor, tile_ready: torch.Tensor, dispatch_seq: int,
+                      dst: torch.Tensor, status: torch.Tensor, num_ctas: int = 16, timeout_ns: int = 0,
+                      stream=None) -> None:
+    row_bytes = recv_x.shape[1] * recv_x.element_size()
+    if dst.shape[0] < recv_x.shape[0] or dst.shape[1] * dst.element_size() != row_bytes:
+        raise ValueError("dst must have recv_x's row size and at least its rows")
+    if status.numel() < 2 or status.element_size() != 4:
+        raise ValueError("status must hold two 32-bit words")
+    _check(_lib.sep_consume_tiles(handle.ptr, _ptr(recv_x), row_bytes, recv_x.shape[0], _ptr(tile_ready),
+                                  tile_ready.numel(), dispatch_seq, _ptr(dst), num_ctas, timeout_ns,
+                                  _ptr(status), _stream(stream)), "sep_consume_tiles")
+
+
+def sep_handle_free(handle: Handle) -> None:
+    handle.close()
+
+
+def alloc_pool(handle: Handle, hidden: int, payload: str = "bf16", scale: str = "none",
+               rows: int | None = None):
+    """Device buffers for a dispatch: recv_x [rows, H] and, for FP8, recv_scales [rows, H/128]."""
+    info = handle.info()
+    if rows is None:
+        rows = info.num_pool_rows if info.num_pool_rows >= 0 else info.max_pool_rows
+    rows = max(int(rows), 1)
+    if payload == "bf16":
+        return torch.empty(rows, hidden, dtype=torch.bfloat16, device="cuda"), None
+    recv = torch.empty(rows, hidden, dtype=torch.uint8, device="cuda")
+    sdt = torch.uint8 if scale == "ue8m0" else torch.float32
+    return recv, torch.empty(rows, hidden // 128, dtype=sdt, device="cuda")

@@ -1,0 +1,277 @@
+/*
+ * sep.h — single-GPU MoE expert-parallel dispatch + combine for B200 (sm_100a).
+ *
+ * C ABI.  Plain pointers and sizes only; every device pointer is CUDA global
+ * memory on the current device, every stream argument is a cudaStream_t passed
+ * as void* (NULL = the legacy default stream).  All calls are stream-ordered:
+ * they validate their arguments on the host, enqueue kernels and return before
+ * the GPU has finished ("DeepEP MoE dispatch/combine" blog, section
+ * "EventOverlap": an asynchronous return does not mean the data is ready).
+ * Nothing here synchronises the device unless a flag below says so.
+ *
+ * The operation ("DeepEP MoE dispatch/combine" blog, "一轮 DeepEP 数据流" — one
+ * round of data flow):
+ *   inputs   x [T, H], topk_idx [T, k], topk_weight [T, k], num_experts E;
+ *   dispatch counts assignments per expert, computes the layout and offsets,
+ *            and moves the hidden states into recv_x grouped by expert;
+ *   combine  restores source token / top-k slot and reduces the
+ *            routing-weighted expert outputs back into token order.
+ * The receive buffer is the StreamEP pool ("StreamEP" README, "Streaming
+ * dispatch in one paragraph"): expert-major and BLOCK_M-padded, expert e's
+ * block starting at row expert_pool_block_offset[e] * BLOCK_M; each slot
+ * belongs to one expert and one BLOCK_M tile; padding rows have
+ * pool_recv_token < 0 and are never read or written.
+ *
+ * Logical owners ("ranks") are contiguous expert ranges: owner r holds experts
+ * [r*E/R, (r+1)*E/R).  Everything runs on one GPU; there is no communication.
+ *
+ * Errors: every entry point returns a sep_status; SEP_OK means the work was
+ * enqueued.  On any other status nothing was enqueued (except SEP_ERR_CUDA,
+ * where a launch may have failed part way) and sep_last_error() gives a
+ * message for the calling thread.  Errors found on the device (an expert id
+ * >= E) are reported by sep_handle_sync().  No call aborts, traps or prints.
+ */
+#ifndef SEP_H
+#define SEP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SEP_ABI_VERSION 1
+
+/* Exported from the shared library even when it is built with hidden visibility. */
+#if defined(__GNUC__) || defined(__clang__)
+#define SEP_API __attribute__((visibility("default")))
+#else
+#define SEP_API
+#endif
+
+typedef enum sep_status {
+    SEP_OK = 0,
+    SEP_ERR_INVALID_ARG = 1,     /* a size, pointer, alignment or mode is not supported */
+    SEP_ERR_CAPACITY = 2,        /* an output buffer has fewer rows than the layout needs */
+    SEP_ERR_BAD_EXPERT_ID = 3,   /* a topk_idx entry was >= num_experts (device-detected) */
+    SEP_ERR_HANDLE_MISMATCH = 4, /* handle used with another routing, shape or epoch */
+    SEP_ERR_TIMEOUT = 5,         /* a bounded wait on the device gave up */
+    SEP_ERR_CUDA = 6             /* a CUDA runtime call failed */
+} sep_status;
+
+/* Payload written into the pool by sep_dispatch. */
+typedef enum sep_payload {
+    SEP_PAYLOAD_BF16 = 0,        /* rows copied bit for bit, 2 bytes per element */
+    SEP_PAYLOAD_FP8_E4M3 = 1     /* rows quantised per 128 channels, 1 byte per element */
+} sep_payload;
+
+/* Per-128-channel scale format for SEP_PAYLOAD_FP8_E4M3 ("DeepEP Low-Latency
+ * Dispatch and Combine Kernels" article, "FP8 and Quantization Support" and
+ * the use_fp8 / round_scale / use_ue8m0 flags of "API Signature and Return
+ * Values").  For a group with amax = max |x|:
+ *   SEP_SCALE_F32      fp32 s = amax / 448 (IEEE division), s = 1 if amax == 0
+ *   SEP_SCALE_UE8M0    byte E* + 127, s = 2^E*, E* the smallest integer with
+ *                      448 * 2^E* >= amax (E* = 0 if amax == 0), clamped to [-127, 127]
+ *   SEP_SCALE_F32_POW2 the same 2^E* stored as fp32 ("round_scale")
+ * and every code is e4m3(x / s), rounded to nearest even, saturated to +-448. */
+typedef enum sep_scale {
+    SEP_SCALE_NONE = 0,
+    SEP_SCALE_F32 = 1,
+    SEP_SCALE_UE8M0 = 2,
+    SEP_SCALE_F32_POW2 = 3
+} sep_scale;
+
+/* sep_layout flags */
+#define SEP_LAYOUT_SYNC_COUNTS   0x1u  /* wait for the stream and copy the exact pool size to
+                                          the host, so capacity checks use it (the "CPU counts"
+                                          of PR #769) instead of the worst case */
+#define SEP_LAYOUT_TOKEN_IN_OWNER 0x2u /* also write is_token_in_rank [T, R] and
+                                          owner_token_counts [R] */
+
+/* Opaque routing layout ("EPHandle" in the blog): valid only for the routing
+ * that produced it (blog, "EPHandle": the handle is valid only for the routing
+ * layout that produced it).  Owns its device metadata. */
+typedef struct sep_handle sep_handle;
+
+/* Sizes and device arrays of a handle.  Device pointers belong to the handle
+ * and stay valid until the next sep_layout into it or sep_handle_free. */
+typedef struct sep_layout_info {
+    int64_t num_tokens;          /* T of the current layout */
+    int32_t top_k, num_experts, num_owners, block_m;
+    int64_t max_tokens;          /* T capacity of the handle */
+    int64_t max_pool_rows;       /* worst-case pool rows for max_tokens: any routing fits */
+    int64_t max_tiles;           /* max_pool_rows / block_m */
+    int64_t num_pool_rows;       /* exact pool rows P (multiple of block_m), -1 unless synced */
+    int64_t num_tiles;           /* exact tile count P / block_m, -1 unless synced */
+    uint32_t epoch;              /* bumped by every sep_layout into this handle */
+    uint32_t flags;              /* flags of the current layout */
+    const int32_t *expert_counts;            /* [E]   n_e: valid assignments per expert */
+    const int32_t *owner_counts;             /* [R]   L_r = sum of n_e over owner r's experts */
+    const int32_t *owner_token_counts;       /* [R]   tokens with >= 1 assignment on owner r
+                                                      (SEP_LAYOUT_TOKEN_IN_OWNER, else zeros) */
+    const uint8_t *is_token_in_rank;         /* [T, R] or NULL without SEP_LAYOUT_TOKEN_IN_OWNER */
+    const int32_t *expert_pool_block_offset; /* [E+1] first tile of expert e; [E] = tiles */
+    const int32_t *owner_pool_row_offset;    /* [R+1] first pool row of owner r; [R] = P */
+    const int32_t *tile_expert;              /* [max_tiles] expert of each tile (first NT valid) */
+    const int32_t *pool_arrival_target;      /* [max_tiles] valid rows in each tile, 1..block_m */
+    const uint32_t *pool_arrival_count;      /* [max_tiles] arrivals counted by a streaming dispatch */
+    const int32_t *src_pool_row;             /* [T, k] pool row of assignment (t, j), -1 if none */
+    const int32_t *pool_recv_token;          /* [max_pool_rows] source token t of a row, -1 = padding */
+    const int32_t *pool_recv_slot;           /* [max_pool_rows] source slot j of a row, -1 = padding */
+    const int64_t *device_sizes;             /* [2] device copy of {P, NT} for the current layout */
+} sep_layout_info;
+
+/*
+ * sep_layout — routing layout (the dispatch layout step: count, scan, assign).
+ *
+ * Counts valid assignments per expert and per owner, scans them into the
+ * expert-major BLOCK_M-padded pool (expert_pool_block_offset in tiles,
+ * tile_expert, pool_arrival_target = valid rows per tile) and assigns every
+ * valid assignment a = t*k + j a pool row.  Rows inside an expert follow
+ * ascending a (a stable counting sort), so the result is unique.
+ *
+ *  topk_idx     device [T, k] row-major, int32 (idx_bytes = 4) or int64 (8).
+ *               Entries < 0 mean "no assignment"; entries >= num_experts are
+ *               errors: skipped, and reported by sep_handle_sync().
+ *  num_tokens   T >= 0 (T = 0 is a valid, empty layout); T * k < 2^31.
+ *  top_k        1..32.
+ *  num_experts  1..1024; num_owners 1..num_experts dividing it.
+ *  block_m      1..1024 rows per tile.
+ *  flags        SEP_LAYOUT_* bits.
+ *  handle       in/out.  *handle == NULL: a new handle sized for exactly T
+ *               tokens is created.  *handle != NULL: it is reused (its epoch
+ *               is bumped, its previous layout is invalidated) if top_k,
+ *               num_experts, num_owners and block_m match and T fits its
+ *               capacity; otherwise SEP_ERR_HANDLE_MISMATCH and nothing changes.
+ * The handle's device memory is allocated stream-ordered on `stream` when it is
+ * created; later layouts into it allocate nothing.
+ */
+SEP_API sep_status sep_layout(const void *topk_idx, int idx_bytes, int64_t num_tokens, int top_k,
+                      int num_experts, int num_owners, int block_m, uint32_t flags,
+                      void *stream, sep_handle **handle);
+
+/* Creates an empty handle with capacity for max_tokens tokens (preallocation,
+ * as the blog's "ElasticBuffer" section recommends; flags as for sep_layout:
+ * SEP_LAYOUT_TOKEN_IN_OWNER reserves is_token_in_rank). */
+SEP_API sep_status sep_handle_create(int64_t max_tokens, int top_k, int num_experts, int num_owners,
+                             int block_m, uint32_t flags, void *stream, sep_handle **handle);
+
+/* Fills *info (host struct) for the handle's current layout.  Never blocks. */
+SEP_API sep_status sep_handle_info(const sep_handle *handle, sep_layout_info *info);
+
+/* Waits for `stream`, then reads the exact pool size and the device error word
+ * of the current layout into the handle (afterwards capacity checks use the
+ * exact size).  Returns SEP_ERR_BAD_EXPERT_ID if the layout met an expert id
+ * >= num_experts, else SEP_OK. */
+SEP_API sep_status sep_handle_sync(sep_handle *handle, void *stream);
+
+/*
+ * sep_dispatch — permute token rows into the pool (optionally FP8-quantised).
+ *
+ * For every valid assignment (t, j): recv_x[src_pool_row[t, j]] = x[t]
+ * (bf16 bits), or the e4m3 codes of x[t] with recv_scales[row] = its per-128
+ * channel scales (quantised once per token, written k times).  Weights are not
+ * applied (they belong to combine).  Padding rows are not written.
+ *
+ *  x             device bf16 [T, hidden], 16-byte aligned.
+ *  hidden        H: multiple of 8 for bf16, of 128 for FP8; H <= 65536.
+ *  payload/scale a sep_payload and a sep_scale (SEP_SCALE_NONE iff bf16).
+ *  recv_x        device [recv_capacity_rows, H] of bf16 or e4m3 bytes, 16-byte aligned.
+ *  recv_scales   device [recv_capacity_rows, H/128] fp32 (F32, F32_POW2) or
+ *                uint8 (UE8M0); NULL for bf16.
+ *  recv_capacity_rows  rows of recv_x (and recv_scales); must be >= the exact
+ *                pool size after a synced layout, else >= max_pool_rows
+ *                (SEP_ERR_CAPACITY otherwise: nothing is silently dropped, as
+ *                the blog's "Imbalance" section asks).
+ *  tile_ready    NULL, or device uint32 [tile_ready_len].  When given, each tile
+ *                is published once all its valid rows are written: the
+ *                dispatch counts arrivals in the handle's pool_arrival_count
+ *                (reset by sep_layout) and the writer that completes a tile
+ *                release-stores dispatch_seq into tile_ready[tile] (StreamEP
+ *                README, "Streaming dispatch in one paragraph").  A consumer
+ *                on another stream may acquire-load tile_ready[tile] and wait
+ *                until it reaches dispatch_seq (see sep_consume_tiles).
+ *  tile_ready_len entries of tile_ready; must cover the layout's tiles: the
+ *                exact tile count after a synced layout, else the worst case
+ *                for the current T (its worst-case pool rows / block_m).
+ *                SEP_ERR_CAPACITY otherwise.
+ *  dispatch_seq  != 0 when tile_ready is given, and (mod 2^32) greater than the
+ *                value used by the previous dispatch of this handle into the
+ *                same tile_ready array, so stale flags are never taken as
+ *                ready; SEP_ERR_INVALID_ARG otherwise.  tile_ready never needs
+ *                a reset.
+ */
+SEP_API sep_status sep_dispatch(sep_handle *handle, const void *x, int64_t hidden, int payload,
+                        int scale, void *recv_x, void *recv_scales,
+                        int64_t recv_capacity_rows, uint32_t *tile_ready,
+                        int64_t tile_ready_len, uint32_t dispatch_seq, void *stream);
+
+/*
+ * sep_combine — weighted top-k reduction back into token order.
+ *
+ * out[t] = bf16( sum over valid j, ascending, of topk_weight[t, j] *
+ *                y_pool[src_pool_row[t, j]] ) with fp32 products and sums
+ * ("DeepEP MoE dispatch/combine" blog, "Router 权重什么时候应用":
+ * y_t = sum_j p_{t,j} o_{t,j}).  Masked assignments contribute nothing; a
+ * token with none gets +0.
+ *
+ *  layout_epoch  the handle's epoch when the caller's routing was laid out;
+ *                a different value means the handle now holds another routing
+ *                (SEP_ERR_HANDLE_MISMATCH: the blog's "EPHandle" and
+ *                integration-contract sections ask to detect this).
+ *  y_pool        device bf16 [y_capacity_rows, hidden] in pool layout, 16-byte aligned.
+ *  hidden        multiple of 8.
+ *  topk_weight   device fp32 [T, k].
+ *  out           device bf16 [T, hidden], 16-byte aligned.
+ */
+SEP_API sep_status sep_combine(const sep_handle *handle, uint32_t layout_epoch, const void *y_pool,
+                       int64_t hidden, int64_t y_capacity_rows, const float *topk_weight,
+                       void *out, void *stream);
+
+/*
+ * sep_consume_tiles — a reference consumer of a streaming dispatch.
+ *
+ * Stands in for the grouped-GEMM consumer of the StreamEP README ("Streaming
+ * dispatch in one paragraph": a consumer spins on the acquire-load of
+ * tile_ready[tile] >= dispatch_seq from another stream, then proceeds).
+ * Launches num_ctas persistent CTAs (1..1024; keep it well below the SM count
+ * so a dispatch launched on another stream can run beside it).  Tiles are
+ * visited in the order a token-major dispatch completes them (tile i of every
+ * expert before tile i+1).  Each CTA waits for its tile with a bounded spin,
+ * then copies the tile's valid rows (pool_recv_token >= 0) from recv_x to the
+ * same rows of dst.  A wait gives up after timeout_ns nanoseconds of
+ * %globaltimer (or a fixed poll budget); then every CTA stops waiting,
+ * status[0] becomes SEP_ERR_TIMEOUT and status[1] counts the tiles not copied.
+ *
+ *  recv_x, dst   device [capacity_rows, row_bytes]; row_bytes a multiple of 16;
+ *                16-byte aligned; capacity_rows as for sep_dispatch's recv_x.
+ *  tile_ready    the array given to sep_dispatch, tile_ready_len entries.
+ *  status        device uint32 [2]; reset by this call, written by the kernel.
+ * Must be stream-ordered after the sep_layout of the handle (e.g. via an event);
+ * it is ordered against the dispatch only through tile_ready.
+ */
+SEP_API sep_status sep_consume_tiles(const sep_handle *handle, const void *recv_x, int64_t row_bytes,
+                             int64_t capacity_rows, const uint32_t *tile_ready,
+                             int64_t tile_ready_len, uint32_t dispatch_seq, void *dst,
+                             int num_ctas, uint64_t timeout_ns, uint32_t *status, void *stream);
+
+/* Frees the handle.  Its device memory is released stream-ordered on the
+ * stream of the last call that used it; the caller must have ordered every
+ * other stream that used the handle before that point.  NULL is a no-op. */
+SEP_API void sep_handle_free(sep_handle *handle);
+
+/* Message for the calling thread's last failed call ("" if none). */
+SEP_API const char *sep_last_error(void);
+
+/* Name of a status code. */
+SEP_API const char *sep_status_string(sep_status status);
+
+/* SEP_ABI_VERSION of the library. */
+SEP_API int sep_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SEP_H */

@@ -9,6 +9,14 @@ if ROOT not in sys.path:
 
 GOLDEN = os.path.join(ROOT, "tests", "golden")
 
+# the CUDA library and the oracle are compiled ahead of the tests (nvcc cross-
+# compiles for sm_100a without a GPU); both builds are no-ops when up to date
+from combine_route_layout_02_b200 import build as _sep_build  # noqa: E402
+import oracle as _oracle  # noqa: E402
+
+_sep_build.build()
+_oracle.build()
+
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
