@@ -108,4 +108,10 @@ cudaError_t launch_combine(const CombineParams &p, cudaStream_t s, int num_sms)
     return cudaGetLastError();
 }
 
+cudaError_t preload_combine_kernels()
+{
+    cudaFuncAttributes a;
+    return cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(combine_kernel));
+}
+
 }  // namespace sep

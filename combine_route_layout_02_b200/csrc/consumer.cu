@@ -100,4 +100,10 @@ cudaError_t launch_consume(const ConsumeParams &p, int num_ctas, cudaStream_t s)
     return cudaGetLastError();
 }
 
+cudaError_t preload_consumer_kernels()
+{
+    cudaFuncAttributes a;
+    return cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(consume_tiles_kernel));
+}
+
 }  // namespace sep

@@ -271,4 +271,24 @@ cudaError_t launch_dispatch(const DispatchParams &p, int payload, cudaStream_t s
     return p.tile_ready != nullptr ? launch_fp8<true>(p, s, num_sms) : launch_fp8<false>(p, s, num_sms);
 }
 
+cudaError_t preload_dispatch_kernels()
+{
+    const void *k[] = {
+        reinterpret_cast<const void *>(dispatch_bf16_kernel<4, false>),
+        reinterpret_cast<const void *>(dispatch_bf16_kernel<4, true>),
+        reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_F32, false>),
+        reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_F32, true>),
+        reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_UE8M0, false>),
+        reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_UE8M0, true>),
+        reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_F32_POW2, false>),
+        reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_F32_POW2, true>)};
+    cudaFuncAttributes a;
+    for (const void *f : k) {
+        const cudaError_t e = cudaFuncGetAttributes(&a, f);
+        if (e != cudaSuccess)
+            return e;
+    }
+    return cudaSuccess;
+}
+
 }  // namespace sep

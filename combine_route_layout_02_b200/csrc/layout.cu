@@ -348,4 +348,20 @@ cudaError_t launch_layout(const LayoutParams &p, int idx_bytes, cudaStream_t s)
     return idx_bytes == 8 ? launch_layout_t<long long>(p, s) : launch_layout_t<int>(p, s);
 }
 
+cudaError_t preload_layout_kernels()
+{
+    const void *k[] = {reinterpret_cast<const void *>(layout_count_kernel<int>),
+                       reinterpret_cast<const void *>(layout_count_kernel<long long>),
+                       reinterpret_cast<const void *>(layout_scan_kernel),
+                       reinterpret_cast<const void *>(layout_assign_kernel<int>),
+                       reinterpret_cast<const void *>(layout_assign_kernel<long long>)};
+    cudaFuncAttributes a;
+    for (const void *f : k) {
+        const cudaError_t e = cudaFuncGetAttributes(&a, f);
+        if (e != cudaSuccess)
+            return e;
+    }
+    return cudaSuccess;
+}
+
 }  // namespace sep

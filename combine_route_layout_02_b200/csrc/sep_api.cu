@@ -85,6 +85,26 @@ size_t carve(size_t *off, size_t bytes)
     return at;
 }
 
+// Load all kernels on this device once (see preload_* in sep_internal.cuh).
+sep_status preload_once(int dev)
+{
+    static bool done[64] = {false};
+    if (dev >= 0 && dev < 64 && done[dev])
+        return SEP_OK;
+    cudaError_t e = sep::preload_layout_kernels();
+    if (e == cudaSuccess)
+        e = sep::preload_dispatch_kernels();
+    if (e == cudaSuccess)
+        e = sep::preload_combine_kernels();
+    if (e == cudaSuccess)
+        e = sep::preload_consumer_kernels();
+    if (e != cudaSuccess)
+        return cuda_fail(e, "loading the library's kernels");
+    if (dev >= 0 && dev < 64)
+        done[dev] = true;
+    return SEP_OK;
+}
+
 sep_status create(int64_t T_cap, int k, int E, int R, int B, uint32_t flags, cudaStream_t s,
                   sep_handle **out)
 {
@@ -93,6 +113,8 @@ sep_status create(int64_t T_cap, int k, int E, int R, int B, uint32_t flags, cud
         return st;
     int dev = -1;
     if ((st = current_device(&dev)) != SEP_OK)
+        return st;
+    if ((st = preload_once(dev)) != SEP_OK)
         return st;
     sep_handle *h = new (std::nothrow) sep_handle();
     if (h == nullptr)

@@ -102,6 +102,15 @@ cudaError_t launch_consume(const ConsumeParams &p, int num_ctas, cudaStream_t s)
 
 // ------------------------------------------------------------------ utils
 
+// Force-load every kernel of a file on the current device.  CUDA loads kernels
+// lazily by default, and a load can synchronise the context; a consumer that
+// spins on flags written by a later kernel must never meet such a load, so the
+// library loads all its kernels up front (on the first handle of a device).
+cudaError_t preload_layout_kernels();
+cudaError_t preload_dispatch_kernels();
+cudaError_t preload_combine_kernels();
+cudaError_t preload_consumer_kernels();
+
 int device_sm_count();
 
 // Resident CTAs per SM for a kernel at a block size (cached per kernel).

@@ -145,7 +145,10 @@ typedef struct sep_layout_info {
  *               num_experts, num_owners and block_m match and T fits its
  *               capacity; otherwise SEP_ERR_HANDLE_MISMATCH and nothing changes.
  * The handle's device memory is allocated stream-ordered on `stream` when it is
- * created; later layouts into it allocate nothing.
+ * created; later layouts into it allocate nothing.  Creating the first handle
+ * on a device also loads all of the library's kernels on it (CUDA otherwise
+ * loads kernels lazily, and a load may wait for running kernels, which would
+ * stall a dispatch behind a consumer that is waiting for it).
  */
 SEP_API sep_status sep_layout(const void *topk_idx, int idx_bytes, int64_t num_tokens, int top_k,
                       int num_experts, int num_owners, int block_m, uint32_t flags,
@@ -249,7 +252,11 @@ SEP_API sep_status sep_combine(const sep_handle *handle, uint32_t layout_epoch, 
  *  tile_ready    the array given to sep_dispatch, tile_ready_len entries.
  *  status        device uint32 [2]; reset by this call, written by the kernel.
  * Must be stream-ordered after the sep_layout of the handle (e.g. via an event);
- * it is ordered against the dispatch only through tile_ready.
+ * it is ordered against the dispatch only through tile_ready.  Between this
+ * call and the sep_dispatch it waits for, the host must not wait for the
+ * device (a device or stream synchronisation, or a copy from pageable host
+ * memory): that wait would hold the dispatch back until the consumer's waits
+ * time out (SEP_ERR_TIMEOUT; nothing hangs).
  */
 SEP_API sep_status sep_consume_tiles(const sep_handle *handle, const void *recv_x, int64_t row_bytes,
                              int64_t capacity_rows, const uint32_t *tile_ready,

@@ -331,12 +331,13 @@ def test_streaming_fp8_publishes_every_tile():
         tile_ready = torch.zeros(NT, dtype=torch.int32, device="cuda")
         dst = torch.zeros_like(recv)
         status = torch.zeros(2, dtype=torch.int32, device="cuda")
+        x = d["x"].cuda()             # before the consumer: a pageable copy would wait for it
         side = torch.cuda.Stream()
         ev = torch.cuda.Event()
         ev.record()
         side.wait_event(ev)
         sep.sep_consume_tiles(h, recv, tile_ready, 11, dst, status, num_ctas=8, stream=side)
-        sep.sep_dispatch(h, d["x"].cuda(), recv, payload="fp8", scale="ue8m0", recv_scales=scales,
+        sep.sep_dispatch(h, x, recv, payload="fp8", scale="ue8m0", recv_scales=scales,
                          tile_ready=tile_ready, dispatch_seq=11)
         torch.cuda.synchronize()
         assert status.cpu().tolist() == [0, 0]
@@ -442,3 +443,45 @@ def test_full_streaming_bench_configuration():
         check_combine(bf16_bits(out), oracle.combine(want, d["topk_weight"].numpy(), lay))
     finally:
         sep.sep_handle_free(h)
+
+
+_FRESH_PROCESS_STREAMING = r"""
+import sys, torch
+sys.path.insert(0, sys.argv[1])
+import combine_route_layout_02_b200 as sep
+import workloads as W
+w = W.scaled(W.WORKLOADS["decode"], 256)
+d = W.make_inputs(w)
+idx, x = d["topk_idx"].cuda(), d["x"].cuda()
+h = sep.sep_layout(idx, w.E, w.R, w.B, flags=sep.SEP_LAYOUT_SYNC_COUNTS)
+info = h.info()
+P, NT = info.num_pool_rows, info.num_tiles
+recv = torch.zeros(P, w.H, dtype=torch.uint8, device="cuda")
+scales = torch.zeros(P, w.H // 128, dtype=torch.float32, device="cuda")
+tile_ready = torch.zeros(NT, dtype=torch.int32, device="cuda")
+dst = torch.zeros_like(recv)
+status = torch.zeros(2, dtype=torch.int32, device="cuda")
+side = torch.cuda.Stream()
+side.wait_stream(torch.cuda.current_stream())
+sep.sep_consume_tiles(h, recv, tile_ready, 1, dst, status, num_ctas=8, stream=side)
+sep.sep_dispatch(h, x, recv, payload="fp8", scale="f32_pow2", recv_scales=scales,
+                 tile_ready=tile_ready, dispatch_seq=1)
+torch.cuda.synchronize()
+ok = status.cpu().tolist() == [0, 0] and bool((tile_ready == 1).all()) and bool(torch.equal(dst, recv))
+sep.sep_handle_free(h)
+print("STATUS", status.cpu().tolist(), "OK" if ok else "BAD")
+sys.exit(0 if ok else 1)
+"""
+
+
+def test_streaming_first_launch_in_a_fresh_process():
+    """Consumer launched first, then a dispatch kernel this process has never
+    run: the library must already have loaded it (a lazy load on first launch
+    would wait for the spinning consumer)."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _FRESH_PROCESS_STREAMING, root], capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0 and "OK" in r.stdout, r.stdout + r.stderr
