@@ -13,17 +13,21 @@
 //   owner_counts               L_r = sum of n_e over owner r's experts (blog,
 //                              "Imbalance 决定 buffer 与尾延迟")
 //
-// Three launches on one stream:
-//   count   one warp per chunk of 32*rounds assignments; __match_any_sync
-//           groups lanes holding the same expert so each distinct expert costs
-//           one shared-memory update per round; writes a per-chunk histogram.
+// Three launches on one stream.  The assignment stream is cut into at most
+// 128 CTA chunks of 8 warps x 32 lanes x `rounds` entries; warp w of chunk c
+// owns a contiguous run of 32*rounds entries, so chunk order, warp order and
+// lane order all follow ascending a.
+//   count   per warp, __match_any_sync groups lanes holding the same expert so
+//           each distinct expert costs one shared-memory add per round; the
+//           CTA sums its warps and writes one histogram column [E][chunk].
 //   scan    one 1024-thread CTA: per-expert exclusive prefix over chunks (all
 //           loads issued before any use), then a block scan of tiles over experts.
-//   assign  the same chunk walk as count; a lane's row is its expert's cursor
-//           plus the number of lower lanes holding that expert.  Also writes the
-//           tile tables and marks padding rows, experts spread over CTAs.
-// The chunk order and the in-warp lane order both follow ascending a, so the
-// result is the unique stable order and needs no atomics on the data path.
+//   assign  recounts its chunk per warp, turns the warp counts into cursors
+//           (expert's pool start + chunk prefix + earlier warps of the chunk),
+//           then walks the chunk again: a lane's row is its expert's cursor
+//           plus the number of lower lanes holding that expert.  Also writes
+//           the tile tables and marks padding rows, experts spread over CTAs.
+// The result is the unique stable order and needs no atomics on the data path.
 #include "sep_internal.cuh"
 
 namespace sep {
@@ -62,22 +66,11 @@ __device__ __forceinline__ int warp_inclusive_scan(int v, int lane)
     return v;
 }
 
+// Per-warp expert counts of the warp's run of the chunk into cnt[E] (shared).
 template <typename IdxT>
-__global__ void __launch_bounds__(kWarps * 32) layout_count_kernel(LayoutParams p)
+__device__ __forceinline__ void count_warp_run(const LayoutParams &p, const IdxT *idx, int64_t a0,
+                                               int32_t *cnt, int lane, bool &bad)
 {
-    extern __shared__ int32_t s_cnt[];                   // [kWarps][E]
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t wc = (int64_t)blockIdx.x * kWarps + warp;
-    if (wc >= p.num_wchunks)
-        return;                                          // whole warp; no block barrier follows
-    int32_t *cnt = s_cnt + warp * p.E;
-    for (int e = lane; e < p.E; e += 32)
-        cnt[e] = 0;
-    __syncwarp();
-
-    const IdxT *idx = static_cast<const IdxT *>(p.topk_idx);
-    const int64_t a0 = wc * 32 * p.rounds;
-    bool bad = false;
     for (int r = 0; r < p.rounds; r += kPrefetch) {
         int ev[kPrefetch];
 #pragma unroll
@@ -95,10 +88,31 @@ __global__ void __launch_bounds__(kWarps * 32) layout_count_kernel(LayoutParams 
             __syncwarp();
         }
     }
-    for (int e = lane; e < p.E; e += 32)
-        p.wchunk_hist[(int64_t)e * p.num_wchunks + wc] = cnt[e];
+}
+
+template <typename IdxT>
+__global__ void __launch_bounds__(kWarps * 32) layout_count_kernel(LayoutParams p)
+{
+    extern __shared__ int32_t s_cnt[];                   // [kWarps][E]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x;
+    for (int i = threadIdx.x; i < kWarps * p.E; i += blockDim.x)
+        s_cnt[i] = 0;
+    __syncthreads();
+    const IdxT *idx = static_cast<const IdxT *>(p.topk_idx);
+    const int64_t a0 = ((int64_t)c * kWarps + warp) * 32 * p.rounds;
+    bool bad = false;
+    count_warp_run(p, idx, a0, s_cnt + warp * p.E, lane, bad);
     if (__any_sync(kFullMask, bad) && lane == 0)
         atomicMax(p.bad_epoch, p.epoch);
+    __syncthreads();
+    for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
+        int sum = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w)
+            sum += s_cnt[w * p.E + e];
+        p.wchunk_hist[(int64_t)e * p.num_wchunks + c] = sum;
+    }
 }
 
 __global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(LayoutParams p)
@@ -199,19 +213,33 @@ __global__ void __launch_bounds__(kScanThreads) layout_scan_kernel(LayoutParams 
 template <typename IdxT>
 __global__ void __launch_bounds__(kWarps * 32) layout_assign_kernel(LayoutParams p)
 {
+    allow_dependents();
     extern __shared__ int32_t s_cur[];                   // [kWarps][E] cursors, then [R]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t wc = (int64_t)blockIdx.x * kWarps + warp;
+    const int c = blockIdx.x;
     const IdxT *idx = static_cast<const IdxT *>(p.topk_idx);
 
-    if (wc < p.num_wchunks) {
-        int32_t *cur = s_cur + warp * p.E;
-        for (int e = lane; e < p.E; e += 32)
-            cur[e] = p.expert_pool_block_offset[e] * p.B + p.wchunk_base[(int64_t)e * p.num_wchunks + wc];
-        __syncwarp();
-        const int64_t a0 = wc * 32 * p.rounds;
-        const unsigned lower = (1u << lane) - 1u;
+    if (c < p.num_wchunks) {                             // block-uniform
+        for (int i = threadIdx.x; i < kWarps * p.E; i += blockDim.x)
+            s_cur[i] = 0;
+        __syncthreads();
+        const int64_t a0 = ((int64_t)c * kWarps + warp) * 32 * p.rounds;
         bool bad = false;
+        count_warp_run(p, idx, a0, s_cur + warp * p.E, lane, bad);
+        __syncthreads();
+        // warp counts -> cursors: pool start of e + earlier chunks + earlier warps
+        for (int e = threadIdx.x; e < p.E; e += blockDim.x) {
+            int run = p.expert_pool_block_offset[e] * p.B + p.wchunk_base[(int64_t)e * p.num_wchunks + c];
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) {
+                const int n = s_cur[w * p.E + e];
+                s_cur[w * p.E + e] = run;
+                run += n;
+            }
+        }
+        __syncthreads();
+        int32_t *cur = s_cur + warp * p.E;
+        const unsigned lower = (1u << lane) - 1u;
         for (int r = 0; r < p.rounds; r += kPrefetch) {
             int ev[kPrefetch];
 #pragma unroll
@@ -241,6 +269,7 @@ __global__ void __launch_bounds__(kWarps * 32) layout_assign_kernel(LayoutParams
                 }
             }
         }
+        __syncthreads();                                 // s_cur is reused below
     }
 
     // tile tables and padding rows; experts spread over CTAs
@@ -304,16 +333,279 @@ __global__ void __launch_bounds__(kWarps * 32) layout_assign_kernel(LayoutParams
     }
 }
 
+// ------------------------------------------------------- single launch
+//
+// The same three steps in one cooperative launch (every CTA resident), split
+// by two grid barriers:
+//   A  count this CTA's chunk; the CTA's histogram column -> wchunk_hist
+//   B  warp w of CTA c scans the chunk column of expert c*8+w (+ multiples of
+//      8*G): per-chunk exclusive bases -> wchunk_base, n_e -> expert_counts
+//   C  every CTA scans ceil(n_e/B) over experts in shared memory, turns its
+//      warp counts from A into cursors and assigns its chunk; CTA 0 writes
+//      the offsets, sizes and owner arrays; tile tables and padding rows
+//      are spread over CTAs as in the three-launch path.
+// Each barrier is a bounded spin on an arrival counter; launches of odd and
+// even epochs use different counters, and each launch zeroes the one the next
+// launch will use.  A barrier that gives up records the epoch in the handle's
+// timeout word and the kernel returns (sep_handle_sync reports it).
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *ptr)
+{
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// All CTAs arrive on *counter; returns false (in every thread of the CTA) if
+// the counter did not reach target within the limit.
+__device__ __forceinline__ bool grid_barrier(const LayoutParams &p, unsigned *counter, unsigned target,
+                                             int *s_flag)
+{
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(counter, 1u);
+        bool ok = false;
+        const uint64_t t0 = global_ns();
+        for (uint32_t it = 0; it < (1u << 22); ++it) {
+            if ((int)(ld_acquire_u32(counter) - target) >= 0) {
+                ok = true;
+                break;
+            }
+            if (global_ns() - t0 > 200000000ull)
+                break;
+            __nanosleep(64);
+        }
+        __threadfence();
+        if (!ok)
+            atomicMax(p.timeout_epoch, p.epoch);
+        *s_flag = ok ? 1 : 0;
+    }
+    __syncthreads();
+    return *s_flag != 0;
+}
+
+template <typename IdxT>
+__global__ void __launch_bounds__(kWarps * 32) layout_fused_kernel(LayoutParams p)
+{
+    extern __shared__ int32_t sm[];          // [kWarps][E] counts/cursors, [E+1] offsets, [R] owner tokens
+    __shared__ int s_flag;
+    __shared__ int s_part[kWarps * 32];
+    int32_t *s_cnt = sm;
+    int32_t *s_off = sm + kWarps * p.E;
+    int32_t *s_own = s_off + p.E + 1;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = blockIdx.x;
+    const int G = gridDim.x;
+    const int E = p.E, nc = p.num_wchunks;
+    const IdxT *idx = static_cast<const IdxT *>(p.topk_idx);
+    allow_dependents();
+    unsigned *counter = p.barrier_words + (p.epoch & 1u);
+    if (c == 0 && threadIdx.x == 0)
+        p.barrier_words[(p.epoch & 1u) ^ 1u] = 0u;      // the next launch's counter
+    if (c == 0)
+        for (int r = threadIdx.x; r < p.R; r += blockDim.x)
+            p.owner_token_counts[r] = 0;
+
+    // A. count
+    for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x)
+        s_cnt[i] = 0;
+    __syncthreads();
+    const int64_t a0 = ((int64_t)c * kWarps + warp) * 32 * p.rounds;
+    bool bad = false;
+    count_warp_run(p, idx, a0, s_cnt + warp * E, lane, bad);
+    if (__any_sync(kFullMask, bad) && lane == 0)
+        atomicMax(p.bad_epoch, p.epoch);
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int sum = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w)
+            sum += s_cnt[w * E + e];
+        p.wchunk_hist[(int64_t)e * nc + c] = sum;
+    }
+    if (!grid_barrier(p, counter, (unsigned)G, &s_flag))
+        return;
+
+    // B. per-expert scan over chunks, one warp per expert
+    for (int e = c * kWarps + warp; e < E; e += G * kWarps) {
+        const int32_t *col = p.wchunk_hist + (int64_t)e * nc;
+        int32_t *bcol = p.wchunk_base + (int64_t)e * nc;
+        int running = 0;
+        for (int c0 = 0; c0 < nc; c0 += 32) {
+            const int cc = c0 + lane;
+            const int x = cc < nc ? __ldcg(col + cc) : 0;     // written by other CTAs
+            const int incl = warp_inclusive_scan(x, lane);
+            if (cc < nc)
+                bcol[cc] = running + incl - x;
+            running += __shfl_sync(kFullMask, incl, 31);
+        }
+        if (lane == 0)
+            p.expert_counts[e] = running;
+    }
+    if (!grid_barrier(p, counter, 2u * (unsigned)G, &s_flag))
+        return;
+
+    // C. tile offsets over experts (each thread sums a run of experts)
+    const int per = (E + blockDim.x - 1) / blockDim.x;
+    const int e0 = threadIdx.x * per;
+    int local = 0;
+    for (int e = e0; e < min(E, e0 + per); ++e)
+        local += (__ldcg(p.expert_counts + e) + p.B - 1) / p.B;
+    const int incl = warp_inclusive_scan(local, lane);
+    if (lane == 31)
+        s_part[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const int v = lane < kWarps ? s_part[lane] : 0;
+        const int inc2 = warp_inclusive_scan(v, lane);
+        if (lane < kWarps)
+            s_part[lane] = inc2 - v;
+    }
+    __syncthreads();
+    int run = s_part[warp] + incl - local;
+    for (int e = e0; e < min(E, e0 + per); ++e) {
+        s_off[e] = run;
+        run += (__ldcg(p.expert_counts + e) + p.B - 1) / p.B;
+    }
+    if (threadIdx.x == blockDim.x - 1)
+        s_off[E] = s_part[warp] + incl;                   // last thread holds the grand total
+    __syncthreads();
+    if (c == 0) {
+        for (int e = threadIdx.x; e <= E; e += blockDim.x)
+            p.expert_pool_block_offset[e] = s_off[e];
+        if (threadIdx.x == 0) {
+            p.sizes[0] = (int64_t)s_off[E] * p.B;
+            p.sizes[1] = s_off[E];
+        }
+        const int E_loc = E / p.R;
+        for (int r = threadIdx.x; r <= p.R; r += blockDim.x) {
+            p.owner_pool_row_offset[r] = s_off[r * E_loc] * p.B;
+            if (r < p.R) {
+                int sum = 0;
+                for (int q = r * E_loc; q < (r + 1) * E_loc; ++q)
+                    sum += __ldcg(p.expert_counts + q);
+                p.owner_counts[r] = sum;
+            }
+        }
+    }
+    // warp counts -> cursors, then the assignment walk
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int cur = s_off[e] * p.B + __ldcg(p.wchunk_base + (int64_t)e * nc + c);
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            const int n = s_cnt[w * E + e];
+            s_cnt[w * E + e] = cur;
+            cur += n;
+        }
+    }
+    __syncthreads();
+    {
+        int32_t *cur = s_cnt + warp * E;
+        const unsigned lower = (1u << lane) - 1u;
+        for (int r = 0; r < p.rounds; r += kPrefetch) {
+            int ev[kPrefetch];
+#pragma unroll
+            for (int u = 0; u < kPrefetch; ++u)
+                ev[u] = (r + u < p.rounds)
+                            ? expert_of(idx, a0 + (int64_t)(r + u) * 32 + lane, p.Na, E, bad)
+                            : -1;
+#pragma unroll
+            for (int u = 0; u < kPrefetch; ++u) {
+                if (r + u >= p.rounds)
+                    break;                               // warp-uniform
+                const int64_t a = a0 + (int64_t)(r + u) * 32 + lane;
+                const int e = ev[u];
+                const unsigned peers = __match_any_sync(kFullMask, e);
+                const int row = e >= 0 ? cur[e] + __popc(peers & lower) : -1;
+                __syncwarp();
+                if (e >= 0 && lane == __ffs(peers) - 1)
+                    cur[e] += __popc(peers);
+                __syncwarp();
+                if (a < p.Na) {
+                    p.src_pool_row[a] = row;
+                    if (row >= 0) {
+                        const unsigned t = (unsigned)a / (unsigned)p.k;
+                        p.pool_recv_token[row] = (int32_t)t;
+                        p.pool_recv_slot[row] = (int32_t)((unsigned)a - t * (unsigned)p.k);
+                    }
+                }
+            }
+        }
+    }
+    // tile tables and padding rows; experts spread over CTAs
+    for (int e = c; e < E; e += G) {
+        const int t0 = s_off[e], t1 = s_off[e + 1];
+        const int n = __ldcg(p.expert_counts + e);
+        for (int i = threadIdx.x; i < t1 - t0; i += blockDim.x) {
+            p.tile_expert[t0 + i] = e;
+            p.pool_arrival_target[t0 + i] = min(p.B, n - i * p.B);
+            p.pool_arrival_count[t0 + i] = 0u;
+        }
+        const int64_t r1 = (int64_t)t1 * p.B;
+        for (int64_t row = (int64_t)t0 * p.B + n + threadIdx.x; row < r1; row += blockDim.x) {
+            p.pool_recv_token[row] = -1;
+            p.pool_recv_slot[row] = -1;
+        }
+    }
+    // optional: which owners each token reaches, and per-owner token counts
+    if (p.is_token_in_rank != nullptr) {
+        for (int r = threadIdx.x; r < p.R; r += blockDim.x)
+            s_own[r] = 0;
+        __syncthreads();
+        const int E_loc = E / p.R;
+        for (int64_t t = (int64_t)c * blockDim.x + threadIdx.x; t < p.T; t += (int64_t)G * blockDim.x) {
+            uint8_t *dst = p.is_token_in_rank + t * p.R;
+            for (int r = 0; r < p.R; ++r) {
+                int in = 0;
+                for (int j = 0; j < p.k; ++j) {
+                    const int e = expert_of(idx, t * p.k + j, p.Na, E, bad);
+                    in |= (e >= 0 && e / E_loc == r);
+                }
+                dst[r] = (uint8_t)in;
+                if (in)
+                    atomicAdd(&s_own[r], 1);
+            }
+        }
+        __syncthreads();
+        for (int r = threadIdx.x; r < p.R; r += blockDim.x)
+            if (s_own[r])
+                atomicAdd(&p.owner_token_counts[r], s_own[r]);
+    }
+}
+
 template <typename IdxT>
 cudaError_t launch_layout_t(const LayoutParams &p, cudaStream_t s)
 {
-    const int blocks = (p.num_wchunks + kWarps - 1) / kWarps;
+    const int chunks = p.num_wchunks;
     const size_t smem_count = (size_t)kWarps * p.E * sizeof(int32_t);
+    const size_t smem_fused = smem_count + (size_t)(p.E + 1 + p.R) * sizeof(int32_t);
+    if (chunks > 0) {
+        // single launch when every CTA can be resident at once
+        int per_sm = 0;
+        int dev = 0, sms = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layout_fused_kernel<IdxT>, kWarps * 32,
+                                                          smem_fused) == cudaSuccess &&
+            chunks <= per_sm * sms) {
+            LayoutParams q = p;
+            void *args[] = {&q};
+            return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(layout_fused_kernel<IdxT>),
+                                               dim3(chunks), dim3(kWarps * 32), args, smem_fused, s);
+        }
+        layout_count_kernel<IdxT><<<chunks, kWarps * 32, smem_count, s>>>(p);
+    }
     const size_t smem_assign = smem_count + (size_t)p.R * sizeof(int32_t);
-    if (blocks > 0)
-        layout_count_kernel<IdxT><<<blocks, kWarps * 32, smem_count, s>>>(p);
     layout_scan_kernel<<<1, kScanThreads, 0, s>>>(p);
-    const int ablocks = max(blocks, min(p.E, 64));
+    const int ablocks = max(chunks, min(p.E, 64));
     layout_assign_kernel<IdxT><<<ablocks, kWarps * 32, smem_assign, s>>>(p);
     return cudaGetLastError();
 }
@@ -322,8 +614,9 @@ cudaError_t launch_layout_t(const LayoutParams &p, cudaStream_t s)
 
 int layout_rounds_for(int64_t Na)
 {
-    // about 128 chunks, 1..64 rounds of 32 assignments per chunk
-    int64_t r = (Na + 32 * 128 - 1) / (32 * 128);
+    // at most 128 CTA chunks of 8 warps; 1..64 rounds of 32 assignments per warp
+    const int64_t per_round = 32LL * kWarps * 128;
+    int64_t r = (Na + per_round - 1) / per_round;
     if (r < 1)
         r = 1;
     if (r > 64)
@@ -333,13 +626,14 @@ int layout_rounds_for(int64_t Na)
 
 int64_t layout_wchunks_for(int64_t Na, int rounds)
 {
-    return (Na + 32LL * rounds - 1) / (32LL * rounds);
+    const int64_t per_chunk = 32LL * kWarps * rounds;
+    return (Na + per_chunk - 1) / per_chunk;
 }
 
 int64_t layout_wchunk_capacity(int64_t Na_cap)
 {
-    // rounds < 64 keeps the count at or below 128; at 64 rounds it grows with Na
-    const int64_t big = (Na_cap + 32LL * 64 - 1) / (32LL * 64);
+    // below 64 rounds the chunk count stays at or below 128; at 64 it grows with Na
+    const int64_t big = (Na_cap + 32LL * kWarps * 64 - 1) / (32LL * kWarps * 64);
     return big > 128 ? big : 128;
 }
 
@@ -350,7 +644,9 @@ cudaError_t launch_layout(const LayoutParams &p, int idx_bytes, cudaStream_t s)
 
 cudaError_t preload_layout_kernels()
 {
-    const void *k[] = {reinterpret_cast<const void *>(layout_count_kernel<int>),
+    const void *k[] = {reinterpret_cast<const void *>(layout_fused_kernel<int>),
+                       reinterpret_cast<const void *>(layout_fused_kernel<long long>),
+                       reinterpret_cast<const void *>(layout_count_kernel<int>),
                        reinterpret_cast<const void *>(layout_count_kernel<long long>),
                        reinterpret_cast<const void *>(layout_scan_kernel),
                        reinterpret_cast<const void *>(layout_assign_kernel<int>),

@@ -136,7 +136,8 @@ sep_status create(int64_t T_cap, int k, int E, int R, int B, uint32_t flags, cud
     const int64_t NT1 = h->NT_cap > 0 ? h->NT_cap : 1;
     const int64_t Na1 = h->Na_cap > 0 ? h->Na_cap : 1;
     size_t off = 0;
-    const size_t o_sizes = carve(&off, 32);              // {P, NT} + bad_epoch, one copy to the host
+    const size_t o_sizes = carve(&off, 32);              // {P, NT}, bad_epoch, timeout_epoch: one copy to the host
+    const size_t o_bar = carve(&off, 8);
     const size_t o_ec = carve(&off, (size_t)E * 4);
     const size_t o_oc = carve(&off, (size_t)R * 4);
     const size_t o_otc = carve(&off, (size_t)R * 4);
@@ -166,6 +167,8 @@ sep_status create(int64_t T_cap, int k, int E, int R, int B, uint32_t flags, cud
     char *b = static_cast<char *>(h->block);
     h->sizes = reinterpret_cast<int64_t *>(b + o_sizes);
     h->bad_epoch = reinterpret_cast<uint32_t *>(b + o_sizes + 16);
+    h->timeout_epoch = reinterpret_cast<uint32_t *>(b + o_sizes + 20);
+    h->barrier_words = reinterpret_cast<uint32_t *>(b + o_bar);
     h->expert_counts = reinterpret_cast<int32_t *>(b + o_ec);
     h->owner_counts = reinterpret_cast<int32_t *>(b + o_oc);
     h->owner_token_counts = reinterpret_cast<int32_t *>(b + o_otc);
@@ -180,7 +183,7 @@ sep_status create(int64_t T_cap, int k, int E, int R, int B, uint32_t flags, cud
     h->wchunk_hist = reinterpret_cast<int32_t *>(b + o_hist);
     h->wchunk_base = reinterpret_cast<int32_t *>(b + o_base);
     h->is_token_in_rank = (flags & SEP_LAYOUT_TOKEN_IN_OWNER) ? reinterpret_cast<uint8_t *>(b + o_in) : nullptr;
-    e = cudaMemsetAsync(h->sizes, 0, 32, s);             // sizes and bad_epoch start at zero
+    e = cudaMemsetAsync(h->sizes, 0, o_bar + 8 - o_sizes, s);   // sizes, error words, barrier counters
     if (e != cudaSuccess) {
         cudaFreeAsync(h->block, s);
         cudaFreeHost(h->host_mirror);
@@ -342,6 +345,8 @@ sep_status sep_layout(const void *topk_idx, int idx_bytes, int64_t num_tokens, i
     p.pool_recv_slot = h->pool_recv_slot;
     p.sizes = h->sizes;
     p.bad_epoch = h->bad_epoch;
+    p.timeout_epoch = h->timeout_epoch;
+    p.barrier_words = h->barrier_words;
     p.epoch = h->epoch;
     if (p.num_wchunks > h->wchunk_cap)
         return fail(SEP_ERR_CUDA, "internal: chunk table too small");
@@ -403,10 +408,12 @@ sep_status sep_handle_sync(sep_handle *h, void *stream)
     h->P = h->host_mirror[0];
     h->NT = h->host_mirror[1];
     h->synced = 1;
-    uint32_t bad = 0;
-    std::memcpy(&bad, h->host_mirror + 2, sizeof bad);
-    if (bad != 0 && bad == h->epoch)
+    uint32_t words[2] = {0, 0};
+    std::memcpy(words, h->host_mirror + 2, sizeof words);
+    if (words[0] != 0 && words[0] == h->epoch)
         return fail(SEP_ERR_BAD_EXPERT_ID, "topk_idx holds an expert id >= num_experts (%d)", h->E);
+    if (words[1] != 0 && words[1] == h->epoch)
+        return fail(SEP_ERR_TIMEOUT, "a layout barrier or dispatch/combine copy did not complete within its wait limit");
     return SEP_OK;
 }
 
@@ -488,6 +495,8 @@ sep_status sep_dispatch(sep_handle *h, const void *x, int64_t hidden, int payloa
     p.pool_arrival_count = h->pool_arrival_count;
     p.pool_arrival_target = h->pool_arrival_target;
     p.seq = dispatch_seq;
+    p.error_epoch = h->timeout_epoch;
+    p.epoch = h->epoch;
     // split a token row over several warps when there are too few tokens to fill the GPU
     const int64_t units = fp8 ? (hidden + 511) / 512 : ((hidden / 8) + 31) / 32;   // warp-steps per row
     const int64_t want_warps = (int64_t)num_sms * 32;
@@ -541,6 +550,8 @@ sep_status sep_combine(const sep_handle *h, uint32_t layout_epoch, const void *y
     p.src_pool_row = h->src_pool_row;
     p.w = topk_weight;
     p.out = out;
+    p.error_epoch = h->timeout_epoch;
+    p.epoch = h->epoch;
     const int64_t units = ((hidden / 8) + 31) / 32;
     const int64_t want_warps = (int64_t)num_sms * 32;
     int64_t segs = (want_warps + h->T - 1) / h->T;

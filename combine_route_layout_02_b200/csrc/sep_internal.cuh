@@ -12,15 +12,16 @@ constexpr unsigned kFullMask = 0xffffffffu;
 
 // ----------------------------------------------------------------- layout
 
-// Per-warp chunks of the assignment stream: warp w of the count / assign
-// kernels owns assignments [w * 32 * rounds, (w + 1) * 32 * rounds).
+// CTA chunks of the assignment stream: CTA c of the count / assign kernels
+// owns assignments [c * 256 * rounds, (c + 1) * 256 * rounds), and its warp w
+// the contiguous run of 32 * rounds entries starting at w * 32 * rounds.
 struct LayoutParams {
     const void *topk_idx;
     int64_t T;
     int k, E, R, B;
     int64_t Na;                      // T * k
-    int rounds;                      // 32-entry rounds per warp chunk
-    int num_wchunks;
+    int rounds;                      // 32-entry rounds per warp
+    int num_wchunks;                 // CTA chunks
     int32_t *wchunk_hist;            // [E][num_wchunks] counts per (expert, chunk)
     int32_t *wchunk_base;            // [E][num_wchunks] exclusive prefix over chunks
     int32_t *expert_counts;          // [E]
@@ -37,6 +38,8 @@ struct LayoutParams {
     int32_t *pool_recv_slot;         // [P_cap]
     int64_t *sizes;                  // [2] = {P, NT}
     uint32_t *bad_epoch;             // last epoch that met an id >= E
+    uint32_t *timeout_epoch;         // last epoch whose grid barrier gave up
+    uint32_t *barrier_words;         // [2] arrival counters, used on alternate epochs
     uint32_t epoch;
 };
 
@@ -62,6 +65,9 @@ struct DispatchParams {
     uint32_t *pool_arrival_count;
     const int32_t *pool_arrival_target;
     uint32_t seq;
+    // a bounded wait that gave up records the layout epoch here
+    uint32_t *error_epoch;
+    uint32_t epoch;
 };
 
 cudaError_t launch_dispatch(const DispatchParams &p, int payload, cudaStream_t s, int num_sms);
@@ -77,6 +83,8 @@ struct CombineParams {
     void *out;                       // bf16 [T][H]
     int segs;                        // warps sharing one token row
     int seg_len;                     // 16-byte vectors per warp
+    uint32_t *error_epoch;           // a bounded wait that gave up records the epoch
+    uint32_t epoch;
 };
 
 cudaError_t launch_combine(const CombineParams &p, cudaStream_t s, int num_sms);
@@ -101,6 +109,44 @@ struct ConsumeParams {
 cudaError_t launch_consume(const ConsumeParams &p, int num_ctas, cudaStream_t s);
 
 // ------------------------------------------------------------------ utils
+
+// Programmatic dependent launch: dispatch and combine are launched so their
+// CTAs may start while the previous kernel of the stream drains, and every
+// one of them executes griddepcontrol.wait before its first global memory
+// access, which waits for the previous grid to complete and its writes to be
+// visible.  Stream-order semantics are unchanged; only launch latency overlaps.
+constexpr bool kUsePDL = true;
+
+__device__ __forceinline__ void grid_dependency_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void allow_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                          Args... args)
+{
+    if (!kUsePDL) {
+        kernel<<<grid, block, smem, s>>>(args...);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 // Force-load every kernel of a file on the current device.  CUDA loads kernels
 // lazily by default, and a load can synchronise the context; a consumer that
@@ -146,6 +192,8 @@ struct sep_handle {
     uint8_t *is_token_in_rank;
     int64_t *sizes;
     uint32_t *bad_epoch;
-    // pinned host mirror of {P, NT, bad_epoch}
+    uint32_t *timeout_epoch;         // a bounded wait gave up during this epoch
+    uint32_t *barrier_words;         // [2] grid-barrier counters of the single-launch layout
+    // pinned host mirror of {P, NT, bad_epoch, timeout_epoch}
     int64_t *host_mirror;
 };

@@ -163,10 +163,11 @@ SEP_API sep_status sep_handle_create(int64_t max_tokens, int top_k, int num_expe
 /* Fills *info (host struct) for the handle's current layout.  Never blocks. */
 SEP_API sep_status sep_handle_info(const sep_handle *handle, sep_layout_info *info);
 
-/* Waits for `stream`, then reads the exact pool size and the device error word
+/* Waits for `stream`, then reads the exact pool size and the device error words
  * of the current layout into the handle (afterwards capacity checks use the
  * exact size).  Returns SEP_ERR_BAD_EXPERT_ID if the layout met an expert id
- * >= num_experts, else SEP_OK. */
+ * >= num_experts, SEP_ERR_TIMEOUT if the layout's grid barrier or a dispatch
+ * or combine of this layout gave up a bounded wait, else SEP_OK. */
 SEP_API sep_status sep_handle_sync(sep_handle *handle, void *stream);
 
 /*
