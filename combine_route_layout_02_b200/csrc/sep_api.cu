@@ -208,6 +208,11 @@ int64_t needed_rows(const sep_handle *h)
 
 namespace sep {
 
+sep_status set_error(sep_status st, const char *msg)
+{
+    return fail(st, "%s", msg);
+}
+
 int device_sm_count()
 {
     static int cached[64] = {0};

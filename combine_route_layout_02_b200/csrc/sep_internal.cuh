@@ -159,6 +159,9 @@ cudaError_t preload_consumer_kernels();
 
 int device_sm_count();
 
+// Records msg as the calling thread's last error and returns st.
+sep_status set_error(sep_status st, const char *msg);
+
 // Resident CTAs per SM for a kernel at a block size (cached per kernel).
 int occupancy_blocks_per_sm(const void *kernel, int threads, size_t smem);
 

@@ -44,6 +44,16 @@ class LayoutInfo(ctypes.Structure):
     ]
 
 
+class LayoutArrays(ctypes.Structure):
+    """Mirror of sep_layout_arrays (caller-owned outputs of sep_layout_noalloc)."""
+    _fields_ = [
+        ("expert_counts", _P), ("owner_counts", _P), ("expert_pool_block_offset", _P),
+        ("owner_pool_row_offset", _P), ("tile_expert", _P), ("pool_arrival_target", _P),
+        ("src_pool_row", _P), ("pool_recv_token", _P), ("pool_recv_slot", _P), ("sizes", _P),
+        ("status", _P), ("max_pool_rows", _i64), ("max_tiles", _i64),
+    ]
+
+
 # (name, restype, argtypes) of every entry point declared in include/sep.h
 _SIGNATURES = [
     ("sep_layout", _i32, [_P, _i32, _i64, _i32, _i32, _i32, _i32, _u32, _P, ctypes.POINTER(_P)]),
@@ -57,13 +67,12 @@ _SIGNATURES = [
     ("sep_last_error", ctypes.c_char_p, []),
     ("sep_status_string", ctypes.c_char_p, [_i32]),
     ("sep_abi_version", _i32, []),
+    ("sep_layout_noalloc", _i32, [_P, _i32, _i64, _i32, _i32, _i32, _i32, ctypes.POINTER(LayoutArrays), _P]),
 ]
 
 
 def _load() -> ctypes.CDLL:
-    path = _build.LIB
-    if not os.path.exists(path):
-        _build.build()
+    path = _build.build()          # compiles only when missing or older than its sources
     lib = ctypes.CDLL(path)
     for name, res, args in _SIGNATURES:
         fn = getattr(lib, name)
@@ -245,3 +254,23 @@ def alloc_pool(handle: Handle, hidden: int, payload: str = "bf16", scale: str = 
     recv = torch.empty(rows, hidden, dtype=torch.uint8, device="cuda")
     sdt = torch.uint8 if scale == "ue8m0" else torch.float32
     return recv, torch.empty(rows, hidden // 128, dtype=sdt, device="cuda")
+
+
+def sep_layout_noalloc(topk_idx: torch.Tensor, num_experts: int, num_owners: int, block_m: int,
+                       arrays: dict, stream=None) -> None:
+    """Layout into caller-owned device tensors without any allocation by the library.
+
+    ``arrays`` maps the sep_layout_arrays field names to device tensors
+    (int32, except ``sizes`` int64 [2] and ``status`` int32 [2]); the pool-row
+    and tile capacities are taken from the tensors' lengths."""
+    if topk_idx.dtype not in (torch.int32, torch.int64) or topk_idx.dim() != 2:
+        raise ValueError("topk_idx must be a [T, k] int32 or int64 tensor")
+    T, k = topk_idx.shape
+    la = LayoutArrays()
+    for name, _ in LayoutArrays._fields_[:11]:
+        setattr(la, name, _ptr(arrays[name]).value)
+    la.max_pool_rows = min(arrays["pool_recv_token"].numel(), arrays["pool_recv_slot"].numel())
+    la.max_tiles = min(arrays["tile_expert"].numel(), arrays["pool_arrival_target"].numel())
+    _check(_lib.sep_layout_noalloc(_ptr(topk_idx) if T else ctypes.c_void_p(None), topk_idx.element_size(),
+                                   T, k, num_experts, num_owners, block_m, ctypes.byref(la), _stream(stream)),
+           "sep_layout_noalloc")

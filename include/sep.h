@@ -278,6 +278,64 @@ SEP_API const char *sep_status_string(sep_status status);
 /* SEP_ABI_VERSION of the library. */
 SEP_API int sep_abi_version(void);
 
+/*
+ * sep_layout_noalloc — the routing layout for callers that cannot allocate.
+ *
+ * Not an operation of the pages: it computes exactly what sep_layout computes
+ * (counts, pool offsets, tile tables, stable slot maps), into arrays the caller
+ * owns, and allocates nothing: no cudaMalloc/cudaMallocAsync/cudaFree, no
+ * host allocation, no handle.  It exists for callers that must not allocate
+ * device memory on this path: a serving runtime that has already handed all
+ * of HBM to its own pool (KV cache and expert workspaces) and forbids further
+ * cudaMalloc, code that runs where an allocation would synchronise the device
+ * or fragment a caching allocator, and callers that need a fixed memory
+ * footprint known at start-up.
+ *
+ * Its working memory (per-chunk expert histograms and prefix sums, and a
+ * grid-barrier counter) is one file-scope __device__ array of 256 KB + 256 B
+ * that every GPU which loads the library holds until the process exits.  Hence
+ * the limits: num_experts <= 256 and num_tokens * top_k <= 2^21 (2 097 152);
+ * larger sizes are rejected with SEP_ERR_INVALID_ARG.  All calls share that
+ * array: calls that overlap on the GPU (two streams, or two threads) race and
+ * give wrong results; order them.  The call clears the barrier counter and
+ * the status words before its kernel; everything else in the array is
+ * overwritten before it is read.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress, with that device current);
+ * make that first call before any stream capture.  No dispatch or combine
+ * goes with it (those take a handle); the maps it writes are the ones
+ * sep_layout would put in a handle.
+ *
+ *  topk_idx, idx_bytes, num_tokens, top_k, num_experts, num_owners, block_m:
+ *      as for sep_layout.
+ *  out      host struct of caller-owned device arrays (below).
+ *  stream   the stream the work is enqueued on; nothing is synchronised.
+ * Errors: SEP_ERR_INVALID_ARG (sizes, limits, pointers, alignment),
+ * SEP_ERR_CAPACITY (an output array shorter than the worst case for T),
+ * SEP_ERR_CUDA.  Device-side findings go to out->status: status[0] = 1 if an
+ * expert id >= num_experts was met (the entry is skipped, as in sep_layout),
+ * status[1] = 1 if the kernel's grid barrier gave up its bounded wait.
+ */
+typedef struct sep_layout_arrays {
+    int32_t *expert_counts;            /* [E] */
+    int32_t *owner_counts;             /* [R] */
+    int32_t *expert_pool_block_offset; /* [E+1] */
+    int32_t *owner_pool_row_offset;    /* [R+1] */
+    int32_t *tile_expert;              /* [max_tiles] */
+    int32_t *pool_arrival_target;      /* [max_tiles] */
+    int32_t *src_pool_row;             /* [T, k] */
+    int32_t *pool_recv_token;          /* [max_pool_rows] */
+    int32_t *pool_recv_slot;           /* [max_pool_rows] */
+    int64_t *sizes;                    /* [2] {P, NT} */
+    uint32_t *status;                  /* [2] see above */
+    int64_t max_pool_rows;             /* rows of the pool_recv_* arrays: >= the worst case
+                                          N_a + min(E, N_a) * (block_m - 1), rounded up to block_m */
+    int64_t max_tiles;                 /* entries of the tile arrays: >= max_pool_rows / block_m */
+} sep_layout_arrays;
+
+SEP_API sep_status sep_layout_noalloc(const void *topk_idx, int idx_bytes, int64_t num_tokens, int top_k,
+                                      int num_experts, int num_owners, int block_m,
+                                      const sep_layout_arrays *out, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
