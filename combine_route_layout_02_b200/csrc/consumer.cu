@@ -8,7 +8,7 @@
 // order belongs to CTA n % gridDim.x.  Thread 0 waits (acquire load, bounded by
 // %globaltimer and a poll budget, with nanosleep back-off), the CTA barrier
 // passes the acquired view to the other threads, and the CTA copies the tile's
-// valid rows with L2-coherent loads.  When a wait gives up, status[0] becomes
+// valid rows with L2-coherent loads, eight 16-byte loads in flight per lane.  When a wait gives up, status[0] becomes
 // SEP_ERR_TIMEOUT; every CTA then stops waiting and counts its remaining tiles
 // in status[1].  No wait is unbounded.
 #include "sep_internal.cuh"
@@ -18,6 +18,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kMaxExperts = 1024;
+constexpr int kCopyUnroll = 8;       // 16-byte loads in flight per lane while copying a row
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *ptr)
 {
@@ -81,8 +82,20 @@ __global__ void __launch_bounds__(kThreads) consume_tiles_kernel(ConsumeParams p
                         continue;                        // padding: never read
                     const uint4 *src = reinterpret_cast<const uint4 *>(p.src) + row * vecs;
                     uint4 *dst = reinterpret_cast<uint4 *>(p.dst) + row * vecs;
-                    for (int64_t v = lane; v < vecs; v += 32)
-                        dst[v] = __ldcg(src + v);
+                    for (int64_t v0 = lane; v0 < vecs; v0 += 32 * kCopyUnroll) {
+                        uint4 buf[kCopyUnroll];
+#pragma unroll
+                        for (int u = 0; u < kCopyUnroll; ++u) {
+                            const int64_t v = v0 + u * 32;
+                            buf[u] = v < vecs ? __ldcg(src + v) : make_uint4(0, 0, 0, 0);
+                        }
+#pragma unroll
+                        for (int u = 0; u < kCopyUnroll; ++u) {
+                            const int64_t v = v0 + u * 32;
+                            if (v < vecs)
+                                dst[v] = buf[u];
+                        }
+                    }
                 }
             } else if (threadIdx.x == 0) {
                 atomicAdd(p.status + 1, 1u);

@@ -48,6 +48,17 @@ __device__ __forceinline__ void st_release_gpu(unsigned *ptr, unsigned v)
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
 }
 
+// Store of one 16-byte piece of a pool row.
+constexpr bool kStreamingStores = false;
+__device__ __forceinline__ void st_row(uint4 *ptr, uint4 v)
+{
+    if (kStreamingStores)
+        asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(ptr), "r"(v.x), "r"(v.y), "r"(v.z),
+                     "r"(v.w) : "memory");
+    else
+        *ptr = v;
+}
+
 // Publish the rows this warp just finished for token t (one arrival per row).
 __device__ __forceinline__ void publish_rows(const DispatchParams &p, int my_row, int lane)
 {
@@ -95,7 +106,7 @@ __global__ void __launch_bounds__(kWarps * 32) dispatch_bf16_kernel(DispatchPara
                 for (int u = 0; u < UNROLL; ++u) {
                     const int v = v0 + u * 32 + lane;
                     if (v < v_end)
-                        dst[v] = buf[u];
+                        st_row(dst + v, buf[u]);
                 }
             }
         }

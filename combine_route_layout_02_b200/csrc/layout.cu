@@ -335,19 +335,23 @@ __global__ void __launch_bounds__(kWarps * 32) layout_assign_kernel(LayoutParams
 
 // ------------------------------------------------------- single launch
 //
-// The same three steps in one cooperative launch (every CTA resident), split
-// by two grid barriers:
-//   A  count this CTA's chunk; the CTA's histogram column -> wchunk_hist
-//   B  warp w of CTA c scans the chunk column of expert c*8+w (+ multiples of
-//      8*G): per-chunk exclusive bases -> wchunk_base, n_e -> expert_counts
-//   C  every CTA scans ceil(n_e/B) over experts in shared memory, turns its
-//      warp counts from A into cursors and assigns its chunk; CTA 0 writes
-//      the offsets, sizes and owner arrays; tile tables and padding rows
-//      are spread over CTAs as in the three-launch path.
-// Each barrier is a bounded spin on an arrival counter; launches of odd and
-// even epochs use different counters, and each launch zeroes the one the next
-// launch will use.  A barrier that gives up records the epoch in the handle's
-// timeout word and the kernel returns (sep_handle_sync reports it).
+// The same computation in one cooperative launch (every CTA resident) with a
+// single grid barrier:
+//   A  count this CTA's chunk per warp (shared memory); write the CTA's row
+//      hist[c][0..E) of a chunk-major table whose row stride is E rounded up
+//      to 4 (the padding is written as zeros)
+//   -- grid barrier --
+//   B  every CTA reads the whole table with 16-byte loads (one L2 round trip
+//      at 128 chunks x 128 experts) and reduces it to n_e over all chunks and
+//      to its own prefix over the chunks before it; the scan of
+//      ceil(n_e / BLOCK_M) over experts follows in shared memory; CTA 0
+//      writes the counts, offsets, sizes and owner arrays
+//   C  the warp counts of A become cursors and the chunk is walked again
+//   D  tile tables and padding rows, experts spread over CTAs
+// The barrier arrives with red.release and waits with ld.acquire, bounded; a
+// barrier that gives up records the epoch in the handle's timeout word and the
+// kernel returns (sep_handle_sync reports it).  Launches of odd and even epochs
+// use different counters, and each launch zeroes the one the next will use.
 
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *ptr)
 {
@@ -363,15 +367,14 @@ __device__ __forceinline__ uint64_t global_ns()
     return t;
 }
 
-// All CTAs arrive on *counter; returns false (in every thread of the CTA) if
-// the counter did not reach target within the limit.
+// All CTAs arrive on *counter; false (in every thread of the CTA) if the
+// counter did not reach target within the limit.
 __device__ __forceinline__ bool grid_barrier(const LayoutParams &p, unsigned *counter, unsigned target,
                                              int *s_flag)
 {
     __syncthreads();
     if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(counter, 1u);
+        asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(counter), "r"(1u) : "memory");
         bool ok = false;
         const uint64_t t0 = global_ns();
         for (uint32_t it = 0; it < (1u << 22); ++it) {
@@ -381,9 +384,8 @@ __device__ __forceinline__ bool grid_barrier(const LayoutParams &p, unsigned *co
             }
             if (global_ns() - t0 > 200000000ull)
                 break;
-            __nanosleep(64);
+            __nanosleep(32);
         }
-        __threadfence();
         if (!ok)
             atomicMax(p.timeout_epoch, p.epoch);
         *s_flag = ok ? 1 : 0;
@@ -392,30 +394,36 @@ __device__ __forceinline__ bool grid_barrier(const LayoutParams &p, unsigned *co
     return *s_flag != 0;
 }
 
+constexpr int kFusedThreads = kWarps * 32;
+constexpr int kRedInts = 1024;               // per reduction table: row groups x padded experts
+
 template <typename IdxT>
-__global__ void __launch_bounds__(kWarps * 32) layout_fused_kernel(LayoutParams p)
+__global__ void __launch_bounds__(kFusedThreads) layout_fused_kernel(LayoutParams p)
 {
-    extern __shared__ int32_t sm[];          // [kWarps][E] counts/cursors, [E+1] offsets, [R] owner tokens
+    extern __shared__ __align__(16) int32_t sm[];
     __shared__ int s_flag;
-    __shared__ int s_part[kWarps * 32];
-    int32_t *s_cnt = sm;
-    int32_t *s_off = sm + kWarps * p.E;
-    int32_t *s_own = s_off + p.E + 1;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int c = blockIdx.x;
-    const int G = gridDim.x;
+    __shared__ int s_part[kWarps];
     const int E = p.E, nc = p.num_wchunks;
+    const int hs = (E + 3) & ~3;                         // padded row stride of the chunk table
+    int32_t *s_red = sm;                                 // [2][kRedInts], read and written as int4: first
+    int32_t *s_cnt = s_red + 2 * kRedInts;               // [kWarps][E]
+    int32_t *s_off = s_cnt + kWarps * E;                 // [E+1]
+    int32_t *s_tot = s_off + E + 1;                      // [E]
+    int32_t *s_pre = s_tot + E;                          // [E]
+    int32_t *s_own = s_pre + E;                          // [R]
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x, G = gridDim.x;
     const IdxT *idx = static_cast<const IdxT *>(p.topk_idx);
     allow_dependents();
     unsigned *counter = p.barrier_words + (p.epoch & 1u);
-    if (c == 0 && threadIdx.x == 0)
+    if (c == 0 && tid == 0)
         p.barrier_words[(p.epoch & 1u) ^ 1u] = 0u;      // the next launch's counter
     if (c == 0)
-        for (int r = threadIdx.x; r < p.R; r += blockDim.x)
+        for (int r = tid; r < p.R; r += blockDim.x)
             p.owner_token_counts[r] = 0;
 
     // A. count
-    for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x)
+    for (int i = tid; i < kWarps * E; i += blockDim.x)
         s_cnt[i] = 0;
     __syncthreads();
     const int64_t a0 = ((int64_t)c * kWarps + warp) * 32 * p.rounds;
@@ -424,41 +432,75 @@ __global__ void __launch_bounds__(kWarps * 32) layout_fused_kernel(LayoutParams 
     if (__any_sync(kFullMask, bad) && lane == 0)
         atomicMax(p.bad_epoch, p.epoch);
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    for (int e = tid; e < hs; e += blockDim.x) {
         int sum = 0;
+        if (e < E) {
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w)
-            sum += s_cnt[w * E + e];
-        p.wchunk_hist[(int64_t)e * nc + c] = sum;
+            for (int w = 0; w < kWarps; ++w)
+                sum += s_cnt[w * E + e];
+        }
+        p.wchunk_hist[(int64_t)c * hs + e] = sum;
     }
     if (!grid_barrier(p, counter, (unsigned)G, &s_flag))
         return;
 
-    // B. per-expert scan over chunks, one warp per expert
-    for (int e = c * kWarps + warp; e < E; e += G * kWarps) {
-        const int32_t *col = p.wchunk_hist + (int64_t)e * nc;
-        int32_t *bcol = p.wchunk_base + (int64_t)e * nc;
-        int running = 0;
-        for (int c0 = 0; c0 < nc; c0 += 32) {
-            const int cc = c0 + lane;
-            const int x = cc < nc ? __ldcg(col + cc) : 0;     // written by other CTAs
-            const int incl = warp_inclusive_scan(x, lane);
-            if (cc < nc)
-                bcol[cc] = running + incl - x;
-            running += __shfl_sync(kFullMask, incl, 31);
+    // B. totals and this chunk's prefix, from the whole table
+    {
+        const int cols = hs / 4;                         // int4 columns per row
+        const int groups = kFusedThreads / cols > 0 ? kFusedThreads / cols : 1;
+        for (int q0 = 0; q0 < cols; q0 += kFusedThreads) {   // more than 1024 experts never happens
+            const int q = q0 + tid % min(cols, kFusedThreads);
+            const int g = tid / min(cols, kFusedThreads);
+            int4 tot = make_int4(0, 0, 0, 0), pre = make_int4(0, 0, 0, 0);
+            if (g < groups && q < cols) {
+                const int4 *col = reinterpret_cast<const int4 *>(p.wchunk_hist) + q;
+                int r = g;
+                for (; r + 3 * groups < nc; r += 4 * groups) {
+                    int4 v[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        v[u] = __ldcg(col + (int64_t)(r + u * groups) * cols);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        tot.x += v[u].x; tot.y += v[u].y; tot.z += v[u].z; tot.w += v[u].w;
+                        if (r + u * groups < c) {
+                            pre.x += v[u].x; pre.y += v[u].y; pre.z += v[u].z; pre.w += v[u].w;
+                        }
+                    }
+                }
+                for (; r < nc; r += groups) {
+                    const int4 v = __ldcg(col + (int64_t)r * cols);
+                    tot.x += v.x; tot.y += v.y; tot.z += v.z; tot.w += v.w;
+                    if (r < c) {
+                        pre.x += v.x; pre.y += v.y; pre.z += v.z; pre.w += v.w;
+                    }
+                }
+                reinterpret_cast<int4 *>(s_red)[g * cols + q - q0] = tot;
+                reinterpret_cast<int4 *>(s_red + kRedInts)[g * cols + q - q0] = pre;
+            }
+            __syncthreads();
+            for (int e = tid; e < min(4 * (cols - q0), 4 * kFusedThreads); e += blockDim.x) {
+                const int ee = 4 * q0 + e;
+                if (ee < E) {
+                    int t = 0, b = 0;
+                    for (int gg = 0; gg < groups; ++gg) {
+                        t += s_red[gg * 4 * min(cols, kFusedThreads) + e];
+                        b += s_red[kRedInts + gg * 4 * min(cols, kFusedThreads) + e];
+                    }
+                    s_tot[ee] = t;
+                    s_pre[ee] = b;
+                }
+            }
+            __syncthreads();
         }
-        if (lane == 0)
-            p.expert_counts[e] = running;
     }
-    if (!grid_barrier(p, counter, 2u * (unsigned)G, &s_flag))
-        return;
 
-    // C. tile offsets over experts (each thread sums a run of experts)
+    // tile offsets over experts (each thread a run of experts), in shared memory
     const int per = (E + blockDim.x - 1) / blockDim.x;
-    const int e0 = threadIdx.x * per;
+    const int e0 = tid * per;
     int local = 0;
     for (int e = e0; e < min(E, e0 + per); ++e)
-        local += (__ldcg(p.expert_counts + e) + p.B - 1) / p.B;
+        local += (s_tot[e] + p.B - 1) / p.B;
     const int incl = warp_inclusive_scan(local, lane);
     if (lane == 31)
         s_part[warp] = incl;
@@ -473,32 +515,36 @@ __global__ void __launch_bounds__(kWarps * 32) layout_fused_kernel(LayoutParams 
     int run = s_part[warp] + incl - local;
     for (int e = e0; e < min(E, e0 + per); ++e) {
         s_off[e] = run;
-        run += (__ldcg(p.expert_counts + e) + p.B - 1) / p.B;
+        run += (s_tot[e] + p.B - 1) / p.B;
     }
-    if (threadIdx.x == blockDim.x - 1)
-        s_off[E] = s_part[warp] + incl;                   // last thread holds the grand total
+    if (tid == blockDim.x - 1)
+        s_off[E] = s_part[warp] + incl;                  // the last thread holds the grand total
     __syncthreads();
     if (c == 0) {
-        for (int e = threadIdx.x; e <= E; e += blockDim.x)
+        for (int e = tid; e <= E; e += blockDim.x) {
             p.expert_pool_block_offset[e] = s_off[e];
-        if (threadIdx.x == 0) {
+            if (e < E)
+                p.expert_counts[e] = s_tot[e];
+        }
+        if (tid == 0) {
             p.sizes[0] = (int64_t)s_off[E] * p.B;
             p.sizes[1] = s_off[E];
         }
         const int E_loc = E / p.R;
-        for (int r = threadIdx.x; r <= p.R; r += blockDim.x) {
+        for (int r = tid; r <= p.R; r += blockDim.x) {
             p.owner_pool_row_offset[r] = s_off[r * E_loc] * p.B;
             if (r < p.R) {
                 int sum = 0;
                 for (int q = r * E_loc; q < (r + 1) * E_loc; ++q)
-                    sum += __ldcg(p.expert_counts + q);
+                    sum += s_tot[q];
                 p.owner_counts[r] = sum;
             }
         }
     }
-    // warp counts -> cursors, then the assignment walk
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int cur = s_off[e] * p.B + __ldcg(p.wchunk_base + (int64_t)e * nc + c);
+
+    // C. warp counts -> cursors, then the assignment walk
+    for (int e = tid; e < E; e += blockDim.x) {
+        int cur = s_off[e] * p.B + s_pre[e];
 #pragma unroll
         for (int w = 0; w < kWarps; ++w) {
             const int n = s_cnt[w * E + e];
@@ -540,28 +586,29 @@ __global__ void __launch_bounds__(kWarps * 32) layout_fused_kernel(LayoutParams 
             }
         }
     }
-    // tile tables and padding rows; experts spread over CTAs
+
+    // D. tile tables and padding rows; experts spread over CTAs
     for (int e = c; e < E; e += G) {
         const int t0 = s_off[e], t1 = s_off[e + 1];
-        const int n = __ldcg(p.expert_counts + e);
-        for (int i = threadIdx.x; i < t1 - t0; i += blockDim.x) {
+        const int n = s_tot[e];
+        for (int i = tid; i < t1 - t0; i += blockDim.x) {
             p.tile_expert[t0 + i] = e;
             p.pool_arrival_target[t0 + i] = min(p.B, n - i * p.B);
             p.pool_arrival_count[t0 + i] = 0u;
         }
         const int64_t r1 = (int64_t)t1 * p.B;
-        for (int64_t row = (int64_t)t0 * p.B + n + threadIdx.x; row < r1; row += blockDim.x) {
+        for (int64_t row = (int64_t)t0 * p.B + n + tid; row < r1; row += blockDim.x) {
             p.pool_recv_token[row] = -1;
             p.pool_recv_slot[row] = -1;
         }
     }
     // optional: which owners each token reaches, and per-owner token counts
     if (p.is_token_in_rank != nullptr) {
-        for (int r = threadIdx.x; r < p.R; r += blockDim.x)
+        for (int r = tid; r < p.R; r += blockDim.x)
             s_own[r] = 0;
         __syncthreads();
         const int E_loc = E / p.R;
-        for (int64_t t = (int64_t)c * blockDim.x + threadIdx.x; t < p.T; t += (int64_t)G * blockDim.x) {
+        for (int64_t t = (int64_t)c * blockDim.x + tid; t < p.T; t += (int64_t)G * blockDim.x) {
             uint8_t *dst = p.is_token_in_rank + t * p.R;
             for (int r = 0; r < p.R; ++r) {
                 int in = 0;
@@ -575,7 +622,7 @@ __global__ void __launch_bounds__(kWarps * 32) layout_fused_kernel(LayoutParams 
             }
         }
         __syncthreads();
-        for (int r = threadIdx.x; r < p.R; r += blockDim.x)
+        for (int r = tid; r < p.R; r += blockDim.x)
             if (s_own[r])
                 atomicAdd(&p.owner_token_counts[r], s_own[r]);
     }
@@ -586,20 +633,29 @@ cudaError_t launch_layout_t(const LayoutParams &p, cudaStream_t s)
 {
     const int chunks = p.num_wchunks;
     const size_t smem_count = (size_t)kWarps * p.E * sizeof(int32_t);
-    const size_t smem_fused = smem_count + (size_t)(p.E + 1 + p.R) * sizeof(int32_t);
+    const size_t smem_fused = (size_t)(kWarps * p.E + 3 * p.E + 1 + 2 * kRedInts + p.R) * sizeof(int32_t);
     if (chunks > 0) {
         // single launch when every CTA can be resident at once
-        int per_sm = 0;
-        int dev = 0, sms = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess &&
+        static bool attr_set[64] = {false};                  // function attributes are per device
+        int dev = 0, sms = 0, per_sm = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+            return cudaErrorInvalidDevice;
+        if (!attr_set[dev]) {
+            const cudaError_t e = cudaFuncSetAttribute(layout_fused_kernel<IdxT>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+            if (e != cudaSuccess)
+                return e;
+            attr_set[dev] = true;
+        }
+        if (
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
-            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layout_fused_kernel<IdxT>, kWarps * 32,
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layout_fused_kernel<IdxT>, kFusedThreads,
                                                           smem_fused) == cudaSuccess &&
             chunks <= per_sm * sms) {
             LayoutParams q = p;
             void *args[] = {&q};
             return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(layout_fused_kernel<IdxT>),
-                                               dim3(chunks), dim3(kWarps * 32), args, smem_fused, s);
+                                               dim3(chunks), dim3(kFusedThreads), args, smem_fused, s);
         }
         layout_count_kernel<IdxT><<<chunks, kWarps * 32, smem_count, s>>>(p);
     }

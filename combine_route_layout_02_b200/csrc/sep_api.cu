@@ -149,7 +149,7 @@ sep_status create(int64_t T_cap, int k, int E, int R, int B, uint32_t flags, cud
     const size_t o_spr = carve(&off, (size_t)Na1 * 4);
     const size_t o_tok = carve(&off, (size_t)P1 * 4);
     const size_t o_slot = carve(&off, (size_t)P1 * 4);
-    const size_t o_hist = carve(&off, (size_t)h->wchunk_cap * E * 4);
+    const size_t o_hist = carve(&off, (size_t)h->wchunk_cap * ((E + 3) / 4 * 4) * 4);   // rows padded to 4
     const size_t o_base = carve(&off, (size_t)h->wchunk_cap * E * 4);
     const size_t o_in = (flags & SEP_LAYOUT_TOKEN_IN_OWNER) ? carve(&off, (size_t)(T_cap > 0 ? T_cap : 1) * R) : 0;
 
@@ -197,6 +197,35 @@ sep_status create(int64_t T_cap, int k, int E, int R, int B, uint32_t flags, cud
     *out = h;
     return SEP_OK;
 }
+
+// Work items of the dispatch and combine kernels are (token, segment of a
+// row).  A row of `units` warp-steps is split so that there are at least
+// `want_warps` items and at least `min_segs` segments per row; returns the
+// segment count and the steps per segment.
+void split_rows(int64_t T, int64_t units, int64_t want_warps, int64_t min_segs, int *segs, int64_t *steps)
+{
+    int64_t n = (want_warps + T - 1) / T;
+    if (n < min_segs)
+        n = min_segs;
+    if (n > units)
+        n = units;
+    if (n < 1)
+        n = 1;
+    *steps = (units + n - 1) / n;
+    *segs = (int)((units + *steps - 1) / *steps);
+}
+
+// Row splitting.  A bf16 dispatch step is 128 vectors of 16 bytes (one pass of
+// the kernel's 4-deep unroll); without tile publication every step is its own
+// work item, so the items divide finely over the waves of CTAs (measured
+// faster than whole rows per warp).  With tile publication a row stays on one
+// warp where possible, since every item pays a fence and one arrival per row.
+// FP8 steps are 512 channels; combine steps are 32 vectors.
+constexpr int64_t kDispatchStepVecs = 128;
+constexpr int64_t kDispatchMinSegs = 1 << 20;
+constexpr int64_t kDispatchPublishMinSegs = 1;
+constexpr int64_t kDispatchFp8MinSegs = 7;
+constexpr int64_t kCombineMinSegs = 1;
 
 // Rows a buffer must hold for the handle's current layout.
 int64_t needed_rows(const sep_handle *h)
@@ -503,16 +532,11 @@ sep_status sep_dispatch(sep_handle *h, const void *x, int64_t hidden, int payloa
     p.error_epoch = h->timeout_epoch;
     p.epoch = h->epoch;
     // split a token row over several warps when there are too few tokens to fill the GPU
-    const int64_t units = fp8 ? (hidden + 511) / 512 : ((hidden / 8) + 31) / 32;   // warp-steps per row
-    const int64_t want_warps = (int64_t)num_sms * 32;
-    int64_t segs = (want_warps + h->T - 1) / h->T;
-    if (segs > units)
-        segs = units;
-    if (segs < 1)
-        segs = 1;
-    const int64_t steps = (units + segs - 1) / segs;
-    p.seg_len = (int)(fp8 ? steps : steps * 32);
-    p.segs = (int)((units + steps - 1) / steps);
+    const int64_t units = fp8 ? (hidden + 511) / 512 : ((hidden / 8) + kDispatchStepVecs - 1) / kDispatchStepVecs;
+    int64_t steps = 1;
+    const int64_t min_segs = fp8 ? kDispatchFp8MinSegs : (tile_ready ? kDispatchPublishMinSegs : kDispatchMinSegs);
+    split_rows(h->T, units, (int64_t)num_sms * 32, min_segs, &p.segs, &steps);
+    p.seg_len = (int)(fp8 ? steps : steps * kDispatchStepVecs);
     cudaError_t e = sep::launch_dispatch(p, payload, s, num_sms);
     return e == cudaSuccess ? SEP_OK : cuda_fail(e, "dispatch launch");
 }
@@ -558,15 +582,9 @@ sep_status sep_combine(const sep_handle *h, uint32_t layout_epoch, const void *y
     p.error_epoch = h->timeout_epoch;
     p.epoch = h->epoch;
     const int64_t units = ((hidden / 8) + 31) / 32;
-    const int64_t want_warps = (int64_t)num_sms * 32;
-    int64_t segs = (want_warps + h->T - 1) / h->T;
-    if (segs > units)
-        segs = units;
-    if (segs < 1)
-        segs = 1;
-    const int64_t steps = (units + segs - 1) / segs;
+    int64_t steps = 1;
+    split_rows(h->T, units, (int64_t)num_sms * 32, kCombineMinSegs, &p.segs, &steps);
     p.seg_len = (int)(steps * 32);
-    p.segs = (int)((units + steps - 1) / steps);
     cudaError_t e = sep::launch_combine(p, s, num_sms);
     return e == cudaSuccess ? SEP_OK : cuda_fail(e, "combine launch");
 }
