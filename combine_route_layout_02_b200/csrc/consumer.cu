@@ -109,6 +109,7 @@ __global__ void __launch_bounds__(kThreads) consume_tiles_kernel(ConsumeParams p
 
 cudaError_t launch_consume(const ConsumeParams &p, int num_ctas, cudaStream_t s)
 {
+    count_launch();
     consume_tiles_kernel<<<num_ctas, kThreads, 0, s>>>(p);
     return cudaGetLastError();
 }

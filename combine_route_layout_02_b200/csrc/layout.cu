@@ -654,14 +654,18 @@ cudaError_t launch_layout_t(const LayoutParams &p, cudaStream_t s)
             chunks <= per_sm * sms) {
             LayoutParams q = p;
             void *args[] = {&q};
+            count_launch();
             return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(layout_fused_kernel<IdxT>),
                                                dim3(chunks), dim3(kFusedThreads), args, smem_fused, s);
         }
+        count_launch();
         layout_count_kernel<IdxT><<<chunks, kWarps * 32, smem_count, s>>>(p);
     }
     const size_t smem_assign = smem_count + (size_t)p.R * sizeof(int32_t);
+    count_launch();
     layout_scan_kernel<<<1, kScanThreads, 0, s>>>(p);
     const int ablocks = max(chunks, min(p.E, 64));
+    count_launch();
     layout_assign_kernel<IdxT><<<ablocks, kWarps * 32, smem_assign, s>>>(p);
     return cudaGetLastError();
 }

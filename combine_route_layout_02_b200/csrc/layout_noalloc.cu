@@ -337,6 +337,7 @@ extern "C" sep_status sep_layout_noalloc(const void *topk_idx, int idx_bytes, in
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || p.chunks > per_sm * sms)
         return set_error(SEP_ERR_CUDA, "sep_layout_noalloc: the layout grid cannot be co-resident");
     void *args[] = {&p};
+    count_launch();
     e = cudaLaunchCooperativeKernel(kernel, dim3(p.chunks), dim3(kWarps * 32), args, 0, s);
     if (e != cudaSuccess)
         return set_error(SEP_ERR_CUDA, "sep_layout_noalloc: launch failed");

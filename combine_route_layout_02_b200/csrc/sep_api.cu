@@ -6,6 +6,7 @@
 // dropped ("DeepEP MoE dispatch/combine" blog, "Imbalance 决定 buffer 与尾延迟"),
 // and a handle carries the epoch of its routing so a combine against a
 // re-laid-out handle is refused (blog, "EPHandle" and "集成时的数据契约").
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -237,6 +238,12 @@ int64_t needed_rows(const sep_handle *h)
 
 namespace sep {
 
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
 sep_status set_error(sep_status st, const char *msg)
 {
     return fail(st, "%s", msg);
@@ -282,6 +289,8 @@ int occupancy_blocks_per_sm(const void *kernel, int threads, size_t smem)
 extern "C" {
 
 int sep_abi_version(void) { return SEP_ABI_VERSION; }
+
+uint64_t sep_launch_count(void) { return sep::g_launches.load(std::memory_order_relaxed); }
 
 const char *sep_last_error(void) { return g_err; }
 

@@ -127,10 +127,14 @@ __device__ __forceinline__ void allow_dependents()
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Kernels this process has launched through the library (sep_launch_count).
+void count_launch();
+
 template <typename... KArgs, typename... Args>
 cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                           Args... args)
 {
+    count_launch();
     if (!kUsePDL) {
         kernel<<<grid, block, smem, s>>>(args...);
         return cudaGetLastError();

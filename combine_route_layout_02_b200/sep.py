@@ -67,6 +67,7 @@ _SIGNATURES = [
     ("sep_last_error", ctypes.c_char_p, []),
     ("sep_status_string", ctypes.c_char_p, [_i32]),
     ("sep_abi_version", _i32, []),
+    ("sep_launch_count", _u64, []),
     ("sep_layout_noalloc", _i32, [_P, _i32, _i64, _i32, _i32, _i32, _i32, ctypes.POINTER(LayoutArrays), _P]),
 ]
 
@@ -274,3 +275,8 @@ def sep_layout_noalloc(topk_idx: torch.Tensor, num_experts: int, num_owners: int
     _check(_lib.sep_layout_noalloc(_ptr(topk_idx) if T else ctypes.c_void_p(None), topk_idx.element_size(),
                                    T, k, num_experts, num_owners, block_m, ctypes.byref(la), _stream(stream)),
            "sep_layout_noalloc")
+
+
+def sep_launch_count() -> int:
+    """Kernels this process has launched through the library."""
+    return int(_lib.sep_launch_count())

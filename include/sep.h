@@ -278,6 +278,10 @@ SEP_API const char *sep_status_string(sep_status status);
 /* SEP_ABI_VERSION of the library. */
 SEP_API int sep_abi_version(void);
 
+/* Number of CUDA kernels this process has launched through the library so far
+ * (all devices, all threads); memsets and copies are not counted. */
+SEP_API uint64_t sep_launch_count(void);
+
 /*
  * sep_layout_noalloc — the routing layout for callers that cannot allocate.
  *

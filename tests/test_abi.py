@@ -22,7 +22,7 @@ def test_library_is_built_for_sm100a_and_in_tree():
 
 def test_exports_match_header():
     declared = sep.declared_entry_points(HEADER)
-    assert len(declared) == 12
+    assert len(declared) == 13
     out = subprocess.run(["nm", "-D", "--defined-only", sep.library_path()], capture_output=True,
                          text=True, check=True).stdout
     exported = sorted(set(re.findall(r"\sT\s+(sep_\w+)$", out, flags=re.M)))
@@ -86,3 +86,7 @@ def test_no_cpu_fallback_in_the_binding():
     assert "oracle" not in src
     for op in ("index_select", "scatter", "torch.sum", ".sum(", "torch.matmul", "gather("):
         assert op not in src
+
+
+def test_launch_counter_starts_without_gpu_work():
+    assert sep.sep_launch_count() >= 0
