@@ -14,7 +14,9 @@
 // Two implementations:
 //  * register path: a warp owns (token, segment); the token's k row indices
 //    and weights are broadcast once into every lane's registers, then each lane
-//    walks its 16-byte columns issuing kRowBatch row loads at a time;
+//    walks its 16-byte columns issuing kRowBatch row loads at a time.  Tokens
+//    are taken in descending order, which reads first the pool rows a preceding
+//    dispatch wrote last (still resident in L2);
 //  * bulk path (used when k <= 32 and two stages of k rows fit in shared
 //    memory): warp 0 of a CTA bulk-loads the token's k rows into a two-stage
 //    shared-memory ring with cp.async.bulk (completion on an mbarrier), every
@@ -84,8 +86,10 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(CombineParams p)
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const uint4 *y = static_cast<const uint4 *>(p.y);
     for (int64_t it = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items; it += nwarps) {
-        const int64_t t = it / p.segs;
-        const int s = (int)(it - t * p.segs);
+        // tokens are visited in descending order: a dispatch that ran just before
+        // wrote the highest tokens' rows last, so those are the rows still in L2
+        const int64_t t = p.T - 1 - it / p.segs;
+        const int s = (int)(it - (p.T - 1 - t) * p.segs);
         const int v_begin = s * p.seg_len;
         const int v_end = min(V, v_begin + p.seg_len);
         const int my_row = lane < p.k ? __ldg(p.src_pool_row + t * p.k + lane) : -1;
