@@ -51,6 +51,8 @@ def load(path: str):
     L.oracle_quant_row.argtypes = [P, i64, i32, P, P, P]
     L.oracle_dequant_rows.argtypes = [P, i64, i64, i32, P, P, P]
     L.oracle_combine.argtypes = [P, i64, i64, i32, P, P, P]
+    L.oracle_dispatch_grads.argtypes = [P, i64, i64, i32, P, P, P, P, P]
+    L.oracle_combine_grads.argtypes = [P, i64, i64, i32, P, P]
     L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
     L.oracle_e4m3_encode.restype = ctypes.c_uint8
     L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
@@ -232,3 +234,28 @@ def f32_to_bf16(v, L=None) -> np.ndarray:
 
 def bf16_to_f32(u: np.ndarray) -> np.ndarray:
     return (np.asarray(u, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def dispatch_grads(grad_out, topk_weight, lay: Layout, y_pool=None, rows: int | None = None, fill: int = 0, L=None):
+    """(grad_y uint16 [rows, H], grad_w float64 [T, k] or None) (oracle_dispatch_grads)."""
+    g = as_u16(grad_out)
+    T, H = g.shape
+    rows = lay.num_pool_rows if rows is None else rows
+    gy = np.full((max(rows, 1), H), fill, np.uint16)
+    w = np.ascontiguousarray(np.asarray(topk_weight), dtype=np.float32)
+    if y_pool is not None:
+        yu = as_u16(y_pool)
+        gw = np.zeros((max(T, 1), lay.k), np.float64)
+        lib(L).oracle_dispatch_grads(_p(g), T, H, lay.k, _p(lay.src_pool_row), _p(w), _p(yu), _p(gy), _p(gw))
+        return gy[:rows], gw[:T]
+    lib(L).oracle_dispatch_grads(_p(g), T, H, lay.k, _p(lay.src_pool_row), _p(w), None, _p(gy), None)
+    return gy[:rows], None
+
+
+def combine_grads(grad_recv, lay: Layout, L=None) -> np.ndarray:
+    """grad_x uint16 [T, H] (oracle_combine_grads)."""
+    g = as_u16(grad_recv)
+    H = g.shape[1]
+    out = np.zeros((max(lay.T, 1), H), np.uint16)
+    lib(L).oracle_combine_grads(_p(g), lay.T, H, lay.k, _p(lay.src_pool_row), _p(out))
+    return out[:lay.T]

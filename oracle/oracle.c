@@ -376,3 +376,57 @@ void oracle_combine(const uint16_t *y_pool, int64_t T, int64_t H, int k,
             out[t * H + h] = oracle_f32_to_bf16(acc);
         }
 }
+
+/* ------------------------------------------------------------- backward */
+
+/*
+ * Backward of combine ("StreamEP" README, "What's in the box": dispatch_grads,
+ * the backward symmetry of combine).  With out[t] = sum_j w[t,j] * y[row(t,j)]:
+ *   grad_y[row(t,j)] = bf16( w[t,j] * grad_out[t] )      (fp32 product, one rounding)
+ *   grad_w[t,j]      = sum_h grad_out[t,h] * y[row(t,j),h] (fp64 here: the exact sum
+ *                                                            up to one final rounding)
+ * Masked assignments get no row and grad_w = 0.  grad_w may be NULL (then y may be too).
+ */
+void oracle_dispatch_grads(const uint16_t *grad_out, int64_t T, int64_t H, int k, const int32_t *src_pool_row,
+                           const float *topk_weight, const uint16_t *y_pool, uint16_t *grad_y, double *grad_w)
+{
+    for (int64_t t = 0; t < T; t++)
+        for (int j = 0; j < k; j++) {
+            int32_t row = src_pool_row[t * k + j];
+            float w = topk_weight[t * k + j];
+            double dot = 0.0;
+            if (row >= 0) {
+                for (int64_t h = 0; h < H; h++) {
+                    float g = oracle_bf16_to_f32(grad_out[t * H + h]);
+                    float prod = w * g;
+                    grad_y[(int64_t)row * H + h] = oracle_f32_to_bf16(prod);
+                    if (grad_w)
+                        dot += (double)g * (double)oracle_bf16_to_f32(y_pool[(int64_t)row * H + h]);
+                }
+            }
+            if (grad_w)
+                grad_w[t * k + j] = dot;
+        }
+}
+
+/*
+ * Backward of dispatch (combine_grads): with recv[row(t,j)] = x[t],
+ *   grad_x[t] = bf16( sum over valid j, ascending, of grad_recv[row(t,j)] )
+ * in fp32 with one rounding at the end: the combine of oracle_combine with
+ * every weight equal to 1.
+ */
+void oracle_combine_grads(const uint16_t *grad_recv, int64_t T, int64_t H, int k, const int32_t *src_pool_row,
+                          uint16_t *grad_x)
+{
+    for (int64_t t = 0; t < T; t++)
+        for (int64_t h = 0; h < H; h++) {
+            float acc = 0.0f;
+            for (int j = 0; j < k; j++) {
+                int32_t row = src_pool_row[t * k + j];
+                if (row < 0)
+                    continue;
+                acc = acc + oracle_bf16_to_f32(grad_recv[(int64_t)row * H + h]);
+            }
+            grad_x[t * H + h] = oracle_f32_to_bf16(acc);
+        }
+}

@@ -15,10 +15,10 @@
 
 All of these run on the CPU.
 """
+import ctypes
 import json
 import os
 import subprocess
-import tempfile
 
 import numpy as np
 import pytest
@@ -433,7 +433,7 @@ MUTANTS = [
     ("while (ldexp(448.0, e - 1) >= a)", "while (ldexp(448.0, e - 1) > a)"),               # boundary
     ("scales_u8[g] = (uint8_t)(E + 127);", "scales_u8[g] = (uint8_t)(E + 128);"),
     ("acc = acc + prod;", "acc = prod;"),                                                 # dropped term
-    ("topk_weight[t * k + j]", "topk_weight[t * k + (k - 1 - j)]"),                       # wrong operand
+    ("float prod = topk_weight[t * k + j] *", "float prod = topk_weight[t * k + (k - 1 - j)] *"),  # wrong operand
     ("if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u)))",
      "if (lower >= 0x8000u)"),                                                            # ties away in bf16
 ]
@@ -455,3 +455,121 @@ def test_planted_oracle_mistake_fails_a_pin(i, tmp_path):
 
 def test_unmutated_oracle_passes_the_compact_pins():
     assert not _pins_fail(None)
+
+
+# --------------------------------------------------------- backward pins
+
+def _bwd_case(seed, T=40, k=4, E=8, R=2, B=4, H=48):
+    rng = np.random.default_rng(seed)
+    idx = rng.integers(-1, E, size=(T, k))
+    lay = oracle.layout(idx, E, R, B)
+    w = rng.uniform(0.05, 1.0, size=(T, k)).astype(np.float32)
+    g = oracle.as_u16(W.random_x(T, H, seed=seed + 1))
+    y = oracle.as_u16(W.random_x(max(lay.num_pool_rows, 1), H, seed=seed + 2))
+    return lay, w, g, y
+
+
+def test_backward_golden_worked_example():
+    g = _golden("backward_worked_example.json")
+    lay = oracle.layout(np.array(g["topk_idx"]), g["E"], g["R"], g["B"])
+    gy, gw = oracle.dispatch_grads(_f32_to_bf16_bits(np.array(g["grad_out"], np.float32)),
+                                   np.array(g["topk_weight"], np.float32), lay,
+                                   y_pool=_f32_to_bf16_bits(np.array(g["y_pool"], np.float32)))
+    np.testing.assert_array_equal(oracle.bf16_to_f32(gy), np.array(g["grad_y"], np.float32))
+    np.testing.assert_array_equal(gw, np.array(g["grad_w"]))
+    gx = oracle.combine_grads(gy, lay)
+    np.testing.assert_array_equal(oracle.bf16_to_f32(gx), np.array(g["grad_x"], np.float32))
+
+
+def test_dispatch_grads_with_unit_weights_is_a_permutation():
+    lay, _, g, y = _bwd_case(3, k=1)
+    gy, _ = oracle.dispatch_grads(g, np.ones((lay.T, 1), np.float32), lay)
+    rows = lay.src_pool_row[:, 0]
+    ok = rows >= 0
+    np.testing.assert_array_equal(gy[rows[ok]], g[ok])
+
+
+def test_combine_grads_of_a_dispatch_counts_assignments():
+    """combine_grads(dispatch(x))[t] = n_t * x[t], n_t the token's valid
+    assignments (exact in bf16 for n_t a power of two)."""
+    rng = np.random.default_rng(4)
+    T, k, E = 64, 4, 8
+    idx = rng.integers(0, E, size=(T, k))
+    idx[::3, 1:] = -1                                    # n_t = 1 on every third token, else 4
+    lay = oracle.layout(idx, E, 2, 4)
+    x = W.random_x(T, 32, seed=5)
+    gx = oracle.bf16_to_f32(oracle.combine_grads(oracle.dispatch_bf16(x, lay), lay))
+    n = (idx >= 0).sum(1)[:, None].astype(np.float32)
+    np.testing.assert_array_equal(gx, x.float().numpy() * n)
+
+
+def test_backward_adjoint_identities():
+    """<grad_y, y> = <g, combine(y, w)> and sum w * grad_w = the same number;
+    <combine_grads(r), x> = <r, dispatch(x)> -- each to within the bf16 and
+    fp32 rounding the definitions allow."""
+    for seed in range(5):
+        lay, w, g, y = _bwd_case(10 + seed)
+        gy, gw = oracle.dispatch_grads(g, w, lay, y_pool=y)
+        gf = oracle.bf16_to_f32(g).astype(np.float64)
+        yf = oracle.bf16_to_f32(y).astype(np.float64)
+        rows = lay.src_pool_row
+        ok = rows >= 0
+        # <g, combine(y, w)> in fp64 from the pinned forward definition's terms
+        terms = np.where(ok[:, :, None], w.astype(np.float64)[:, :, None] * yf[np.where(ok, rows, 0)], 0.0)
+        lhs = float((gf * terms.sum(1)).sum())
+        valid_rows = lay.pool_recv_token >= 0
+        rhs = float((oracle.bf16_to_f32(gy).astype(np.float64)[valid_rows] * yf[valid_rows]).sum())
+        mag = float(np.abs(gf[:, None, :] * terms).sum())
+        assert abs(lhs - rhs) <= 2.0 ** -8 * mag + 1e-9
+        assert abs(float((w.astype(np.float64) * gw).sum()) - lhs) <= 1e-12 * mag + 1e-9
+        # dispatch / combine_grads adjoint
+        x = W.random_x(lay.T, y.shape[1], seed=seed)
+        r = oracle.as_u16(W.random_x(max(lay.num_pool_rows, 1), y.shape[1], seed=seed + 7))
+        d = oracle.bf16_to_f32(oracle.dispatch_bf16(x, lay)).astype(np.float64)
+        rf = oracle.bf16_to_f32(r).astype(np.float64)
+        lhs2 = float((oracle.bf16_to_f32(oracle.combine_grads(r, lay)).astype(np.float64)
+                      * x.float().numpy()).sum())
+        rhs2 = float((rf[valid_rows] * d[valid_rows]).sum())
+        mag2 = float(np.abs(rf[valid_rows] * d[valid_rows]).sum())
+        assert abs(lhs2 - rhs2) <= 2.0 ** -8 * mag2 * (lay.k + 1) + 1e-9
+
+
+BACKWARD_MUTANTS = [
+    ("float prod = w * g;", "float prod = g;"),                                     # weight dropped
+    ("float w = topk_weight[t * k + j];", "float w = topk_weight[t * k + (k - 1 - j)];"),
+    ("dot += (double)g * (double)oracle_bf16_to_f32(y_pool[(int64_t)row * H + h]);",
+     "dot += (double)g * (double)oracle_bf16_to_f32(y_pool[(int64_t)row * H + (H - 1 - h)]);"),
+    ("acc = acc + oracle_bf16_to_f32(grad_recv[(int64_t)row * H + h]);",
+     "acc = oracle_bf16_to_f32(grad_recv[(int64_t)row * H + h]);"),
+]
+
+
+@pytest.mark.parametrize("i", range(len(BACKWARD_MUTANTS)))
+def test_planted_backward_mistake_fails_a_pin(i, tmp_path):
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "oracle.c")).read()
+    old, new = BACKWARD_MUTANTS[i]
+    assert src.count(old) == 1, old
+    c = tmp_path / "m.c"
+    so = tmp_path / f"mb{i}.so"
+    c.write_text(src.replace(old, new))
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared",
+                           "-o", str(so), str(c), "-lm"])
+    L = oracle.load(str(so))
+    L.oracle_dispatch_grads.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int] + \
+        [ctypes.c_void_p] * 5
+    L.oracle_combine_grads.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
+                                       ctypes.c_void_p, ctypes.c_void_p]
+    g = _golden("backward_worked_example.json")
+    caught = False
+    try:
+        lay = oracle.layout(np.array(g["topk_idx"]), g["E"], g["R"], g["B"], L=L)
+        gy, gw = oracle.dispatch_grads(_f32_to_bf16_bits(np.array(g["grad_out"], np.float32)),
+                                       np.array(g["topk_weight"], np.float32), lay,
+                                       y_pool=_f32_to_bf16_bits(np.array(g["y_pool"], np.float32)), L=L)
+        np.testing.assert_array_equal(oracle.bf16_to_f32(gy), np.array(g["grad_y"], np.float32))
+        np.testing.assert_array_equal(gw, np.array(g["grad_w"]))
+        gx = oracle.combine_grads(gy, lay, L=L)
+        np.testing.assert_array_equal(oracle.bf16_to_f32(gx), np.array(g["grad_x"], np.float32))
+    except AssertionError:
+        caught = True
+    assert caught, f"backward mutant {i} passed the golden pin"
