@@ -9,20 +9,28 @@
 // rounded add (no fused multiply-add), starting at +0: exactly the fp32
 // arithmetic of the definition, so the result is bit-identical to it; the
 // final bf16 rounding is to nearest even.  Masked assignments (row < 0) are
-// skipped.
+// skipped.  With no weights (w == nullptr) every weight is 1: that is the
+// backward of dispatch, combine_grads (StreamEP README, "What's in the box"),
+// and 1 * y is exact, so it too is bit-identical to its definition.
 //
-// Two implementations:
-//  * register path: a warp owns (token, segment); the token's k row indices
-//    and weights are broadcast once into every lane's registers, then each lane
-//    walks its 16-byte columns issuing kRowBatch row loads at a time.  Tokens
-//    are taken in descending order, which reads first the pool rows a preceding
-//    dispatch wrote last (still resident in L2);
-//  * bulk path (used when k <= 32 and two stages of k rows fit in shared
-//    memory): warp 0 of a CTA bulk-loads the token's k rows into a two-stage
-//    shared-memory ring with cp.async.bulk (completion on an mbarrier), every
-//    thread waits on the barrier (bounded), reduces its columns from shared
-//    memory and stores the bf16 result; the stage is refilled with the CTA's
-//    next-but-one token after a CTA barrier.
+// A warp owns (token, segment); the token's k row indices and weights are
+// broadcast once into every lane's registers, then each lane walks its
+// 16-byte columns issuing kRowBatch row loads at a time.  Tokens are taken in
+// descending order, which reads first the pool rows a preceding dispatch wrote
+// last (still resident in L2).
+//
+// Gated combine (StreamEP README, opening section: the per-recv-token gate
+// y_done_per_token lets combine start on a token as soon as that token's
+// compute has drained).  The grid is persistent and bounded by the caller so
+// that the producer keeps SMs; tokens are taken in ascending order, the order
+// in which a tile-ordered producer finishes them.  Lane 0 waits (acquire load,
+// bounded by %globaltimer and a poll budget) for y_done[t] >= done_seq, the
+// warp barrier passes the acquired view to the other lanes, and the rows are
+// read through L2 (they are written by a kernel that is still running, so the
+// non-coherent path is not used).  A token without valid assignments is not
+// waited for (its output is +0).  A wait that gives up sets status[0] =
+// SEP_ERR_TIMEOUT; every warp then stops waiting and counts the tokens it did
+// not reduce in status[1].
 #include <cuda_bf16.h>
 
 #include "sep_internal.cuh"
@@ -31,12 +39,8 @@ namespace sep {
 namespace {
 
 constexpr int kWarps = 8;
-constexpr int kRowBatch = 4;         // rows loaded before they are summed (register path)
+constexpr int kRowBatch = 4;         // rows loaded before they are summed
 constexpr int kKMax = 8;             // row indices / weights held in registers
-constexpr bool kBulkCombine = false;
-constexpr int kBulkStages = 2;
-constexpr int kBulkThreads = 256;
-constexpr int kBulkMaxSmem = 200 * 1024;
 
 __device__ __forceinline__ uint4 ld_stream(const uint4 *ptr)
 {
@@ -45,6 +49,43 @@ __device__ __forceinline__ uint4 ld_stream(const uint4 *ptr)
         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
         : "l"(ptr));
     return v;
+}
+
+template <bool GATED>
+__device__ __forceinline__ uint4 ld_row(const uint4 *ptr)
+{
+    return GATED ? __ldcg(ptr) : ld_stream(ptr);
+}
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *ptr)
+{
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint64_t global_time_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// 1 once y_done[t] has reached done_seq; 0 if this or another warp gave up.
+__device__ int wait_token(const CombineParams &p, int64_t t)
+{
+    const uint64_t t0 = global_time_ns();
+    for (uint32_t polls = 0;; ++polls) {
+        if ((int32_t)(ld_acquire_gpu(p.y_done + t) - p.done_seq) >= 0)
+            return 1;
+        if (*reinterpret_cast<volatile const uint32_t *>(p.status) != 0u)
+            return 0;
+        if (polls >= p.max_polls || global_time_ns() - t0 > p.timeout_ns) {
+            atomicCAS(p.status, 0u, (uint32_t)SEP_ERR_TIMEOUT);
+            return 0;
+        }
+        __nanosleep(128);
+    }
 }
 
 __device__ __forceinline__ void accumulate_word(float &lo, float &hi, uint32_t word, float w)
@@ -74,8 +115,7 @@ __device__ __forceinline__ uint4 pack_out(const float *acc)
                       pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
 }
 
-// ------------------------------------------------------------ register path
-
+template <bool GATED>
 __global__ void __launch_bounds__(kWarps * 32) combine_kernel(CombineParams p)
 {
     grid_dependency_wait();
@@ -86,14 +126,26 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(CombineParams p)
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const uint4 *y = static_cast<const uint4 *>(p.y);
     for (int64_t it = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items; it += nwarps) {
-        // tokens are visited in descending order: a dispatch that ran just before
-        // wrote the highest tokens' rows last, so those are the rows still in L2
-        const int64_t t = p.T - 1 - it / p.segs;
-        const int s = (int)(it - (p.T - 1 - t) * p.segs);
+        // ungated, tokens are visited in descending order: a dispatch that ran just
+        // before wrote the highest tokens' rows last, so those are still in L2
+        const int64_t t = GATED ? it / p.segs : p.T - 1 - it / p.segs;
+        const int s = (int)(GATED ? it - t * p.segs : it - (p.T - 1 - t) * p.segs);
         const int v_begin = s * p.seg_len;
         const int v_end = min(V, v_begin + p.seg_len);
         const int my_row = lane < p.k ? __ldg(p.src_pool_row + t * p.k + lane) : -1;
-        const float my_w = lane < p.k ? __ldg(p.w + t * p.k + lane) : 0.f;
+        if (GATED && __any_sync(kFullMask, my_row >= 0)) {   // a token with no rows has nothing to wait for
+            int go = 0;
+            if (lane == 0) {
+                go = wait_token(p, t);
+                if (!go)
+                    atomicAdd(p.status + 1, 1u);
+            }
+            go = __shfl_sync(kFullMask, go, 0);
+            __syncwarp();
+            if (!go)
+                continue;
+        }
+        const float my_w = lane < p.k ? (p.w ? __ldg(p.w + t * p.k + lane) : 1.f) : 0.f;
         uint4 *out = static_cast<uint4 *>(p.out) + t * V;
         if (p.k <= kKMax) {
             int rows[kKMax];
@@ -110,7 +162,7 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(CombineParams p)
                     uint4 buf[kRowBatch];
 #pragma unroll
                     for (int u = 0; u < kRowBatch; ++u)
-                        buf[u] = rows[j0 + u] >= 0 ? ld_stream(y + (int64_t)rows[j0 + u] * V + v)
+                        buf[u] = rows[j0 + u] >= 0 ? ld_row<GATED>(y + (int64_t)rows[j0 + u] * V + v)
                                                    : make_uint4(0, 0, 0, 0);
 #pragma unroll
                     for (int u = 0; u < kRowBatch; ++u)
@@ -132,7 +184,7 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(CombineParams p)
                         const int j = j0 + u;
                         const int row = __shfl_sync(kFullMask, my_row, j & 31);
                         rows[u] = j < p.k ? row : -1;
-                        buf[u] = (rows[u] >= 0 && act) ? ld_stream(y + (int64_t)rows[u] * V + v)
+                        buf[u] = (rows[u] >= 0 && act) ? ld_row<GATED>(y + (int64_t)rows[u] * V + v)
                                                        : make_uint4(0, 0, 0, 0);
                     }
 #pragma unroll
@@ -149,166 +201,108 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(CombineParams p)
     }
 }
 
-// ---------------------------------------------------------------- bulk path
+// Ungated, k <= 8, with 32-byte row loads (sm_100 ld .v8.b32): a lane sums 16
+// channels per load, kWideBatch rows at a time.  Same arithmetic and order.
+constexpr bool kWideVectors = false;
+constexpr int kWideBatch = 2;
 
-__device__ __forceinline__ uint32_t smem_u32(const void *ptr)
+struct alignas(32) Vec32 {
+    uint32_t w[8];
+};
+
+__device__ __forceinline__ Vec32 ld_stream32(const Vec32 *ptr)
 {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(ptr));
+    Vec32 v;
+    asm("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]), "=r"(v.w[5]), "=r"(v.w[6]),
+          "=r"(v.w[7])
+        : "l"(ptr));
+    return v;
 }
 
-__device__ __forceinline__ uint64_t now_ns()
+__global__ void __launch_bounds__(kWarps * 32) combine_wide_kernel(CombineParams p)
 {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns)
-{
-    const uint64_t t0 = now_ns();
-    for (uint32_t it = 0; it < (1u << 24); ++it) {
-        if (mbar_try_wait(bar, parity))
-            return true;
-        if (now_ns() - t0 > limit_ns)
-            return false;
-    }
-    return false;
-}
-
-// Warp 0: fetch token t's rows and weights into the stage's tables and start
-// the bulk loads of its valid rows (one expect_tx for their total size).
-__device__ __forceinline__ void issue_token(const CombineParams &p, int64_t t, uint32_t stage_smem,
-                                            uint32_t bar, int *s_rows, float *s_w, uint32_t row_bytes)
-{
-    const int lane = threadIdx.x & 31;
-    const int row = lane < p.k ? __ldg(p.src_pool_row + t * p.k + lane) : -1;
-    if (lane < p.k) {
-        s_rows[lane] = row;
-        s_w[lane] = __ldg(p.w + t * p.k + lane);
-    }
-    const unsigned valid = __ballot_sync(kFullMask, row >= 0);
-    if (lane == 0)
-        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
-                     ::"r"(bar), "r"((uint32_t)__popc(valid) * row_bytes) : "memory");
-    for (int j = 0; j < p.k; ++j) {
-        const int r = __shfl_sync(kFullMask, row, j);
-        if (lane == 0 && r >= 0)
-            asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                         ::"r"(stage_smem + (uint32_t)j * row_bytes),
-                           "l"(static_cast<const uint8_t *>(p.y) + (int64_t)r * row_bytes), "r"(row_bytes),
-                           "r"(bar) : "memory");
-    }
-}
-
-__global__ void __launch_bounds__(kBulkThreads) combine_bulk_kernel(CombineParams p)
-{
-    extern __shared__ __align__(128) uint8_t stage_mem[];   // [stages][k][row bytes]
-    __shared__ __align__(8) uint64_t bars[kBulkStages];
-    __shared__ int s_rows[kBulkStages][32];
-    __shared__ float s_w[kBulkStages][32];
     grid_dependency_wait();
     allow_dependents();
-    const int tid = threadIdx.x;
-    const int warp = tid >> 5;
-    const int V = p.H / 8;
-    const uint32_t row_bytes = (uint32_t)p.H * 2u;
-    const uint32_t stage_bytes = (uint32_t)p.k * row_bytes;
-    const uint32_t base = smem_u32(stage_mem);
-    const int64_t n = p.T > blockIdx.x ? (p.T - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-    auto token = [&](int64_t i) { return (int64_t)blockIdx.x + i * gridDim.x; };
-
-    if (warp == 0) {
-        if (tid == 0) {
-            for (int s = 0; s < kBulkStages; ++s)
-                asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[s])));
-            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    const int lane = threadIdx.x & 31;
+    const int V = p.H / 16;
+    const int seg = p.seg_len / 2;
+    const int64_t items = p.T * p.segs;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const Vec32 *y = static_cast<const Vec32 *>(p.y);
+    for (int64_t it = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items; it += nwarps) {
+        const int64_t t = p.T - 1 - it / p.segs;
+        const int s = (int)(it - (p.T - 1 - t) * p.segs);
+        const int v_begin = s * seg;
+        const int v_end = min(V, v_begin + seg);
+        const int my_row = lane < p.k ? __ldg(p.src_pool_row + t * p.k + lane) : -1;
+        const float my_w = lane < p.k ? (p.w ? __ldg(p.w + t * p.k + lane) : 1.f) : 0.f;
+        int rows[kKMax];
+        float ws[kKMax];
+#pragma unroll
+        for (int j = 0; j < kKMax; ++j) {
+            rows[j] = __shfl_sync(kFullMask, my_row, j);
+            ws[j] = __shfl_sync(kFullMask, my_w, j);
         }
-        __syncwarp();
-        for (int64_t i = 0; i < n && i < kBulkStages; ++i)
-            issue_token(p, token(i), base + (uint32_t)i * stage_bytes, smem_u32(&bars[i]), s_rows[i], s_w[i],
-                        row_bytes);
-    }
-    __syncthreads();
-    int64_t issued = n < kBulkStages ? n : kBulkStages;
-    const uint4 *stage16 = reinterpret_cast<const uint4 *>(stage_mem);
-    for (int64_t i = 0; i < n; ++i) {
-        const int s = (int)(i % kBulkStages);
-        const bool ok = mbar_wait_bounded(smem_u32(&bars[s]), (uint32_t)((i / kBulkStages) & 1), 100000000ull);
-        if (!__syncthreads_and(ok)) {
-            if (tid == 0) {
-                atomicMax(p.error_epoch, p.epoch);
-                for (int64_t q = i; q < issued; ++q)        // let issued loads land before exiting
-                    mbar_wait_bounded(smem_u32(&bars[q % kBulkStages]), (uint32_t)((q / kBulkStages) & 1),
-                                      100000000ull);
+        Vec32 *out = static_cast<Vec32 *>(p.out) + t * V;
+        for (int v = v_begin + lane; v < v_end; v += 32) {
+            float acc[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                acc[i] = 0.f;
+#pragma unroll
+            for (int j0 = 0; j0 < kKMax; j0 += kWideBatch) {
+                Vec32 buf[kWideBatch];
+#pragma unroll
+                for (int u = 0; u < kWideBatch; ++u)
+                    if (rows[j0 + u] >= 0)
+                        buf[u] = ld_stream32(y + (int64_t)rows[j0 + u] * V + v);
+#pragma unroll
+                for (int u = 0; u < kWideBatch; ++u)
+                    if (rows[j0 + u] >= 0)
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            accumulate_word(acc[2 * i], acc[2 * i + 1], buf[u].w[i], ws[j0 + u]);
             }
-            return;
+            Vec32 o;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                o.w[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
+            asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                         ::"l"(out + v), "r"(o.w[0]), "r"(o.w[1]), "r"(o.w[2]), "r"(o.w[3]), "r"(o.w[4]),
+                           "r"(o.w[5]), "r"(o.w[6]), "r"(o.w[7]) : "memory");
         }
-        const int64_t t = token(i);
-        const uint4 *st = stage16 + (size_t)s * (stage_bytes / 16);
-        uint4 *out = static_cast<uint4 *>(p.out) + t * V;
-        for (int v = tid; v < V; v += kBulkThreads) {
-            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            for (int j = 0; j < p.k; ++j)
-                if (s_rows[s][j] >= 0)
-                    accumulate(acc, st[(size_t)j * V + v], s_w[s][j]);
-            out[v] = pack_out(acc);
-        }
-        __syncthreads();                                 // the stage and its tables are free again
-        if (warp == 0 && issued < n) {
-            issue_token(p, token(issued), base + (uint32_t)s * stage_bytes, smem_u32(&bars[s]), s_rows[s],
-                        s_w[s], row_bytes);
-        }
-        if (issued < n)
-            ++issued;
     }
 }
 
 }  // namespace
 
-cudaError_t launch_combine(const CombineParams &p, cudaStream_t s, int num_sms)
+cudaError_t launch_combine(const CombineParams &p, cudaStream_t s, int num_ctas)
 {
     const int64_t items = p.T * p.segs;
     if (items == 0)
         return cudaSuccess;
-    const int64_t smem = (int64_t)kBulkStages * p.k * p.H * 2;
-    if (kBulkCombine && p.k <= 32 && smem <= kBulkMaxSmem) {
-        static int attr_set = 0;
-        if (!attr_set) {
-            cudaError_t e = cudaFuncSetAttribute(combine_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 kBulkMaxSmem);
-            if (e != cudaSuccess)
-                return e;
-            attr_set = 1;
-        }
-        int per_sm = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_bulk_kernel, kBulkThreads,
-                                                          (size_t)smem) != cudaSuccess || per_sm < 1)
-            per_sm = 1;
-        const int64_t cap = (int64_t)num_sms * per_sm;
-        return launch_kernel(combine_bulk_kernel, dim3((int)(p.T < cap ? p.T : cap)), dim3(kBulkThreads),
-                             (size_t)smem, s, p);
-    }
     const int64_t want = (items + kWarps - 1) / kWarps;
-    return launch_kernel(combine_kernel, dim3((int)want), dim3(kWarps * 32), 0, s, p);
+    if (p.y_done) {
+        // persistent: at most num_ctas CTAs, so that the producer keeps its SMs
+        const int64_t n = want < num_ctas ? want : num_ctas;
+        return launch_kernel(combine_kernel<true>, dim3((int)n), dim3(kWarps * 32), 0, s, p);
+    }
+    const bool wide = kWideVectors && p.k <= kKMax && p.H % 16 == 0 && p.seg_len % 2 == 0 &&
+                      ((reinterpret_cast<uintptr_t>(p.y) | reinterpret_cast<uintptr_t>(p.out)) & 31u) == 0;
+    if (wide)
+        return launch_kernel(combine_wide_kernel, dim3((int)want), dim3(kWarps * 32), 0, s, p);
+    return launch_kernel(combine_kernel<false>, dim3((int)want), dim3(kWarps * 32), 0, s, p);
 }
 
 cudaError_t preload_combine_kernels()
 {
     cudaFuncAttributes a;
-    cudaError_t e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(combine_kernel));
+    cudaError_t e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(combine_kernel<false>));
     if (e == cudaSuccess)
-        e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(combine_bulk_kernel));
+        e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(combine_kernel<true>));
+    if (e == cudaSuccess)
+        e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(combine_wide_kernel));
     return e;
 }
 

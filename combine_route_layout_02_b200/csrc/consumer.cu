@@ -11,6 +11,12 @@
 // valid rows with L2-coherent loads, eight 16-byte loads in flight per lane.  When a wait gives up, status[0] becomes
 // SEP_ERR_TIMEOUT; every CTA then stops waiting and counts its remaining tiles
 // in status[1].  No wait is unbounded.
+//
+// With per-token stamps the consumer stands in for the expert compute that
+// feeds a gated combine (identity experts: the copy is the expert output):
+// once a tile's rows are stored, each row adds one arrival to its token's
+// counter and the arrival that completes the token release-stores done_seq
+// into y_done[token] (StreamEP README, opening section: y_done_per_token).
 #include "sep_internal.cuh"
 
 namespace sep {
@@ -51,6 +57,35 @@ __device__ int wait_tile(const ConsumeParams &p, int tile)
     }
 }
 
+__device__ __forceinline__ unsigned atom_add_acq_rel_gpu(unsigned *ptr, unsigned v)
+{
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(ptr), "r"(v) : "memory");
+    return old;
+}
+
+__device__ __forceinline__ void st_release_gpu(unsigned *ptr, unsigned v)
+{
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+}
+
+// After the CTA has copied a tile: one arrival per valid row on its token's
+// counter; the arrival that completes the token (all its valid assignments)
+// release-stores done_seq into y_done[token].
+__device__ void stamp_tokens(const ConsumeParams &p, int tile)
+{
+    for (int r = threadIdx.x; r < p.B; r += blockDim.x) {
+        const int tok = __ldg(p.pool_recv_token + (int64_t)tile * p.B + r);
+        if (tok < 0)
+            continue;
+        unsigned need = 0;
+        for (int j = 0; j < p.k; ++j)
+            need += __ldg(p.src_pool_row + (int64_t)tok * p.k + j) >= 0 ? 1u : 0u;
+        if (atom_add_acq_rel_gpu(p.token_arrivals + tok, 1u) + 1u == need)
+            st_release_gpu(p.y_done + tok, p.done_seq);
+    }
+}
+
 __global__ void __launch_bounds__(kThreads) consume_tiles_kernel(ConsumeParams p)
 {
     __shared__ int s_off[kMaxExperts + 1];
@@ -74,7 +109,8 @@ __global__ void __launch_bounds__(kThreads) consume_tiles_kernel(ConsumeParams p
             if (threadIdx.x == 0)
                 s_go = wait_tile(p, tile);
             __syncthreads();
-            if (s_go) {
+            const int go = s_go;
+            if (go) {
                 const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
                 for (int r = warp; r < p.B; r += kThreads / 32) {
                     const int64_t row = (int64_t)tile * p.B + r;
@@ -97,10 +133,14 @@ __global__ void __launch_bounds__(kThreads) consume_tiles_kernel(ConsumeParams p
                         }
                     }
                 }
+                if (p.y_done)
+                    __threadfence();                     // this thread's rows before the CTA barrier
             } else if (threadIdx.x == 0) {
                 atomicAdd(p.status + 1, 1u);
             }
             __syncthreads();
+            if (go && p.y_done)
+                stamp_tokens(p, tile);
         }
     }
 }

@@ -99,6 +99,12 @@ sep_status preload_once(int dev)
         e = sep::preload_combine_kernels();
     if (e == cudaSuccess)
         e = sep::preload_consumer_kernels();
+    if (e == cudaSuccess)
+        e = sep::preload_gather_kernels();
+    if (e == cudaSuccess)
+        e = sep::preload_backward_kernels();
+    if (e == cudaSuccess)
+        e = sep::preload_scatter_kernels();
     if (e != cudaSuccess)
         return cuda_fail(e, "loading the library's kernels");
     if (dev >= 0 && dev < 64)
@@ -153,6 +159,7 @@ sep_status create(int64_t T_cap, int k, int E, int R, int B, uint32_t flags, cud
     const size_t o_hist = carve(&off, (size_t)h->wchunk_cap * ((E + 3) / 4 * 4) * 4);   // rows padded to 4
     const size_t o_base = carve(&off, (size_t)h->wchunk_cap * E * 4);
     const size_t o_in = (flags & SEP_LAYOUT_TOKEN_IN_OWNER) ? carve(&off, (size_t)(T_cap > 0 ? T_cap : 1) * R) : 0;
+    const size_t o_arr = carve(&off, (size_t)(T_cap > 0 ? T_cap : 1) * 4);
 
     cudaError_t e = cudaMallocAsync(&h->block, off, s);
     if (e != cudaSuccess) {
@@ -184,6 +191,7 @@ sep_status create(int64_t T_cap, int k, int E, int R, int B, uint32_t flags, cud
     h->wchunk_hist = reinterpret_cast<int32_t *>(b + o_hist);
     h->wchunk_base = reinterpret_cast<int32_t *>(b + o_base);
     h->is_token_in_rank = (flags & SEP_LAYOUT_TOKEN_IN_OWNER) ? reinterpret_cast<uint8_t *>(b + o_in) : nullptr;
+    h->token_arrivals = reinterpret_cast<uint32_t *>(b + o_arr);
     e = cudaMemsetAsync(h->sizes, 0, o_bar + 8 - o_sizes, s);   // sizes, error words, barrier counters
     if (e != cudaSuccess) {
         cudaFreeAsync(h->block, s);
@@ -227,6 +235,27 @@ constexpr int64_t kDispatchMinSegs = 1 << 20;
 constexpr int64_t kDispatchPublishMinSegs = 1;
 constexpr int64_t kDispatchFp8MinSegs = 7;
 constexpr int64_t kCombineMinSegs = 1;
+
+// A borrowed view leases the handle's row map to its consumers.
+sep_status check_not_leased(const sep_handle *h)
+{
+    if (h->leased)
+        return fail(SEP_ERR_HANDLE_MISMATCH, "a borrowed view of this handle is active: call sep_view_release first");
+    return SEP_OK;
+}
+
+// Order work on stream s after the consumers a view release recorded.
+sep_status wait_for_release(sep_handle *h, cudaStream_t s, bool clear)
+{
+    for (int i = 0; i < h->n_release; ++i) {
+        const cudaError_t e = cudaStreamWaitEvent(s, h->release_events[i], 0);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaStreamWaitEvent (view release)");
+    }
+    if (clear)
+        h->n_release = 0;
+    return SEP_OK;
+}
 
 // Rows a buffer must hold for the handle's current layout.
 int64_t needed_rows(const sep_handle *h)
@@ -349,6 +378,10 @@ sep_status sep_layout(const void *topk_idx, int idx_bytes, int64_t num_tokens, i
                         (long long)h->T_cap, (long long)num_tokens);
         if ((flags & SEP_LAYOUT_TOKEN_IN_OWNER) && h->is_token_in_rank == nullptr)
             return fail(SEP_ERR_HANDLE_MISMATCH, "handle was made without SEP_LAYOUT_TOKEN_IN_OWNER");
+        if ((st = check_not_leased(h)) != SEP_OK)
+            return st;
+        if ((st = wait_for_release(h, s, true)) != SEP_OK)   // consumers of the old row map finish first
+            return st;
     } else {
         if ((st = create(num_tokens, top_k, num_experts, num_owners, block_m, flags, s, &h)) != SEP_OK)
             return st;
@@ -467,6 +500,8 @@ sep_status sep_dispatch(sep_handle *h, const void *x, int64_t hidden, int payloa
     if (h == nullptr)
         return fail(SEP_ERR_INVALID_ARG, "NULL handle");
     sep_status st = check_device(h);
+    if (st == SEP_OK)
+        st = check_not_leased(h);
     if (st != SEP_OK)
         return st;
     if (payload != SEP_PAYLOAD_BF16 && payload != SEP_PAYLOAD_FP8_E4M3)
@@ -507,6 +542,8 @@ sep_status sep_dispatch(sep_handle *h, const void *x, int64_t hidden, int payloa
                         dispatch_seq, h->last_seq);
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = wait_for_release(h, s, false)) != SEP_OK)
+        return st;
     h->last_stream = s;
     if (tile_ready != nullptr) {
         h->last_tile_ready = tile_ready;
@@ -550,8 +587,15 @@ sep_status sep_dispatch(sep_handle *h, const void *x, int64_t hidden, int payloa
     return e == cudaSuccess ? SEP_OK : cuda_fail(e, "dispatch launch");
 }
 
-sep_status sep_combine(const sep_handle *h, uint32_t layout_epoch, const void *y_pool, int64_t hidden,
-                       int64_t y_capacity_rows, const float *topk_weight, void *out, void *stream)
+namespace {
+
+// Checks shared by the combine family and the parameters they launch with.
+// y is a pool-layout bf16 array of y_rows rows, w the routing weights (NULL:
+// unit weights), out the token-order result.  *empty is set when the layout
+// has no tokens (nothing to launch).
+sep_status prepare_combine(const sep_handle *h, uint32_t layout_epoch, const void *y, int64_t hidden,
+                           int64_t y_rows, const float *w, bool weighted, void *out, cudaStream_t s,
+                           sep::CombineParams *p, bool *empty)
 {
     if (h == nullptr)
         return fail(SEP_ERR_INVALID_ARG, "NULL handle");
@@ -561,47 +605,222 @@ sep_status sep_combine(const sep_handle *h, uint32_t layout_epoch, const void *y
     if (layout_epoch != h->epoch)
         return fail(SEP_ERR_HANDLE_MISMATCH, "handle epoch is %u, caller's routing has epoch %u",
                     h->epoch, layout_epoch);
+    if ((st = check_not_leased(h)) != SEP_OK)
+        return st;
     if (hidden < 1 || hidden > 65536 || hidden % 8 != 0)
         return fail(SEP_ERR_INVALID_ARG, "hidden must be a multiple of 8 in 1..65536 (got %lld)",
                     (long long)hidden);
-    if (h->T > 0 && (y_pool == nullptr || topk_weight == nullptr || out == nullptr))
-        return fail(SEP_ERR_INVALID_ARG, "y_pool, topk_weight or out is NULL");
-    if (!aligned16(y_pool) || !aligned16(out))
-        return fail(SEP_ERR_INVALID_ARG, "y_pool and out must be 16-byte aligned");
-    if ((reinterpret_cast<uintptr_t>(topk_weight) & 3u) != 0)
+    if (h->T > 0 && (y == nullptr || (weighted && w == nullptr) || out == nullptr))
+        return fail(SEP_ERR_INVALID_ARG, weighted ? "y_pool, topk_weight or out is NULL"
+                                                  : "grad_recv or grad_x is NULL");
+    if (!aligned16(y) || !aligned16(out))
+        return fail(SEP_ERR_INVALID_ARG, "pool rows and output must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(w) & 3u) != 0)
         return fail(SEP_ERR_INVALID_ARG, "topk_weight must be 4-byte aligned");
     const int64_t need = needed_rows(h);
-    if (y_capacity_rows < need)
-        return fail(SEP_ERR_CAPACITY, "y_pool holds %lld rows, the layout needs %lld",
-                    (long long)y_capacity_rows, (long long)need);
-    if (h->T == 0)
+    if (y_rows < need)
+        return fail(SEP_ERR_CAPACITY, "the pool array holds %lld rows, the layout needs %lld",
+                    (long long)y_rows, (long long)need);
+    if ((st = wait_for_release(const_cast<sep_handle *>(h), s, false)) != SEP_OK)
+        return st;
+    *empty = h->T == 0;
+    if (*empty)
         return SEP_OK;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     const_cast<sep_handle *>(h)->last_stream = s;
 
     const int num_sms = sep::device_sm_count();
-    sep::CombineParams p{};
+    *p = sep::CombineParams{};
+    p->y = y;
+    p->T = h->T;
+    p->H = (int)hidden;
+    p->k = h->k;
+    p->src_pool_row = h->src_pool_row;
+    p->w = weighted ? w : nullptr;
+    p->out = out;
+    p->error_epoch = h->timeout_epoch;
+    p->epoch = h->epoch;
+    const int64_t units = ((hidden / 8) + 31) / 32;
+    int64_t steps = 1;
+    split_rows(h->T, units, (int64_t)num_sms * 32, kCombineMinSegs, &p->segs, &steps);
+    p->seg_len = (int)(steps * 32);
+    return SEP_OK;
+}
+
+uint32_t poll_budget(uint64_t timeout_ns)
+{
+    const uint64_t polls = timeout_ns / 128 + 1024;
+    return polls > 0xffffffffull ? 0xffffffffu : (uint32_t)polls;
+}
+
+}  // namespace
+
+sep_status sep_combine(const sep_handle *h, uint32_t layout_epoch, const void *y_pool, int64_t hidden,
+                       int64_t y_capacity_rows, const float *topk_weight, void *out, void *stream)
+{
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    sep::CombineParams p;
+    bool empty = false;
+    sep_status st = prepare_combine(h, layout_epoch, y_pool, hidden, y_capacity_rows, topk_weight, true, out, s,
+                                    &p, &empty);
+    if (st != SEP_OK || empty)
+        return st;
+    cudaError_t e = sep::launch_combine(p, s, 0);
+    return e == cudaSuccess ? SEP_OK : cuda_fail(e, "combine launch");
+}
+
+sep_status sep_combine_scatter(const sep_handle *h, uint32_t layout_epoch, const void *y_pool, int64_t hidden,
+                               int64_t y_capacity_rows, const float *topk_weight, void *out, void *stream)
+{
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    sep::CombineParams c;
+    bool empty = false;
+    sep_status st = prepare_combine(h, layout_epoch, y_pool, hidden, y_capacity_rows, topk_weight, true, out, s,
+                                    &c, &empty);
+    if (st != SEP_OK || empty)
+        return st;
+    cudaError_t e = cudaMemsetAsync(out, 0, (size_t)h->T * (size_t)hidden * 2, s);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaMemsetAsync (out)");
+    const int num_sms = sep::device_sm_count();
+    sep::ScatterParams p{};
     p.y = y_pool;
+    p.H = (int)hidden;
+    p.k = h->k;
+    p.pool_recv_token = h->pool_recv_token;
+    p.pool_recv_slot = h->pool_recv_slot;
+    p.w = topk_weight;
+    p.out = out;
+    p.num_pool_rows = h->sizes;
+    p.rows_cap = needed_rows(h);
+    // a pool row splits into the dispatch's 4 KB steps
+    const int64_t units = ((hidden / 8) + kDispatchStepVecs - 1) / kDispatchStepVecs;
+    int64_t steps = 1;
+    split_rows(p.rows_cap, units, (int64_t)num_sms * 32, kDispatchMinSegs, &p.segs, &steps);
+    p.seg_len = (int)(steps * kDispatchStepVecs);
+    e = sep::launch_combine_scatter(p, s);
+    return e == cudaSuccess ? SEP_OK : cuda_fail(e, "scatter combine launch");
+}
+
+sep_status sep_combine_grads(const sep_handle *h, uint32_t layout_epoch, const void *grad_recv, int64_t hidden,
+                             int64_t capacity_rows, void *grad_x, void *stream)
+{
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    sep::CombineParams p;
+    bool empty = false;
+    sep_status st = prepare_combine(h, layout_epoch, grad_recv, hidden, capacity_rows, nullptr, false, grad_x, s,
+                                    &p, &empty);
+    if (st != SEP_OK || empty)
+        return st;
+    cudaError_t e = sep::launch_combine(p, s, 0);
+    return e == cudaSuccess ? SEP_OK : cuda_fail(e, "combine_grads launch");
+}
+
+sep_status sep_combine_gated(const sep_handle *h, uint32_t layout_epoch, const void *y_pool, int64_t hidden,
+                             int64_t y_capacity_rows, const float *topk_weight, void *out, const uint32_t *y_done,
+                             int64_t y_done_len, uint32_t done_seq, int num_ctas, uint64_t timeout_ns,
+                             uint32_t *status, void *stream)
+{
+    if (h != nullptr) {
+        if (y_done == nullptr || status == nullptr)
+            return fail(SEP_ERR_INVALID_ARG, "NULL y_done or status");
+        if (((reinterpret_cast<uintptr_t>(y_done) | reinterpret_cast<uintptr_t>(status)) & 3u) != 0)
+            return fail(SEP_ERR_INVALID_ARG, "y_done and status must be 4-byte aligned");
+        if (done_seq == 0)
+            return fail(SEP_ERR_INVALID_ARG, "done_seq must be nonzero");
+        if (num_ctas < 1 || num_ctas > 1024)
+            return fail(SEP_ERR_INVALID_ARG, "num_ctas must be in 1..1024");
+        if (y_done_len < h->T)
+            return fail(SEP_ERR_CAPACITY, "y_done holds %lld entries, the layout has %lld tokens",
+                        (long long)y_done_len, (long long)h->T);
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    sep::CombineParams p;
+    bool empty = false;
+    sep_status st = prepare_combine(h, layout_epoch, y_pool, hidden, y_capacity_rows, topk_weight, true, out, s,
+                                    &p, &empty);
+    if (st != SEP_OK)
+        return st;
+    cudaError_t e = cudaMemsetAsync(status, 0, 2 * sizeof(uint32_t), s);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaMemsetAsync (status)");
+    if (empty)
+        return SEP_OK;
+    // a warp reduces a whole token, so a token is either reduced or left unwritten
+    p.segs = 1;
+    p.seg_len = (int)(hidden / 8);
+    p.y_done = y_done;
+    p.done_seq = done_seq;
+    p.timeout_ns = timeout_ns ? timeout_ns : 1000000000ull;
+    p.max_polls = poll_budget(p.timeout_ns);
+    p.status = status;
+    e = sep::launch_combine(p, s, num_ctas);
+    return e == cudaSuccess ? SEP_OK : cuda_fail(e, "gated combine launch");
+}
+
+sep_status sep_dispatch_grads(const sep_handle *h, uint32_t layout_epoch, const void *grad_out, int64_t hidden,
+                              const float *topk_weight, const void *y_pool, int64_t y_capacity_rows, void *grad_y,
+                              int64_t grad_y_capacity_rows, float *grad_w, void *stream)
+{
+    if (h == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "NULL handle");
+    sep_status st = check_device(h);
+    if (st != SEP_OK)
+        return st;
+    if (layout_epoch != h->epoch)
+        return fail(SEP_ERR_HANDLE_MISMATCH, "handle epoch is %u, caller's routing has epoch %u",
+                    h->epoch, layout_epoch);
+    if ((st = check_not_leased(h)) != SEP_OK)
+        return st;
+    if (hidden < 1 || hidden > 65536 || hidden % 8 != 0)
+        return fail(SEP_ERR_INVALID_ARG, "hidden must be a multiple of 8 in 1..65536 (got %lld)",
+                    (long long)hidden);
+    if (h->T > 0 && (grad_out == nullptr || topk_weight == nullptr || grad_y == nullptr))
+        return fail(SEP_ERR_INVALID_ARG, "grad_out, topk_weight or grad_y is NULL");
+    if (h->T > 0 && grad_w != nullptr && y_pool == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "grad_w needs y_pool (the forward expert outputs)");
+    if (!aligned16(grad_out) || !aligned16(grad_y) || !aligned16(y_pool))
+        return fail(SEP_ERR_INVALID_ARG, "grad_out, grad_y and y_pool must be 16-byte aligned");
+    if (((reinterpret_cast<uintptr_t>(topk_weight) | reinterpret_cast<uintptr_t>(grad_w)) & 3u) != 0)
+        return fail(SEP_ERR_INVALID_ARG, "topk_weight and grad_w must be 4-byte aligned");
+    const int64_t need = needed_rows(h);
+    if (grad_y_capacity_rows < need)
+        return fail(SEP_ERR_CAPACITY, "grad_y holds %lld rows, the layout needs %lld",
+                    (long long)grad_y_capacity_rows, (long long)need);
+    if (grad_w != nullptr && y_capacity_rows < need)
+        return fail(SEP_ERR_CAPACITY, "y_pool holds %lld rows, the layout needs %lld",
+                    (long long)y_capacity_rows, (long long)need);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = wait_for_release(const_cast<sep_handle *>(h), s, false)) != SEP_OK)
+        return st;
+    if (h->T == 0)
+        return SEP_OK;
+    const_cast<sep_handle *>(h)->last_stream = s;
+
+    const int num_sms = sep::device_sm_count();
+    sep::DispatchGradsParams p{};
+    p.g = grad_out;
+    p.w = topk_weight;
+    p.y = grad_w ? y_pool : nullptr;
+    p.grad_y = grad_y;
+    p.grad_w = grad_w;
     p.T = h->T;
     p.H = (int)hidden;
     p.k = h->k;
     p.src_pool_row = h->src_pool_row;
-    p.w = topk_weight;
-    p.out = out;
-    p.error_epoch = h->timeout_epoch;
-    p.epoch = h->epoch;
-    const int64_t units = ((hidden / 8) + 31) / 32;
+    // without grad_w, rows split into the forward dispatch's steps
+    const int64_t units = ((hidden / 8) + kDispatchStepVecs - 1) / kDispatchStepVecs;
     int64_t steps = 1;
-    split_rows(h->T, units, (int64_t)num_sms * 32, kCombineMinSegs, &p.segs, &steps);
-    p.seg_len = (int)(steps * 32);
-    cudaError_t e = sep::launch_combine(p, s, num_sms);
-    return e == cudaSuccess ? SEP_OK : cuda_fail(e, "combine launch");
+    split_rows(h->T, units, (int64_t)num_sms * 32, kDispatchMinSegs, &p.segs, &steps);
+    p.seg_len = (int)(steps * kDispatchStepVecs);
+    cudaError_t e = sep::launch_dispatch_grads(p, s, num_sms);
+    return e == cudaSuccess ? SEP_OK : cuda_fail(e, "dispatch_grads launch");
 }
 
-sep_status sep_consume_tiles(const sep_handle *h, const void *recv_x, int64_t row_bytes,
-                             int64_t capacity_rows, const uint32_t *tile_ready, int64_t tile_ready_len,
-                             uint32_t dispatch_seq, void *dst, int num_ctas, uint64_t timeout_ns,
-                             uint32_t *status, void *stream)
+namespace {
+
+sep_status consume(const sep_handle *h, const void *recv_x, int64_t row_bytes, int64_t capacity_rows,
+                   const uint32_t *tile_ready, int64_t tile_ready_len, uint32_t dispatch_seq, void *dst, int num_ctas,
+                   uint64_t timeout_ns, uint32_t *status, uint32_t *y_done, uint32_t done_seq, cudaStream_t s)
 {
     if (h == nullptr)
         return fail(SEP_ERR_INVALID_ARG, "NULL handle");
@@ -614,8 +833,9 @@ sep_status sep_consume_tiles(const sep_handle *h, const void *recv_x, int64_t ro
         return fail(SEP_ERR_INVALID_ARG, "row_bytes must be a multiple of 16 in 16..2^20");
     if (!aligned16(recv_x) || !aligned16(dst))
         return fail(SEP_ERR_INVALID_ARG, "recv_x and dst must be 16-byte aligned");
-    if (((reinterpret_cast<uintptr_t>(tile_ready) | reinterpret_cast<uintptr_t>(status)) & 3u) != 0)
-        return fail(SEP_ERR_INVALID_ARG, "tile_ready and status must be 4-byte aligned");
+    if (((reinterpret_cast<uintptr_t>(tile_ready) | reinterpret_cast<uintptr_t>(status) |
+          reinterpret_cast<uintptr_t>(y_done)) & 3u) != 0)
+        return fail(SEP_ERR_INVALID_ARG, "tile_ready, status and y_done must be 4-byte aligned");
     if (dispatch_seq == 0)
         return fail(SEP_ERR_INVALID_ARG, "dispatch_seq must be nonzero");
     if (num_ctas < 1 || num_ctas > 1024)
@@ -627,12 +847,16 @@ sep_status sep_consume_tiles(const sep_handle *h, const void *recv_x, int64_t ro
     if (tile_ready_len < need / h->B)
         return fail(SEP_ERR_CAPACITY, "tile_ready holds %lld entries, the layout needs %lld",
                     (long long)tile_ready_len, (long long)(need / h->B));
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemsetAsync(status, 0, 2 * sizeof(uint32_t), s);
     if (e != cudaSuccess)
         return cuda_fail(e, "cudaMemsetAsync (status)");
     if (h->T == 0)
         return SEP_OK;
+    if (y_done != nullptr) {
+        e = cudaMemsetAsync(h->token_arrivals, 0, (size_t)h->T * 4, s);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaMemsetAsync (token counters)");
+    }
     sep::ConsumeParams p{};
     p.src = static_cast<const uint8_t *>(recv_x);
     p.dst = static_cast<uint8_t *>(dst);
@@ -644,18 +868,137 @@ sep_status sep_consume_tiles(const sep_handle *h, const void *recv_x, int64_t ro
     p.tile_ready = tile_ready;
     p.seq = dispatch_seq;
     p.timeout_ns = timeout_ns ? timeout_ns : 1000000000ull;
-    const uint64_t polls = p.timeout_ns / 128 + 1024;
-    p.max_polls = polls > 0xffffffffull ? 0xffffffffu : (uint32_t)polls;
+    p.max_polls = poll_budget(p.timeout_ns);
     p.status = status;
     p.abort_flag = status;
+    p.y_done = y_done;
+    p.token_arrivals = h->token_arrivals;
+    p.src_pool_row = h->src_pool_row;
+    p.k = h->k;
+    p.done_seq = done_seq;
     e = sep::launch_consume(p, num_ctas, s);
     return e == cudaSuccess ? SEP_OK : cuda_fail(e, "consumer launch");
+}
+
+}  // namespace
+
+sep_status sep_consume_tiles(const sep_handle *h, const void *recv_x, int64_t row_bytes,
+                             int64_t capacity_rows, const uint32_t *tile_ready, int64_t tile_ready_len,
+                             uint32_t dispatch_seq, void *dst, int num_ctas, uint64_t timeout_ns,
+                             uint32_t *status, void *stream)
+{
+    return consume(h, recv_x, row_bytes, capacity_rows, tile_ready, tile_ready_len, dispatch_seq, dst, num_ctas,
+                   timeout_ns, status, nullptr, 0, static_cast<cudaStream_t>(stream));
+}
+
+sep_status sep_consume_tiles_stamp(const sep_handle *h, const void *recv_x, int64_t row_bytes,
+                                   int64_t capacity_rows, const uint32_t *tile_ready, int64_t tile_ready_len,
+                                   uint32_t dispatch_seq, void *dst, int num_ctas, uint64_t timeout_ns,
+                                   uint32_t *status, uint32_t *y_done, int64_t y_done_len, uint32_t done_seq,
+                                   void *stream)
+{
+    if (h != nullptr) {
+        if (y_done == nullptr)
+            return fail(SEP_ERR_INVALID_ARG, "NULL y_done");
+        if (done_seq == 0)
+            return fail(SEP_ERR_INVALID_ARG, "done_seq must be nonzero");
+        if (y_done_len < h->T)
+            return fail(SEP_ERR_CAPACITY, "y_done holds %lld entries, the layout has %lld tokens",
+                        (long long)y_done_len, (long long)h->T);
+    }
+    return consume(h, recv_x, row_bytes, capacity_rows, tile_ready, tile_ready_len, dispatch_seq, dst, num_ctas,
+                   timeout_ns, status, y_done, done_seq, static_cast<cudaStream_t>(stream));
+}
+
+sep_status sep_dispatch_borrow(sep_handle *h, const void *x, int64_t hidden, int payload, sep_recv_view *view)
+{
+    if (h == nullptr || view == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "NULL handle or view");
+    sep_status st = check_device(h);
+    if (st == SEP_OK)
+        st = check_not_leased(h);
+    if (st != SEP_OK)
+        return st;
+    if (payload != SEP_PAYLOAD_BF16)
+        return fail(SEP_ERR_INVALID_ARG, "a borrowed view supports the bf16 payload only (FP8 must quantise)");
+    if (!h->synced)
+        return fail(SEP_ERR_INVALID_ARG, "a borrowed view needs CPU counts: sync the layout first");
+    if (hidden < 1 || hidden > 65536 || hidden % 8 != 0)
+        return fail(SEP_ERR_INVALID_ARG, "hidden must be a multiple of 8 in 1..65536 (got %lld)", (long long)hidden);
+    if (h->T > 0 && x == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "x is NULL");
+    if (!aligned16(x))
+        return fail(SEP_ERR_INVALID_ARG, "x must be 16-byte aligned");
+    view->slab = x;
+    view->row_indices = h->pool_recv_token;
+    view->num_rows = h->P;
+    view->row_bytes = hidden * 2;
+    view->indexed = 1;
+    view->epoch = h->epoch;
+    h->leased = 1;
+    return SEP_OK;
+}
+
+sep_status sep_view_release(sep_handle *h, void *const *streams, int num_streams)
+{
+    if (h == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "NULL handle");
+    if (!h->leased)
+        return fail(SEP_ERR_INVALID_ARG, "the handle has no active borrowed view");
+    if (num_streams < 0 || num_streams > 8 || (num_streams > 0 && streams == nullptr))
+        return fail(SEP_ERR_INVALID_ARG, "num_streams must be in 0..8");
+    sep_status st = check_device(h);
+    if (st != SEP_OK)
+        return st;
+    for (int i = 0; i < num_streams; ++i) {
+        if (i >= h->release_events_made) {
+            const cudaError_t e = cudaEventCreateWithFlags(&h->release_events[i], cudaEventDisableTiming);
+            if (e != cudaSuccess)
+                return cuda_fail(e, "cudaEventCreateWithFlags (view release)");
+            h->release_events_made = i + 1;
+        }
+        const cudaError_t e = cudaEventRecord(h->release_events[i], static_cast<cudaStream_t>(streams[i]));
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaEventRecord (view release)");
+    }
+    h->n_release = num_streams;
+    h->leased = 0;
+    return SEP_OK;
+}
+
+sep_status sep_gather_rows(const sep_recv_view *view, void *dst, int64_t dst_rows, void *stream)
+{
+    if (view == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "NULL view");
+    const sep_recv_view &v = *view;
+    if (v.num_rows < 0 || v.row_bytes < 16 || v.row_bytes % 16 != 0 || v.row_bytes > (1LL << 20))
+        return fail(SEP_ERR_INVALID_ARG, "view needs num_rows >= 0 and row_bytes a multiple of 16 in 16..2^20");
+    if (v.num_rows > 0 && (v.slab == nullptr || v.row_indices == nullptr || dst == nullptr))
+        return fail(SEP_ERR_INVALID_ARG, "NULL slab, row_indices or dst");
+    if (!aligned16(v.slab) || !aligned16(dst) || (reinterpret_cast<uintptr_t>(v.row_indices) & 3u))
+        return fail(SEP_ERR_INVALID_ARG, "slab and dst must be 16-byte aligned, row_indices 4-byte aligned");
+    if (dst_rows < v.num_rows)
+        return fail(SEP_ERR_CAPACITY, "dst holds %lld rows, the view has %lld", (long long)dst_rows,
+                    (long long)v.num_rows);
+    sep::GatherParams p{};
+    p.slab = static_cast<const uint8_t *>(v.slab);
+    p.row_indices = v.row_indices;
+    p.dst = static_cast<uint8_t *>(dst);
+    p.rows = v.num_rows;
+    p.row_bytes = v.row_bytes;
+    p.indexed = v.indexed ? 1 : 0;
+    const cudaError_t e = sep::launch_gather(p, static_cast<cudaStream_t>(stream), sep::device_sm_count());
+    return e == cudaSuccess ? SEP_OK : cuda_fail(e, "gather launch");
 }
 
 void sep_handle_free(sep_handle *h)
 {
     if (h == nullptr)
         return;
+    if (h->leased) {
+        fail(SEP_ERR_HANDLE_MISMATCH, "sep_handle_free: a borrowed view is active; the handle was not freed");
+        return;
+    }
     int prev = -1;
     const bool switched = cudaGetDevice(&prev) == cudaSuccess && prev != h->device &&
                           cudaSetDevice(h->device) == cudaSuccess;
@@ -663,6 +1006,8 @@ void sep_handle_free(sep_handle *h)
         cudaFreeAsync(h->block, h->last_stream);
     if (h->host_mirror != nullptr)
         cudaFreeHost(h->host_mirror);
+    for (int i = 0; i < h->release_events_made; ++i)
+        cudaEventDestroy(h->release_events[i]);
     if (switched)
         cudaSetDevice(prev);
     delete h;

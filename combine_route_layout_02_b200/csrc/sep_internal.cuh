@@ -72,6 +72,24 @@ struct DispatchParams {
 
 cudaError_t launch_dispatch(const DispatchParams &p, int payload, cudaStream_t s, int num_sms);
 
+// -------------------------------------------------------- backward pair
+
+struct DispatchGradsParams {
+    const void *g;                   // bf16 [T][H]: gradient of the combine output
+    const float *w;                  // [T][k]
+    const void *y;                   // bf16 [rows][H]: expert outputs (grad_w only)
+    void *grad_y;                    // bf16 [rows][H]
+    float *grad_w;                   // [T][k] or nullptr
+    int64_t T;
+    int H, k;
+    const int32_t *src_pool_row;     // [T][k]
+    int segs;                        // warps sharing one token row (no grad_w)
+    int seg_len;                     // 16-byte vectors per warp
+};
+
+cudaError_t launch_dispatch_grads(const DispatchGradsParams &p, cudaStream_t s, int num_sms);
+cudaError_t preload_backward_kernels();
+
 // ---------------------------------------------------------------- combine
 
 struct CombineParams {
@@ -85,9 +103,33 @@ struct CombineParams {
     int seg_len;                     // 16-byte vectors per warp
     uint32_t *error_epoch;           // a bounded wait that gave up records the epoch
     uint32_t epoch;
+    // per-token gate (y_done != nullptr): token t is reduced once y_done[t] >= done_seq
+    const uint32_t *y_done;          // [T]
+    uint32_t done_seq;
+    uint64_t timeout_ns;
+    uint32_t max_polls;
+    uint32_t *status;                // [2]: code, tokens not reduced
 };
 
 cudaError_t launch_combine(const CombineParams &p, cudaStream_t s, int num_sms);
+
+// ---------------------------------------------------- atomic-scatter combine
+
+struct ScatterParams {
+    const void *y;                   // bf16 [rows][H]
+    int H, k;
+    const int32_t *pool_recv_token;  // [rows]
+    const int32_t *pool_recv_slot;   // [rows]
+    const float *w;                  // [T][k]
+    void *out;                       // bf16 [T][H], zero at launch
+    const int64_t *num_pool_rows;    // device word: P of the current layout
+    int64_t rows_cap;                // rows the grid covers (>= P)
+    int segs;                        // warps sharing one pool row
+    int seg_len;                     // 16-byte vectors per warp
+};
+
+cudaError_t launch_combine_scatter(const ScatterParams &p, cudaStream_t s);
+cudaError_t preload_scatter_kernels();
 
 // --------------------------------------------------------------- consumer
 
@@ -104,9 +146,27 @@ struct ConsumeParams {
     uint32_t max_polls;
     uint32_t *status;                // [2]: code, tiles not copied
     uint32_t *abort_flag;            // = &status[0]
+    // per-token completion stamps (y_done != nullptr)
+    uint32_t *y_done;                // [T]
+    uint32_t *token_arrivals;        // [T], zero at launch
+    const int32_t *src_pool_row;     // [T][k]
+    int k;
+    uint32_t done_seq;
 };
 
 cudaError_t launch_consume(const ConsumeParams &p, int num_ctas, cudaStream_t s);
+
+struct GatherParams {
+    const uint8_t *slab;
+    const int32_t *row_indices;
+    uint8_t *dst;
+    int64_t rows;
+    int64_t row_bytes;
+    int indexed;
+};
+
+cudaError_t launch_gather(const GatherParams &p, cudaStream_t s, int num_sms);
+cudaError_t preload_gather_kernels();
 
 // ------------------------------------------------------------------ utils
 
@@ -201,6 +261,12 @@ struct sep_handle {
     uint32_t *bad_epoch;
     uint32_t *timeout_epoch;         // a bounded wait gave up during this epoch
     uint32_t *barrier_words;         // [2] grid-barrier counters of the single-launch layout
+    uint32_t *token_arrivals;        // [T_cap] per-token row counters of the stamping consumer
+    // borrowed-view lease and the consumer events its release recorded
+    int leased;
+    int n_release;
+    cudaEvent_t release_events[8];
+    int release_events_made;
     // pinned host mirror of {P, NT, bad_epoch, timeout_epoch}
     int64_t *host_mirror;
 };

@@ -54,6 +54,12 @@ class LayoutArrays(ctypes.Structure):
     ]
 
 
+class RecvView(ctypes.Structure):
+    """Mirror of sep_recv_view."""
+    _fields_ = [("slab", _P), ("row_indices", _P), ("num_rows", _i64), ("row_bytes", _i64),
+                ("indexed", ctypes.c_int32), ("epoch", _u32)]
+
+
 # (name, restype, argtypes) of every entry point declared in include/sep.h
 _SIGNATURES = [
     ("sep_layout", _i32, [_P, _i32, _i64, _i32, _i32, _i32, _i32, _u32, _P, ctypes.POINTER(_P)]),
@@ -68,7 +74,16 @@ _SIGNATURES = [
     ("sep_status_string", ctypes.c_char_p, [_i32]),
     ("sep_abi_version", _i32, []),
     ("sep_launch_count", _u64, []),
+    ("sep_dispatch_borrow", _i32, [_P, _P, _i64, _i32, ctypes.POINTER(RecvView)]),
+    ("sep_view_release", _i32, [_P, ctypes.POINTER(_P), _i32]),
+    ("sep_gather_rows", _i32, [ctypes.POINTER(RecvView), _P, _i64, _P]),
     ("sep_layout_noalloc", _i32, [_P, _i32, _i64, _i32, _i32, _i32, _i32, ctypes.POINTER(LayoutArrays), _P]),
+    ("sep_consume_tiles_stamp", _i32, [_P, _P, _i64, _i64, _P, _i64, _u32, _P, _i32, _u64, _P, _P, _i64, _u32,
+                                       _P]),
+    ("sep_combine_gated", _i32, [_P, _u32, _P, _i64, _i64, _P, _P, _P, _i64, _u32, _i32, _u64, _P, _P]),
+    ("sep_dispatch_grads", _i32, [_P, _u32, _P, _i64, _P, _P, _i64, _P, _i64, _P, _P]),
+    ("sep_combine_grads", _i32, [_P, _u32, _P, _i64, _i64, _P, _P]),
+    ("sep_combine_scatter", _i32, [_P, _u32, _P, _i64, _i64, _P, _P, _P]),
 ]
 
 
@@ -239,6 +254,67 @@ def sep_consume_tiles(handle: Handle, recv_x: torch.Tensor, tile_ready: torch.Te
                                   _ptr(status), _stream(stream)), "sep_consume_tiles")
 
 
+def sep_combine_scatter(handle: Handle, y_pool: torch.Tensor, topk_weight: torch.Tensor, out: torch.Tensor,
+                        layout_epoch: int | None = None, stream=None) -> None:
+    """The combine by bf16 atomic scatter from the pool rows (not deterministic)."""
+    if y_pool.dtype != torch.bfloat16 or out.dtype != torch.bfloat16 or topk_weight.dtype != torch.float32:
+        raise ValueError("y_pool/out must be bf16 and topk_weight fp32")
+    epoch = handle.epoch if layout_epoch is None else layout_epoch
+    _check(_lib.sep_combine_scatter(handle.ptr, epoch, _ptr(y_pool), y_pool.shape[1], y_pool.shape[0],
+                                    _ptr(topk_weight), _ptr(out), _stream(stream)), "sep_combine_scatter")
+
+
+def sep_consume_tiles_stamp(handle: Handle, recv_x: torch.Tensor, tile_ready: torch.Tensor, dispatch_seq: int,
+                            dst: torch.Tensor, status: torch.Tensor, y_done: torch.Tensor, done_seq: int,
+                            num_ctas: int = 16, timeout_ns: int = 0, stream=None) -> None:
+    row_bytes = recv_x.shape[1] * recv_x.element_size()
+    if dst.shape[0] < recv_x.shape[0] or dst.shape[1] * dst.element_size() != row_bytes:
+        raise ValueError("dst must have recv_x's row size and at least its rows")
+    if status.numel() < 2 or status.element_size() != 4 or y_done.element_size() != 4:
+        raise ValueError("status and y_done hold 32-bit words")
+    _check(_lib.sep_consume_tiles_stamp(handle.ptr, _ptr(recv_x), row_bytes, recv_x.shape[0], _ptr(tile_ready),
+                                        tile_ready.numel(), dispatch_seq, _ptr(dst), num_ctas, timeout_ns,
+                                        _ptr(status), _ptr(y_done), y_done.numel(), done_seq, _stream(stream)),
+           "sep_consume_tiles_stamp")
+
+
+def sep_combine_gated(handle: Handle, y_pool: torch.Tensor, topk_weight: torch.Tensor, out: torch.Tensor,
+                      y_done: torch.Tensor, done_seq: int, status: torch.Tensor, num_ctas: int = 64,
+                      timeout_ns: int = 0, layout_epoch: int | None = None, stream=None) -> None:
+    if y_pool.dtype != torch.bfloat16 or out.dtype != torch.bfloat16 or topk_weight.dtype != torch.float32:
+        raise ValueError("y_pool/out must be bf16 and topk_weight fp32")
+    if status.numel() < 2 or status.element_size() != 4 or y_done.element_size() != 4:
+        raise ValueError("status and y_done hold 32-bit words")
+    epoch = handle.epoch if layout_epoch is None else layout_epoch
+    _check(_lib.sep_combine_gated(handle.ptr, epoch, _ptr(y_pool), y_pool.shape[1], y_pool.shape[0],
+                                  _ptr(topk_weight), _ptr(out), _ptr(y_done), y_done.numel(), done_seq, num_ctas,
+                                  timeout_ns, _ptr(status), _stream(stream)), "sep_combine_gated")
+
+
+def sep_dispatch_grads(handle: Handle, grad_out: torch.Tensor, topk_weight: torch.Tensor, grad_y: torch.Tensor,
+                       y_pool: torch.Tensor | None = None, grad_w: torch.Tensor | None = None,
+                       layout_epoch: int | None = None, stream=None) -> None:
+    """grad_y[row(t,j)] = bf16(w[t,j] * grad_out[t]); grad_w[t,j] = <grad_out[t], y_pool[row(t,j)]> if given."""
+    if grad_out.dtype != torch.bfloat16 or grad_y.dtype != torch.bfloat16 or topk_weight.dtype != torch.float32:
+        raise ValueError("grad_out/grad_y must be bf16 and topk_weight fp32")
+    if grad_w is not None and (grad_w.dtype != torch.float32 or y_pool is None or y_pool.dtype != torch.bfloat16):
+        raise ValueError("grad_w must be fp32 and needs a bf16 y_pool")
+    epoch = handle.epoch if layout_epoch is None else layout_epoch
+    _check(_lib.sep_dispatch_grads(handle.ptr, epoch, _ptr(grad_out), grad_out.shape[1], _ptr(topk_weight),
+                                   _ptr(y_pool), 0 if y_pool is None else y_pool.shape[0], _ptr(grad_y),
+                                   grad_y.shape[0], _ptr(grad_w), _stream(stream)), "sep_dispatch_grads")
+
+
+def sep_combine_grads(handle: Handle, grad_recv: torch.Tensor, grad_x: torch.Tensor,
+                      layout_epoch: int | None = None, stream=None) -> None:
+    """grad_x[t] = bf16(sum over valid j of grad_recv[row(t,j)])."""
+    if grad_recv.dtype != torch.bfloat16 or grad_x.dtype != torch.bfloat16:
+        raise ValueError("grad_recv/grad_x must be bf16")
+    epoch = handle.epoch if layout_epoch is None else layout_epoch
+    _check(_lib.sep_combine_grads(handle.ptr, epoch, _ptr(grad_recv), grad_recv.shape[1], grad_recv.shape[0],
+                                  _ptr(grad_x), _stream(stream)), "sep_combine_grads")
+
+
 def sep_handle_free(handle: Handle) -> None:
     handle.close()
 
@@ -280,3 +356,41 @@ def sep_layout_noalloc(topk_idx: torch.Tensor, num_experts: int, num_owners: int
 def sep_launch_count() -> int:
     """Kernels this process has launched through the library."""
     return int(_lib.sep_launch_count())
+
+
+def sep_dispatch_borrow(handle: Handle, x: torch.Tensor) -> RecvView:
+    """Borrowed receive: a view (x, row map) instead of a copied pool; leases the handle."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a [T, H] bf16 tensor")
+    view = RecvView()
+    _check(_lib.sep_dispatch_borrow(handle.ptr, _ptr(x), x.shape[1], SEP_PAYLOAD_BF16, ctypes.byref(view)),
+           "sep_dispatch_borrow")
+    view._keep = x                                   # the slab must outlive the view
+    return view
+
+
+def sep_view_release(handle: Handle, streams=()) -> None:
+    arr = (_P * max(len(streams), 1))(*[_stream(st).value for st in streams])
+    _check(_lib.sep_view_release(handle.ptr, arr, len(streams)), "sep_view_release")
+
+
+def pool_view(handle: Handle, recv_x: torch.Tensor) -> RecvView:
+    """A view of a copied pool (indexed = 0): the copy path's input to sep_gather_rows."""
+    info = handle.info()
+    if info.num_pool_rows < 0:
+        raise ValueError("the layout must be synced to know the pool size")
+    view = RecvView()
+    view.slab = _ptr(recv_x).value
+    view.row_indices = info.pool_recv_token
+    view.num_rows = info.num_pool_rows
+    view.row_bytes = recv_x.shape[1] * recv_x.element_size()
+    view.indexed = 0
+    view.epoch = info.epoch
+    view._keep = recv_x
+    return view
+
+
+def sep_gather_rows(view: RecvView, dst: torch.Tensor, stream=None) -> None:
+    if dst.shape[1] * dst.element_size() != view.row_bytes:
+        raise ValueError("dst rows must have the view's row size")
+    _check(_lib.sep_gather_rows(ctypes.byref(view), _ptr(dst), dst.shape[0], _stream(stream)), "sep_gather_rows")

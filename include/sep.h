@@ -264,9 +264,176 @@ SEP_API sep_status sep_consume_tiles(const sep_handle *handle, const void *recv_
                              int64_t tile_ready_len, uint32_t dispatch_seq, void *dst,
                              int num_ctas, uint64_t timeout_ns, uint32_t *status, void *stream);
 
+/*
+ * sep_combine_scatter — the combine driven from the pool side with bf16
+ * atomic reductions (StreamEP README, "What's in the box": kernel_y's
+ * AtomicScatterStore, per-warp coalesced bf16 atomic scatter into the output).
+ *
+ * Zeroes out, then for every valid pool row r adds bf16(topk_weight[t, j] *
+ * y_pool[r]) into out[t] (t = pool_recv_token[r], j = pool_recv_slot[r]) with
+ * bf16x2 reductions.  Same arguments and errors as sep_combine; the result is
+ * NOT deterministic: the k terms of a token are each rounded to bf16 and added
+ * in bf16 in arrival order, so it differs from sep_combine by at most about
+ * 2k * 2^-8 * sum_j |w[t, j] * y[row(t, j)]| per element.  Works on an
+ * unsynced layout (the pool size is read on the device).
+ */
+SEP_API sep_status sep_combine_scatter(const sep_handle *handle, uint32_t layout_epoch, const void *y_pool,
+                                       int64_t hidden, int64_t y_capacity_rows, const float *topk_weight,
+                                       void *out, void *stream);
+
+/*
+ * Per-token combine gate (StreamEP README, opening section: y_done_per_token
+ * lets the combine start on a token as soon as that token's compute has
+ * drained, instead of after the whole compute kernel).  On one GPU the gate is
+ * an array y_done [T] in token order: the producer of y_pool release-stores a
+ * sequence number into y_done[t] once every valid row of token t is written;
+ * the gated combine waits (acquire, bounded) for y_done[t] >= done_seq before
+ * it reads token t's rows.  Sequence numbers compare modulo 2^32 (as
+ * int32(y_done[t] - done_seq) >= 0); start y_done at 0 and use a new nonzero
+ * done_seq for each pass.
+ */
+
+/*
+ * sep_consume_tiles_stamp — sep_consume_tiles plus per-token completion stamps.
+ *
+ * The same reference consumer; after a CTA has copied a tile it adds one
+ * arrival per valid row to the row's token counter, and the arrival that
+ * completes token t (its count of valid assignments) release-stores done_seq
+ * into y_done[t].  With dst used as y_pool this stands in for the expert
+ * compute that feeds a gated combine (identity experts).  The token counters
+ * belong to the handle and are reset on `stream` by this call, so two stamping
+ * consumers of one handle must not overlap on the GPU.
+ *
+ *  y_done      device uint32 [y_done_len >= T], 4-byte aligned.
+ *  done_seq    nonzero.
+ * Other arguments, ordering rules and errors as sep_consume_tiles.
+ */
+SEP_API sep_status sep_consume_tiles_stamp(const sep_handle *handle, const void *recv_x, int64_t row_bytes,
+                                           int64_t capacity_rows, const uint32_t *tile_ready,
+                                           int64_t tile_ready_len, uint32_t dispatch_seq, void *dst,
+                                           int num_ctas, uint64_t timeout_ns, uint32_t *status,
+                                           uint32_t *y_done, int64_t y_done_len, uint32_t done_seq,
+                                           void *stream);
+
+/*
+ * sep_combine_gated — sep_combine that waits per token on the gate.
+ *
+ * Same result as sep_combine for every token whose wait succeeds (a token
+ * with no valid assignment is not waited for: it gets +0).  Launches at
+ * most num_ctas (1..1024) persistent CTAs, so keep it below the SM count left
+ * over by the producer; tokens are visited in ascending order.  A wait gives
+ * up after timeout_ns nanoseconds of %globaltimer (0: one second) or a fixed
+ * poll budget; then every warp stops waiting, status[0] becomes
+ * SEP_ERR_TIMEOUT, status[1] counts the tokens not reduced, and their out rows
+ * are left unwritten.
+ *
+ *  y_done      device uint32 [y_done_len >= T], written by the producer.
+ *  status      device uint32 [2]; reset by this call, written by the kernel.
+ * Other arguments as sep_combine.  Like sep_consume_tiles, the host must not
+ * wait for the device between this call and the work that sets the gate.
+ */
+SEP_API sep_status sep_combine_gated(const sep_handle *handle, uint32_t layout_epoch, const void *y_pool,
+                                     int64_t hidden, int64_t y_capacity_rows, const float *topk_weight,
+                                     void *out, const uint32_t *y_done, int64_t y_done_len, uint32_t done_seq,
+                                     int num_ctas, uint64_t timeout_ns, uint32_t *status, void *stream);
+
+/*
+ * Backward pair (StreamEP README, "What's in the box": dispatch_grads and
+ * combine_grads give the backward symmetry of dispatch and combine).
+ *
+ * sep_dispatch_grads — the backward of sep_combine.  With
+ * out[t] = sum_j w[t, j] * y[row(t, j)]:
+ *   grad_y[row(t, j)] = bf16( w[t, j] * grad_out[t] )   fp32 product, rounded
+ *                                                       to nearest even
+ *   grad_w[t, j]      = sum_h grad_out[t, h] * y[row(t, j), h]
+ *                       fp32 sums in a fixed order (reproducible run to run);
+ *                       0 for a masked assignment.
+ *  grad_out     device bf16 [T, hidden], 16-byte aligned.
+ *  topk_weight  device fp32 [T, k] (the forward weights).
+ *  y_pool       device bf16 [y_capacity_rows, hidden], the forward expert
+ *               outputs in pool layout; read only when grad_w != NULL.
+ *  grad_y       device bf16 [grad_y_capacity_rows, hidden] in pool layout;
+ *               padding rows are not written.
+ *  grad_w       device fp32 [T, k], or NULL to skip the weight gradient.
+ * Errors as sep_combine.
+ */
+SEP_API sep_status sep_dispatch_grads(const sep_handle *handle, uint32_t layout_epoch, const void *grad_out,
+                                      int64_t hidden, const float *topk_weight, const void *y_pool,
+                                      int64_t y_capacity_rows, void *grad_y, int64_t grad_y_capacity_rows,
+                                      float *grad_w, void *stream);
+
+/*
+ * sep_combine_grads — the backward of sep_dispatch (bf16 payload).
+ *   grad_x[t] = bf16( sum over valid j, ascending, of grad_recv[row(t, j)] )
+ * in fp32 (sep_combine with every weight 1; exact up to the final rounding
+ * order of the definition).  A token with no valid assignment gets +0.
+ *  grad_recv  device bf16 [capacity_rows, hidden] in pool layout, 16-byte aligned.
+ *  grad_x     device bf16 [T, hidden], 16-byte aligned.
+ * Errors as sep_combine.
+ */
+SEP_API sep_status sep_combine_grads(const sep_handle *handle, uint32_t layout_epoch, const void *grad_recv,
+                                     int64_t hidden, int64_t capacity_rows, void *grad_x, void *stream);
+
+/*
+ * Borrowed receive (PR #769 "Add opt-in borrowed receive storage for compact
+ * BF16 dispatch", "Description"): instead of copying every assigned token row
+ * into the pool, the dispatch hands out a view (slab, row_indices) that an
+ * indexed consumer reads directly.  On one GPU the slab is x itself and
+ * row_indices is the layout's pool_recv_token: pool row r holds
+ * slab[row_indices[r]] (row_indices[r] < 0: padding, never read).
+ */
+typedef struct sep_recv_view {
+    const void *slab;              /* device rows the view reads from */
+    const int32_t *row_indices;    /* device [num_rows]: slab row of each pool row, -1 = padding */
+    int64_t num_rows;              /* pool rows P */
+    int64_t row_bytes;             /* bytes per row (multiple of 16) */
+    int32_t indexed;               /* 1: pool row r is slab[row_indices[r]]; 0: pool row r is slab[r]
+                                      (a pool that was copied; row_indices only marks validity) */
+    uint32_t epoch;                /* layout epoch of the handle the view came from */
+} sep_recv_view;
+
+/*
+ * sep_dispatch_borrow — a dispatch that copies nothing.
+ *
+ * Fills *view = {x, pool_recv_token, P, 2*hidden, indexed=1, epoch} and puts an
+ * exclusive lease on the handle: until sep_view_release, sep_layout,
+ * sep_dispatch, sep_dispatch_borrow and sep_combine on this handle are refused
+ * (SEP_ERR_HANDLE_MISMATCH) and sep_handle_free leaves it allocated, because
+ * they would change or free the row map the consumers are reading.  x must stay
+ * valid and unchanged until the release.  Supported, as in the PR, only for a
+ * bf16 payload after a synced layout (SEP_LAYOUT_SYNC_COUNTS or
+ * sep_handle_sync: the "CPU counts" that give P); everything else is rejected
+ * up front with SEP_ERR_INVALID_ARG.  Launches nothing.
+ */
+SEP_API sep_status sep_dispatch_borrow(sep_handle *handle, const void *x, int64_t hidden, int payload,
+                                       sep_recv_view *view);
+
+/*
+ * sep_view_release — ends the lease of sep_dispatch_borrow.
+ *
+ * Records an event on each of the num_streams consumer streams; the handle's
+ * next layout, dispatch or combine waits for all of them on its own stream
+ * before it touches the row map (the PR's release(*streams): the next
+ * communication is ordered after the consumers).  SEP_ERR_INVALID_ARG if the
+ * handle has no active view or num_streams is not in 0..8.
+ */
+SEP_API sep_status sep_view_release(sep_handle *handle, void *const *streams, int num_streams);
+
+/*
+ * sep_gather_rows — a reference indexed consumer of a view.
+ *
+ * dst[r] = (view->indexed ? slab[row_indices[r]] : slab[r]) for every pool row
+ * r < num_rows with row_indices[r] >= 0; padding rows of dst are not written.
+ * dst: device [dst_rows, row_bytes], 16-byte aligned, dst_rows >= num_rows.
+ * It stands in for the gathered-GEMM consumer of the PR; with indexed = 0 it
+ * reads a copied pool in place, which gives the copy path's consumer.
+ */
+SEP_API sep_status sep_gather_rows(const sep_recv_view *view, void *dst, int64_t dst_rows, void *stream);
+
 /* Frees the handle.  Its device memory is released stream-ordered on the
  * stream of the last call that used it; the caller must have ordered every
- * other stream that used the handle before that point.  NULL is a no-op. */
+ * other stream that used the handle before that point.  NULL is a no-op; a
+ * handle with an active borrowed view is not freed (release the view first). */
 SEP_API void sep_handle_free(sep_handle *handle);
 
 /* Message for the calling thread's last failed call ("" if none). */

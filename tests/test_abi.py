@@ -22,7 +22,7 @@ def test_library_is_built_for_sm100a_and_in_tree():
 
 def test_exports_match_header():
     declared = sep.declared_entry_points(HEADER)
-    assert len(declared) == 13
+    assert len(declared) == 21
     out = subprocess.run(["nm", "-D", "--defined-only", sep.library_path()], capture_output=True,
                          text=True, check=True).stdout
     exported = sorted(set(re.findall(r"\sT\s+(sep_\w+)$", out, flags=re.M)))
@@ -66,6 +66,13 @@ def test_calls_on_null_handle_are_rejected():
     assert lib.sep_dispatch(None, None, 8, 0, 0, None, None, 0, None, 0, 0, None) == sep.SEP_ERR_INVALID_ARG
     assert lib.sep_combine(None, 0, None, 8, 0, None, None, None) == sep.SEP_ERR_INVALID_ARG
     assert lib.sep_consume_tiles(None, None, 16, 0, None, 0, 1, None, 1, 0, None, None) == sep.SEP_ERR_INVALID_ARG
+    assert lib.sep_consume_tiles_stamp(None, None, 16, 0, None, 0, 1, None, 1, 0, None, None, 0, 1,
+                                       None) == sep.SEP_ERR_INVALID_ARG
+    assert lib.sep_combine_gated(None, 0, None, 8, 0, None, None, None, 0, 1, 1, 0, None,
+                                 None) == sep.SEP_ERR_INVALID_ARG
+    assert lib.sep_dispatch_grads(None, 0, None, 8, None, None, 0, None, 0, None, None) == sep.SEP_ERR_INVALID_ARG
+    assert lib.sep_combine_grads(None, 0, None, 8, 0, None, None) == sep.SEP_ERR_INVALID_ARG
+    assert lib.sep_combine_scatter(None, 0, None, 8, 0, None, None, None) == sep.SEP_ERR_INVALID_ARG
     assert lib.sep_handle_sync(None, None) == sep.SEP_ERR_INVALID_ARG
     assert lib.sep_handle_info(None, None) == sep.SEP_ERR_INVALID_ARG
     lib.sep_handle_free(None)            # no-op
@@ -84,7 +91,8 @@ def test_no_cpu_fallback_in_the_binding():
     # imports the oracle or reaches for torch compute on the data path
     src = open(os.path.join(os.path.dirname(sep.__file__), "sep.py")).read()
     assert "oracle" not in src
-    for op in ("index_select", "scatter", "torch.sum", ".sum(", "torch.matmul", "gather("):
+    for op in ("index_select", ".scatter(", ".scatter_(", "scatter_add", "torch.sum", ".sum(", "torch.matmul",
+               "torch.gather", ".gather("):
         assert op not in src
 
 

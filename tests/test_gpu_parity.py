@@ -489,3 +489,103 @@ def test_streaming_first_launch_in_a_fresh_process():
     r = subprocess.run([sys.executable, "-c", _FRESH_PROCESS_STREAMING, root], capture_output=True,
                        text=True, timeout=300)
     assert r.returncode == 0 and "OK" in r.stdout, r.stdout + r.stderr
+
+
+# ------------------------------------------------------ borrowed receive
+
+def test_borrowed_view_rows_equal_the_copied_pool():
+    """PR #769's borrowed receive: the view (x, row map) read by an indexed
+    consumer gives exactly the rows a copying dispatch writes."""
+    w, d = _inputs(W.WORKLOADS["train8k"], 2000)
+    lay = oracle.layout(d["topk_idx"].numpy(), w.E, w.R, w.B)
+    want = oracle.dispatch_bf16(d["x"], lay)
+    valid = lay.pool_recv_token >= 0
+    h = sep.sep_layout(d["topk_idx"].cuda(), w.E, w.R, w.B, flags=sep.SEP_LAYOUT_SYNC_COUNTS)
+    try:
+        x = d["x"].cuda()
+        P = h.info().num_pool_rows
+        # copy path: dispatch, then the consumer reads the pool in place
+        recv = poisoned_bf16(P, w.H)
+        sep.sep_dispatch(h, x, recv)
+        dst_copy = poisoned_bf16(P, w.H)
+        sep.sep_gather_rows(sep.pool_view(h, recv), dst_copy)
+        # borrowed path: no copy, the consumer gathers from x through the row map
+        view = sep.sep_dispatch_borrow(h, x)
+        assert view.num_rows == P and view.indexed == 1 and view.row_bytes == 2 * w.H
+        rows = torch.as_tensor(sep.sep._DeviceArray(view.row_indices, (P,), "<i4"), device="cuda").clone()
+        np.testing.assert_array_equal(rows.cpu().numpy(), lay.pool_recv_token)
+        dst = poisoned_bf16(P, w.H)
+        sep.sep_gather_rows(view, dst)
+        sep.sep_view_release(h, [torch.cuda.current_stream()])
+        torch.cuda.synchronize()
+        for got in (bf16_bits(dst), bf16_bits(dst_copy)):
+            np.testing.assert_array_equal(got[valid], want[valid])
+            assert (got[~valid] == POISON_BF16).all()
+    finally:
+        sep.sep_handle_free(h)
+
+
+def test_borrowed_view_is_rejected_up_front_and_leases_the_handle():
+    w, d = _inputs(W.WORKLOADS["tiny"])
+    x = d["x"].cuda()
+    h = sep.sep_layout(d["topk_idx"].cuda(), w.E, w.R, w.B)
+    try:
+        with pytest.raises(sep.SepError) as ei:              # needs CPU counts
+            sep.sep_dispatch_borrow(h, x)
+        assert ei.value.status == sep.SEP_ERR_INVALID_ARG
+        sep.sep_handle_sync(h)
+        lib = sep.library()
+        view = sep.RecvView()
+        import ctypes
+        st = lib.sep_dispatch_borrow(h.ptr, ctypes.c_void_p(x.data_ptr()), w.H, sep.sep.SEP_PAYLOAD_FP8_E4M3,
+                                     ctypes.byref(view))
+        assert st == sep.SEP_ERR_INVALID_ARG                   # FP8 cannot be borrowed
+        view = sep.sep_dispatch_borrow(h, x)
+        recv = poisoned_bf16(h.info().num_pool_rows, w.H)
+        out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device="cuda")
+        for call in (lambda: sep.sep_layout(d["topk_idx"].cuda(), w.E, w.R, w.B, handle=h),
+                     lambda: sep.sep_dispatch(h, x, recv),
+                     lambda: sep.sep_dispatch_borrow(h, x),
+                     lambda: sep.sep_combine(h, recv, d["topk_weight"].cuda(), out)):
+            with pytest.raises(sep.SepError) as ei:
+                call()
+            assert ei.value.status == sep.SEP_ERR_HANDLE_MISMATCH
+        lib.sep_handle_free(h.ptr)                              # refused while the view is active
+        assert "borrowed view" in lib.sep_last_error().decode()
+        sep.sep_view_release(h, [])
+        with pytest.raises(sep.SepError):                       # nothing left to release
+            sep.sep_view_release(h, [])
+        sep.sep_dispatch(h, x, recv)                            # usable again
+        torch.cuda.synchronize()
+    finally:
+        sep.sep_handle_free(h)
+
+
+def test_borrowed_view_delayed_cross_stream_reader():
+    """The consumer runs late on another stream; after the release, the next
+    layout into the handle (a different routing) waits for it, so the consumer
+    still reads the old row map."""
+    w, d = _inputs(W.WORKLOADS["train8k"], 1500)
+    lay = oracle.layout(d["topk_idx"].numpy(), w.E, w.R, w.B)
+    want = oracle.dispatch_bf16(d["x"], lay)
+    valid = lay.pool_recv_token >= 0
+    other = W.edge_routing("uniform", 1500, w.k, w.E, w.R, seed=3)
+    h = sep.sep_layout(d["topk_idx"].cuda(), w.E, w.R, w.B, flags=sep.SEP_LAYOUT_SYNC_COUNTS)
+    try:
+        x = d["x"].cuda()
+        P = h.info().num_pool_rows
+        dst = poisoned_bf16(h.info().max_pool_rows, w.H)
+        idx2 = other.cuda()
+        torch.cuda.synchronize()
+        side = torch.cuda.Stream()
+        view = sep.sep_dispatch_borrow(h, x)
+        with torch.cuda.stream(side):
+            torch.cuda._sleep(20_000_000)                       # a late reader (bounded spin, ~10 ms)
+        sep.sep_gather_rows(view, dst, stream=side)
+        sep.sep_view_release(h, [side])
+        sep.sep_layout(idx2, w.E, w.R, w.B, handle=h)           # must wait for the reader
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(bf16_bits(dst)[:P][valid], want[valid])
+        check_layout(h, oracle.layout(other.numpy(), w.E, w.R, w.B))
+    finally:
+        sep.sep_handle_free(h)
