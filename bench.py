@@ -54,6 +54,10 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle work for cpu_baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--consumer-ctas", type=int, default=64)
+    ap.add_argument("--gate-ctas", type=int, default=0,
+                    help="CTAs of the gated combine in the combine_gate measurement (0: the consumer's)")
+    ap.add_argument("--graph", action="store_true",
+                    help="also time the step replayed from a CUDA graph (non-streaming workloads)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the backward-pair, combine-gate and scatter-combine measurements")
     return ap.parse_args(argv)
@@ -356,6 +360,8 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
     if w.streaming:
         assert status.cpu().tolist() == [0, 0], f"consumer status {status.cpu().tolist()}"
 
+    graph_ms = replay_step_graph(args, w, step, main, flush, world, dev) if (args.graph and not w.streaming) else None
+
     lay_ms = [e[0].elapsed_time(e[1]) for e in events]
     dis_ms = [e[1].elapsed_time(e[2]) for e in events]
     com_ms = [e[2].elapsed_time(e[3]) for e in events]
@@ -509,6 +515,9 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "mode": e2e_mode,
                 "l2": "not flushed: every step uploads its inputs and the step's working set cycles the L2"},
         "gpu_launches": launches,
+        **({"graph_replay": {"ms_per_step": graph_ms, "value": world * T / (graph_ms * 1e-3),
+                             "note": "the same step captured once in a CUDA graph and replayed (one host launch "
+                                     "per step); L2 flushed between replays"}} if graph_ms else {}),
         **({"borrowed_receive": borrowed} if borrowed else {}),
         **({"backward": backward} if backward else {}),
         **({"combine_gate": gate} if gate else {}),
@@ -518,6 +527,38 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(wr, d, args.cpu_budget)
     return res if rank == 0 else None
+
+
+def replay_step_graph(args, w, step, main, flush, world, dev):
+    """The same step captured once in a CUDA graph and replayed: one launch per
+    step from the host, so for small workloads the time is the kernels' own
+    rather than the host's launch rate.  Events bracket each replay on the
+    launching stream; the L2 is flushed between replays as in the eager loop."""
+    import torch
+    cap = torch.cuda.Stream()
+    cap.wait_stream(main)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        step()
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        if flush is not None:
+            flush.zero_()
+        g.replay()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+        ev[i][0].record(main)
+        g.replay()
+        ev[i][1].record(main)
+    torch.cuda.synchronize()
+    barrier(world)
+    (ms,) = reduce_max([statistics.fmean(a.elapsed_time(b) for a, b in ev)], world, dev)
+    del g
+    return ms
 
 
 def _time_arm(fn, steps, flush=None, warmup=5):
@@ -589,6 +630,9 @@ def scatter_compare(w, h, idx, wt, y, flush, peak_gbs, steps=100):
                     "L2 flushed before every call"}
 
 
+_gate_seq = [1 << 20]
+
+
 def gate_compare(args, w, h, x, idx, wt, recv, dev, steps=50):
     """The per-token combine gate in the streaming pipeline: a streaming
     dispatch, the reference consumer standing in for identity experts (it
@@ -608,8 +652,9 @@ def gate_compare(args, w, h, x, idx, wt, recv, dev, steps=50):
     y_done = torch.zeros(w.T, dtype=torch.int32, device=dev)
     st_c = torch.zeros(2, dtype=torch.int32, device=dev)
     st_g = torch.zeros(2, dtype=torch.int32, device=dev)
-    seq = [0]
+    seq = _gate_seq                                      # advances across calls: tile_ready may reuse an address
     ctas = args.consumer_ctas
+    gctas = args.gate_ctas or ctas
 
     def serial():
         seq[0] += 1
@@ -625,7 +670,7 @@ def gate_compare(args, w, h, x, idx, wt, recv, dev, steps=50):
         third.wait_stream(main)
         sep.sep_consume_tiles_stamp(h, recv, tile_ready, seq[0], y, st_c, y_done, seq[0], num_ctas=ctas,
                                     stream=side)
-        sep.sep_combine_gated(h, y, wt, out, y_done, seq[0], st_g, num_ctas=ctas, stream=third)
+        sep.sep_combine_gated(h, y, wt, out, y_done, seq[0], st_g, num_ctas=gctas, stream=third)
         sep.sep_dispatch(h, x, recv, tile_ready=tile_ready, dispatch_seq=seq[0])
         main.wait_stream(side)
         main.wait_stream(third)
@@ -636,6 +681,7 @@ def gate_compare(args, w, h, x, idx, wt, recv, dev, steps=50):
         res[name + "_us"] = _time_arm(fn, steps)
         assert st_c.cpu().tolist() == [0, 0] and st_g.cpu().tolist() == [0, 0], (name, st_c, st_g)
     res["delta_pct"] = 100.0 * (res["gated_us"] - res["serial_us"]) / res["serial_us"]
+    res["gate_ctas"] = gctas
     res["note"] = (f"dispatch + reference consumer ({ctas} CTAs, identity experts) + combine after one layout, "
                    "L2 not flushed; the consumer stands in for the expert compute")
     return res

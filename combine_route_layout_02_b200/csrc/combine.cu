@@ -201,80 +201,6 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(CombineParams p)
     }
 }
 
-// Ungated, k <= 8, with 32-byte row loads (sm_100 ld .v8.b32): a lane sums 16
-// channels per load, kWideBatch rows at a time.  Same arithmetic and order.
-constexpr bool kWideVectors = false;
-constexpr int kWideBatch = 2;
-
-struct alignas(32) Vec32 {
-    uint32_t w[8];
-};
-
-__device__ __forceinline__ Vec32 ld_stream32(const Vec32 *ptr)
-{
-    Vec32 v;
-    asm("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-        : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]), "=r"(v.w[5]), "=r"(v.w[6]),
-          "=r"(v.w[7])
-        : "l"(ptr));
-    return v;
-}
-
-__global__ void __launch_bounds__(kWarps * 32) combine_wide_kernel(CombineParams p)
-{
-    grid_dependency_wait();
-    allow_dependents();
-    const int lane = threadIdx.x & 31;
-    const int V = p.H / 16;
-    const int seg = p.seg_len / 2;
-    const int64_t items = p.T * p.segs;
-    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    const Vec32 *y = static_cast<const Vec32 *>(p.y);
-    for (int64_t it = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items; it += nwarps) {
-        const int64_t t = p.T - 1 - it / p.segs;
-        const int s = (int)(it - (p.T - 1 - t) * p.segs);
-        const int v_begin = s * seg;
-        const int v_end = min(V, v_begin + seg);
-        const int my_row = lane < p.k ? __ldg(p.src_pool_row + t * p.k + lane) : -1;
-        const float my_w = lane < p.k ? (p.w ? __ldg(p.w + t * p.k + lane) : 1.f) : 0.f;
-        int rows[kKMax];
-        float ws[kKMax];
-#pragma unroll
-        for (int j = 0; j < kKMax; ++j) {
-            rows[j] = __shfl_sync(kFullMask, my_row, j);
-            ws[j] = __shfl_sync(kFullMask, my_w, j);
-        }
-        Vec32 *out = static_cast<Vec32 *>(p.out) + t * V;
-        for (int v = v_begin + lane; v < v_end; v += 32) {
-            float acc[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                acc[i] = 0.f;
-#pragma unroll
-            for (int j0 = 0; j0 < kKMax; j0 += kWideBatch) {
-                Vec32 buf[kWideBatch];
-#pragma unroll
-                for (int u = 0; u < kWideBatch; ++u)
-                    if (rows[j0 + u] >= 0)
-                        buf[u] = ld_stream32(y + (int64_t)rows[j0 + u] * V + v);
-#pragma unroll
-                for (int u = 0; u < kWideBatch; ++u)
-                    if (rows[j0 + u] >= 0)
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            accumulate_word(acc[2 * i], acc[2 * i + 1], buf[u].w[i], ws[j0 + u]);
-            }
-            Vec32 o;
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                o.w[i] = pack_bf16x2(acc[2 * i], acc[2 * i + 1]);
-            asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
-                         ::"l"(out + v), "r"(o.w[0]), "r"(o.w[1]), "r"(o.w[2]), "r"(o.w[3]), "r"(o.w[4]),
-                           "r"(o.w[5]), "r"(o.w[6]), "r"(o.w[7]) : "memory");
-        }
-    }
-}
-
 }  // namespace
 
 cudaError_t launch_combine(const CombineParams &p, cudaStream_t s, int num_ctas)
@@ -288,10 +214,6 @@ cudaError_t launch_combine(const CombineParams &p, cudaStream_t s, int num_ctas)
         const int64_t n = want < num_ctas ? want : num_ctas;
         return launch_kernel(combine_kernel<true>, dim3((int)n), dim3(kWarps * 32), 0, s, p);
     }
-    const bool wide = kWideVectors && p.k <= kKMax && p.H % 16 == 0 && p.seg_len % 2 == 0 &&
-                      ((reinterpret_cast<uintptr_t>(p.y) | reinterpret_cast<uintptr_t>(p.out)) & 31u) == 0;
-    if (wide)
-        return launch_kernel(combine_wide_kernel, dim3((int)want), dim3(kWarps * 32), 0, s, p);
     return launch_kernel(combine_kernel<false>, dim3((int)want), dim3(kWarps * 32), 0, s, p);
 }
 
@@ -301,8 +223,6 @@ cudaError_t preload_combine_kernels()
     cudaError_t e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(combine_kernel<false>));
     if (e == cudaSuccess)
         e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(combine_kernel<true>));
-    if (e == cudaSuccess)
-        e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(combine_wide_kernel));
     return e;
 }
 

@@ -115,73 +115,6 @@ __global__ void __launch_bounds__(kWarps * 32) dispatch_bf16_kernel(DispatchPara
     }
 }
 
-// bf16 with 32-byte accesses (sm_100 ld/st .v8.b32): the same work items,
-// half the load and store instructions.  Used without tile publication when x
-// and the pool are 32-byte aligned and H is a multiple of 16.
-constexpr bool kWideVectors = false;
-
-struct alignas(32) Vec32 {
-    uint32_t w[8];
-};
-
-__device__ __forceinline__ Vec32 ld_stream32(const Vec32 *ptr)
-{
-    Vec32 v;
-    asm("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-        : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]), "=r"(v.w[5]), "=r"(v.w[6]),
-          "=r"(v.w[7])
-        : "l"(ptr));
-    return v;
-}
-
-__device__ __forceinline__ void st32(Vec32 *ptr, const Vec32 &v)
-{
-    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
-                 ::"l"(ptr), "r"(v.w[0]), "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]),
-                   "r"(v.w[6]), "r"(v.w[7]) : "memory");
-}
-
-template <int UNROLL>
-__global__ void __launch_bounds__(kWarps * 32) dispatch_bf16_wide_kernel(DispatchParams p)
-{
-    grid_dependency_wait();
-    allow_dependents();
-    const int lane = threadIdx.x & 31;
-    const int V = p.H / 16;                              // 32-byte vectors per row
-    const int64_t items = p.T * p.segs;
-    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    const int seg = p.seg_len / 2;                       // seg_len counts 16-byte vectors
-    for (int64_t it = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items; it += nwarps) {
-        const int64_t t = it / p.segs;
-        const int s = (int)(it - t * p.segs);
-        const int v_begin = s * seg;
-        const int v_end = min(V, v_begin + seg);
-        const int my_row = lane < p.k ? __ldg(p.src_pool_row + t * p.k + lane) : -1;
-        const Vec32 *src = static_cast<const Vec32 *>(p.x) + t * V;
-        for (int v0 = v_begin; v0 < v_end; v0 += 32 * UNROLL) {
-            Vec32 buf[UNROLL];
-#pragma unroll
-            for (int u = 0; u < UNROLL; ++u) {
-                const int v = v0 + u * 32 + lane;
-                if (v < v_end)
-                    buf[u] = ld_stream32(src + v);
-            }
-            for (int j = 0; j < p.k; ++j) {
-                const int row = __shfl_sync(kFullMask, my_row, j);
-                if (row < 0)
-                    continue;                            // warp-uniform
-                Vec32 *dst = static_cast<Vec32 *>(p.recv) + (int64_t)row * V;
-#pragma unroll
-                for (int u = 0; u < UNROLL; ++u) {
-                    const int v = v0 + u * 32 + lane;
-                    if (v < v_end)
-                        st32(dst + v, buf[u]);
-                }
-            }
-        }
-    }
-}
-
 // ---------------------------------------------------------------- bulk copy
 //
 // bf16 dispatch through the TMA unit (non-streaming only): a CTA is one warp
@@ -479,11 +412,6 @@ cudaError_t launch_dispatch(const DispatchParams &p, int payload, cudaStream_t s
             return launch_kernel(dispatch_bf16_bulk_kernel, dim3((int)(want < cap ? want : cap)), dim3(32),
                                  (size_t)smem, s, p);
         }
-        const bool wide = kWideVectors && p.tile_ready == nullptr && p.H % 16 == 0 && p.seg_len % 2 == 0 &&
-                          ((reinterpret_cast<uintptr_t>(p.x) | reinterpret_cast<uintptr_t>(p.recv)) & 31u) == 0;
-        if (wide)
-            return launch_kernel(dispatch_bf16_wide_kernel<2>, dim3(blocks_for(0, items, num_sms)),
-                                 dim3(kWarps * 32), 0, s, p);
         if (p.tile_ready != nullptr)
             return launch_kernel(dispatch_bf16_kernel<4, true>, dim3(blocks_for(0, items, num_sms)),
                                  dim3(kWarps * 32), 0, s, p);
@@ -498,7 +426,6 @@ cudaError_t preload_dispatch_kernels()
     const void *k[] = {
         reinterpret_cast<const void *>(dispatch_bf16_bulk_kernel),
         reinterpret_cast<const void *>(dispatch_bf16_kernel<4, false>),
-        reinterpret_cast<const void *>(dispatch_bf16_wide_kernel<2>),
         reinterpret_cast<const void *>(dispatch_bf16_kernel<4, true>),
         reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_F32, false>),
         reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_F32, true>),

@@ -348,10 +348,10 @@ __global__ void __launch_bounds__(kWarps * 32) layout_assign_kernel(LayoutParams
 //      writes the counts, offsets, sizes and owner arrays
 //   C  the warp counts of A become cursors and the chunk is walked again
 //   D  tile tables and padding rows, experts spread over CTAs
-// The barrier arrives with red.release and waits with ld.acquire, bounded; a
+// The barrier arrives with atom.release and waits with ld.acquire, bounded; a
 // barrier that gives up records the epoch in the handle's timeout word and the
-// kernel returns (sep_handle_sync reports it).  Launches of odd and even epochs
-// use different counters, and each launch zeroes the one the next will use.
+// kernel returns (sep_handle_sync reports it).  The counter is never reset:
+// each launch advances it by one fixed window (see grid_barrier).
 
 __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned *ptr)
 {
@@ -367,14 +367,25 @@ __device__ __forceinline__ uint64_t global_ns()
     return t;
 }
 
+// A launch moves the barrier counter by exactly kBarrierWindow, whatever its
+// grid size G (< kBarrierWindow): CTA 0 adds kBarrierWindow - (G - 1), every other CTA
+// adds 1.  So every arrival of one launch returns an old value inside the same
+// window [base, base + kBarrierWindow), the window is found from the old value
+// alone, and the counter never needs a reset: the barrier depends on no host
+// state and stays correct when the launch is replayed from a CUDA graph.
+// 2^32 is a multiple of the window, so the counter may wrap.
+constexpr unsigned kBarrierWindow = 4096;
+
 // All CTAs arrive on *counter; false (in every thread of the CTA) if the
-// counter did not reach target within the limit.
-__device__ __forceinline__ bool grid_barrier(const LayoutParams &p, unsigned *counter, unsigned target,
-                                             int *s_flag)
+// window did not fill within the limit.
+__device__ __forceinline__ bool grid_barrier(const LayoutParams &p, unsigned *counter, int *s_flag)
 {
     __syncthreads();
     if (threadIdx.x == 0) {
-        asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(counter), "r"(1u) : "memory");
+        const unsigned add = blockIdx.x == 0 ? kBarrierWindow - (gridDim.x - 1) : 1u;
+        unsigned old;
+        asm volatile("atom.release.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(counter), "r"(add) : "memory");
+        const unsigned target = (old & ~(kBarrierWindow - 1)) + kBarrierWindow;
         bool ok = false;
         const uint64_t t0 = global_ns();
         for (uint32_t it = 0; it < (1u << 22); ++it) {
@@ -415,9 +426,7 @@ __global__ void __launch_bounds__(kFusedThreads) layout_fused_kernel(LayoutParam
     const int c = blockIdx.x, G = gridDim.x;
     const IdxT *idx = static_cast<const IdxT *>(p.topk_idx);
     allow_dependents();
-    unsigned *counter = p.barrier_words + (p.epoch & 1u);
-    if (c == 0 && tid == 0)
-        p.barrier_words[(p.epoch & 1u) ^ 1u] = 0u;      // the next launch's counter
+    unsigned *counter = p.barrier_words;
     if (c == 0)
         for (int r = tid; r < p.R; r += blockDim.x)
             p.owner_token_counts[r] = 0;
@@ -441,7 +450,7 @@ __global__ void __launch_bounds__(kFusedThreads) layout_fused_kernel(LayoutParam
         }
         p.wchunk_hist[(int64_t)c * hs + e] = sum;
     }
-    if (!grid_barrier(p, counter, (unsigned)G, &s_flag))
+    if (!grid_barrier(p, counter, &s_flag))
         return;
 
     // B. totals and this chunk's prefix, from the whole table
@@ -651,7 +660,7 @@ cudaError_t launch_layout_t(const LayoutParams &p, cudaStream_t s)
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layout_fused_kernel<IdxT>, kFusedThreads,
                                                           smem_fused) == cudaSuccess &&
-            chunks <= per_sm * sms) {
+            chunks <= per_sm * sms && chunks < (int)kBarrierWindow) {
             LayoutParams q = p;
             void *args[] = {&q};
             count_launch();

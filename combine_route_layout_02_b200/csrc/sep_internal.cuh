@@ -39,7 +39,7 @@ struct LayoutParams {
     int64_t *sizes;                  // [2] = {P, NT}
     uint32_t *bad_epoch;             // last epoch that met an id >= E
     uint32_t *timeout_epoch;         // last epoch whose grid barrier gave up
-    uint32_t *barrier_words;         // [2] arrival counters, used on alternate epochs
+    uint32_t *barrier_words;         // [2]: [0] the grid barrier's arrival counter (never reset)
     uint32_t epoch;
 };
 
@@ -260,7 +260,7 @@ struct sep_handle {
     int64_t *sizes;
     uint32_t *bad_epoch;
     uint32_t *timeout_epoch;         // a bounded wait gave up during this epoch
-    uint32_t *barrier_words;         // [2] grid-barrier counters of the single-launch layout
+    uint32_t *barrier_words;         // grid-barrier counter of the single-launch layout
     uint32_t *token_arrivals;        // [T_cap] per-token row counters of the stamping consumer
     // borrowed-view lease and the consumer events its release recorded
     int leased;
