@@ -56,8 +56,8 @@ def parse_args(argv=None):
     ap.add_argument("--consumer-ctas", type=int, default=64)
     ap.add_argument("--gate-ctas", type=int, default=0,
                     help="CTAs of the gated combine in the combine_gate measurement (0: the consumer's)")
-    ap.add_argument("--graph", action="store_true",
-                    help="also time the step replayed from a CUDA graph (non-streaming workloads)")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="skip timing the step replayed from a CUDA graph (non-streaming workloads)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the backward-pair, combine-gate and scatter-combine measurements")
     return ap.parse_args(argv)
@@ -310,12 +310,15 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
     flush = None if flush_buf is None else _Flush()
     n_sms = torch.cuda.get_device_properties(dev).multi_processor_count
 
-    def step(ev=None, xs=x, idxs=idx, wts=wt):
+    def step(ev=None, xs=x, idxs=idx, wts=wt, phases=False):
+        # ev[0] / ev[3] bracket the step; ev[1] / ev[2] split it into phases only
+        # when asked, since an event between two kernels keeps the second from
+        # starting while the first drains (programmatic dependent launch)
         if ev is not None:
             ev[0].record(main)
         sep.sep_layout(idxs, w.E, w.R, w.B, handle=h)
         epoch = h.epoch
-        if ev is not None:
+        if ev is not None and phases:
             ev[1].record(main)
         if w.streaming:
             seq[0] += 1
@@ -325,7 +328,7 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
             sep.sep_dispatch(h, xs, recv, tile_ready=tile_ready, dispatch_seq=seq[0])
         else:
             sep.sep_dispatch(h, xs, recv, payload=w.payload, scale=w.scale, recv_scales=scales)
-        if ev is not None:
+        if ev is not None and phases:
             ev[2].record(main)
         sep.sep_combine(h, y, wts, out, layout_epoch=epoch)
         if ev is not None:
@@ -345,6 +348,8 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
 
     nev = 5 if w.streaming else 4
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    n_phase = min(args.steps, 200)
+    phase_events = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(n_phase)]
     barrier(world)
     torch.cuda.synchronize()
     sampler = ClockSampler(local)
@@ -360,19 +365,30 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
     if w.streaming:
         assert status.cpu().tolist() == [0, 0], f"consumer status {status.cpu().tolist()}"
 
-    graph_ms = replay_step_graph(args, w, step, main, flush, world, dev) if (args.graph and not w.streaming) else None
+    # phase split, in a separate loop (its events cost the step its kernel overlap)
+    for i in range(n_phase):
+        if flush is not None:
+            flush.zero_()
+        step(phase_events[i], phases=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    if w.streaming:
+        assert status.cpu().tolist() == [0, 0], f"consumer status {status.cpu().tolist()}"
 
-    lay_ms = [e[0].elapsed_time(e[1]) for e in events]
-    dis_ms = [e[1].elapsed_time(e[2]) for e in events]
-    com_ms = [e[2].elapsed_time(e[3]) for e in events]
+    graph_ms = replay_step_graph(args, w, step, main, flush, world, dev) if (not args.no_graph and not w.streaming) else None
+
+    lay_ms = [e[0].elapsed_time(e[1]) for e in phase_events]
+    dis_ms = [e[1].elapsed_time(e[2]) for e in phase_events]
+    com_ms = [e[2].elapsed_time(e[3]) for e in phase_events]
+    phased_ms = [e[0].elapsed_time(e[3]) for e in phase_events]
     # the step is layout -> dispatch (with the consumer running beside it on the
     # side stream) -> combine on the main stream; for the streaming workload the
     # time until the consumer has also finished is reported separately
     tot_ms = [e[0].elapsed_time(e[3]) for e in events]
     all_ms = [e[0].elapsed_time(e[nev - 1]) for e in events]
     mean = statistics.fmean
-    local_vals = [mean(tot_ms), mean(lay_ms), mean(dis_ms), mean(com_ms), mean(all_ms)]
-    step_ms, layout_ms, dispatch_ms, combine_ms, with_consumer_ms = reduce_max(local_vals, world, dev)
+    local_vals = [mean(tot_ms), mean(lay_ms), mean(dis_ms), mean(com_ms), mean(all_ms), mean(phased_ms)]
+    step_ms, layout_ms, dispatch_ms, combine_ms, with_consumer_ms, phased_step_ms = reduce_max(local_vals, world, dev)
 
     # end to end through the C ABI: every step uploads its inputs from pinned
     # host memory and downloads its combined output.  Two buffer sets and two
@@ -498,7 +514,10 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
                    "sm_count": n_sms, "timing": "CUDA events per step on the launching stream, mean of steps, max over ranks"},
         "achieved_gbs": step_gbs,
         "pct_of_peak": 100.0 * step_gbs / peaks["hbm_gbs"],
-        "phases_us": {"layout": layout_ms * 1e3, "dispatch": dispatch_ms * 1e3, "combine": combine_ms * 1e3},
+        "phases_us": {"layout": layout_ms * 1e3, "dispatch": dispatch_ms * 1e3, "combine": combine_ms * 1e3,
+                      "step_with_phase_events": phased_step_ms * 1e3, "steps": n_phase,
+                      "note": "a separate loop with an event between phases (which stops each kernel from "
+                              "starting while the previous drains); ms_per_step has events only around the step"},
         "phase_gbs": {"layout": ab["layout"] / (layout_ms * 1e-3) / 1e9,
                       "dispatch": ab["dispatch"] / (dispatch_ms * 1e-3) / 1e9,
                       "combine": ab["combine"] / (combine_ms * 1e-3) / 1e9},
