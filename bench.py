@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import glob
 import json
 import os
@@ -59,7 +60,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-graph", action="store_true",
                     help="skip timing the step replayed from a CUDA graph (non-streaming workloads)")
     ap.add_argument("--no-extras", action="store_true",
-                    help="skip the backward-pair, combine-gate and scatter-combine measurements")
+                    help="skip the borrowed-receive, backward-pair, combine-gate and scatter-combine measurements")
     return ap.parse_args(argv)
 
 
@@ -107,15 +108,20 @@ def load_peaks() -> dict:
         return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
 
 
+KERNEL_PARAMS = {"layout": "LayoutParams", "dispatch": "DispatchParams", "combine": "CombineParams"}
+
+
 def kernel_source_hash(kernel: str) -> str:
-    """Hash of what decides a kernel's memory traffic: its source file, the
-    shared parameter header and the host code that sizes its launch."""
+    """Hash of what decides a kernel's memory traffic: its source file (kernels
+    and launch shape), its parameter struct and the shared row-split helper."""
     csrc = os.path.join(ROOT, "combine_route_layout_02_b200", "csrc")
-    h = hashlib.sha256()
-    for name in (f"{kernel}.cu", "sep_internal.cuh", "sep_api.cu"):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
-    return h.hexdigest()[:16]
+    with open(os.path.join(csrc, "sep_internal.cuh")) as f:
+        header = f.read()
+    parts = [open(os.path.join(csrc, f"{kernel}.cu")).read()]
+    for pattern in (r"struct %s \{.*?\n\};" % KERNEL_PARAMS[kernel], r"inline void split_rows\(.*?\n\}"):
+        m = re.search(pattern, header, flags=re.S)
+        parts.append(m.group(0) if m else "")
+    return hashlib.sha256("\x00".join(parts).encode()).hexdigest()[:16]
 
 
 def profiled_traffic(workload: str, kernel: str):
@@ -476,12 +482,15 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
         e2e_mode = "pipelined: two buffer sets, uploads / kernels / downloads on three streams"
     (e2e_ms,) = reduce_max([e2e_local], world, dev)
     peaks = load_peaks()
-    borrowed = borrow_compare(args, w, h, x, idx, recv, dev) if (w.payload == "bf16" and not w.streaming) else None
+    borrowed = (borrow_compare(args, w, h, x, idx, recv, dev)
+                if (w.payload == "bf16" and not w.streaming and not args.no_extras) else None)
     backward = (backward_compare(w, h, idx, wt, y, None if flush is None else flush.zero_, peaks["hbm_gbs"])
                 if w.payload == "bf16" and not args.no_extras else None)
     gate = gate_compare(args, w, h, x, idx, wt, recv, dev) if w.payload == "bf16" and not args.no_extras else None
     scatter = (scatter_compare(w, h, idx, wt, y, None if flush is None else flush.zero_, peaks["hbm_gbs"])
                if not args.no_extras else None)
+    ep = (ep_compare(w, dev, None if flush is None else flush.zero_, peaks["hbm_gbs"])
+          if w.payload == "bf16" and not w.streaming and not args.no_extras and w.T % w.R == 0 else None)
     sep.sep_handle_free(h)
 
     ab = algorithmic_bytes(w)
@@ -541,6 +550,7 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
         **({"backward": backward} if backward else {}),
         **({"combine_gate": gate} if gate else {}),
         **({"combine_scatter": scatter} if scatter else {}),
+        **({"ep_emulated": ep} if ep else {}),
         "clocks": sampler.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -647,6 +657,61 @@ def scatter_compare(w, h, idx, wt, y, flush, peak_gbs, steps=100):
             "delta_pct": 100.0 * (scatter_us - gather_us) / gather_us,
             "note": "same combine bytes for both (the scatter also writes out's zeros first); "
                     "L2 flushed before every call"}
+
+
+def ep_compare(w, dev, flush, peak_gbs, steps=100):
+    """Expert parallelism across the workload's R owners as ranks, emulated on
+    one GPU: the workload's T tokens split into R rank shards of T/R (own
+    seeds), each rank laid out alone, the counts planned, then every rank's
+    dispatch into the owners' pools and every rank's combine from them (the
+    kernels a multi-GPU group runs with peer pointers).  Against the
+    single-GPU dispatch + combine of the same tokens concatenated (same rows,
+    same bytes).  Layouts and the plan are outside the timed region in both."""
+    import numpy as np
+    import torch
+    import combine_route_layout_02_b200 as sep
+    R, Tr = w.R, w.T // w.R
+    shards = [W.make_inputs(replace(w, T=Tr, seed=w.seed + 7919 * (r + 1))) for r in range(R)]
+    hs = [sep.sep_layout(sd["topk_idx"].to(dev), w.E, R, w.B, flags=sep.SEP_LAYOUT_SYNC_COUNTS) for sd in shards]
+    counts = np.stack([h.view("expert_counts").cpu().numpy() for h in hs]).astype(np.int32)
+    plans = [sep.sep_ep_plan(counts, r, w.B) for r in range(R)]
+    rows = [int(v) for v in plans[0]["owner_rows"]]
+    pools = [torch.empty(max(n, 1), w.H, dtype=torch.bfloat16, device=dev) for n in rows]
+    deltas = [torch.from_numpy(p["delta"]).to(dev) for p in plans]
+    xs = [sd["x"].to(dev) for sd in shards]
+    ws = [sd["topk_weight"].to(dev) for sd in shards]
+    outs = [torch.empty(Tr, w.H, dtype=torch.bfloat16, device=dev) for _ in range(R)]
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def ep_step():
+        for r in range(R):
+            sep.sep_ep_dispatch(hs[r], xs[r], r, deltas[r], pools, rows, err)
+        for r in range(R):
+            sep.sep_ep_combine(hs[r], pools, rows, deltas[r], ws[r], outs[r], err)
+
+    idx_cat = torch.cat([sd["topk_idx"] for sd in shards]).to(dev)
+    x_cat = torch.cat([sd["x"] for sd in shards]).to(dev)
+    w_cat = torch.cat([sd["topk_weight"] for sd in shards]).to(dev)
+    h1 = sep.sep_layout(idx_cat, w.E, R, w.B, flags=sep.SEP_LAYOUT_SYNC_COUNTS)
+    pool1 = torch.empty(h1.info().num_pool_rows, w.H, dtype=torch.bfloat16, device=dev)
+    out1 = torch.empty(R * Tr, w.H, dtype=torch.bfloat16, device=dev)
+
+    def single_step():
+        sep.sep_dispatch(h1, x_cat, pool1)
+        sep.sep_combine(h1, pool1, w_cat, out1)
+
+    ep_us = _time_arm(ep_step, steps, flush)
+    single_us = _time_arm(single_step, steps, flush)
+    assert int(err.item()) == 0, "a row fell outside its owner's pool"
+    for h in hs + [h1]:
+        sep.sep_handle_free(h)
+    b = algorithmic_bytes(replace(w, T=R * Tr))
+    moved = b["dispatch"] + b["combine"]
+    return {"ranks": R, "tokens_per_rank": Tr, "ep_us": ep_us, "single_gpu_us": single_us,
+            "ep_gbs": moved / (ep_us * 1e-6) / 1e9, "ep_frac": moved / (ep_us * 1e-6) / 1e9 / peak_gbs,
+            "note": "R ranks emulated on one GPU (2R launches: every rank's dispatch, then every rank's combine, "
+                    "into / from the owners' pools); single_gpu is the same tokens' dispatch + combine; "
+                    "layouts outside the timed region; L2 flushed before every step"}
 
 
 _gate_seq = [1 << 20]

@@ -165,11 +165,14 @@ int blocks_for(int64_t warp_items)
 
 }  // namespace
 
-cudaError_t launch_dispatch_grads(const DispatchGradsParams &p, cudaStream_t s, int num_sms)
+cudaError_t launch_dispatch_grads(DispatchGradsParams p, cudaStream_t s, int num_sms)
 {
     if (p.T == 0)
         return cudaSuccess;
-    (void)num_sms;
+    // without grad_w, rows split into the forward dispatch's 128-vector steps, one item each
+    int64_t steps = 1;
+    split_rows(p.T, ((p.H / 8) + 127) / 128, (int64_t)num_sms * 32, 1 << 20, &p.segs, &steps);
+    p.seg_len = (int)(steps * 128);
     if (p.grad_w)
         return launch_kernel(dispatch_grads_dot_kernel, dim3(blocks_for(p.T * p.k)), dim3(kWarps * 32), 0, s, p);
     return launch_kernel(dispatch_grads_kernel, dim3(blocks_for(p.T * p.segs)), dim3(kWarps * 32), 0, s, p);

@@ -203,11 +203,20 @@ __global__ void __launch_bounds__(kWarps * 32) combine_kernel(CombineParams p)
 
 }  // namespace
 
-cudaError_t launch_combine(const CombineParams &p, cudaStream_t s, int num_ctas)
+cudaError_t launch_combine(CombineParams p, cudaStream_t s, int num_sms, int num_ctas)
 {
-    const int64_t items = p.T * p.segs;
-    if (items == 0)
+    if (p.T == 0)
         return cudaSuccess;
+    if (p.y_done) {
+        p.segs = 1;                                      // a token is either reduced or left unwritten
+        p.seg_len = p.H / 8;
+    } else {
+        // steps of 32 vectors (one per lane); rows split only when tokens are too few to fill the GPU
+        int64_t steps = 1;
+        split_rows(p.T, ((p.H / 8) + 31) / 32, (int64_t)num_sms * 32, 1, &p.segs, &steps);
+        p.seg_len = (int)(steps * 32);
+    }
+    const int64_t items = p.T * p.segs;
     const int64_t want = (items + kWarps - 1) / kWarps;
     if (p.y_done) {
         // persistent: at most num_ctas CTAs, so that the producer keeps its SMs

@@ -387,11 +387,28 @@ cudaError_t launch_fp8(const DispatchParams &p, cudaStream_t s, int num_sms)
 
 }  // namespace
 
-cudaError_t launch_dispatch(const DispatchParams &p, int payload, cudaStream_t s, int num_sms)
+// Row splitting.  A bf16 step is 128 vectors of 16 bytes (one pass of the
+// kernel's 4-deep unroll); without tile publication every step is its own work
+// item, so the items divide finely over the waves of CTAs (measured faster
+// than whole rows per warp).  With tile publication a row stays on one warp
+// where possible, since every item pays a fence and one arrival per row.  FP8
+// steps are 512 channels, and a row splits over up to 7 warps.
+constexpr int64_t kStepVecs = 128;
+constexpr int64_t kMinSegs = 1 << 20;
+constexpr int64_t kPublishMinSegs = 1;
+constexpr int64_t kFp8MinSegs = 7;
+
+cudaError_t launch_dispatch(DispatchParams p, int payload, cudaStream_t s, int num_sms)
 {
-    const int64_t items = p.T * p.segs;
-    if (items == 0)
+    if (p.T == 0)
         return cudaSuccess;
+    const bool fp8 = payload != SEP_PAYLOAD_BF16;
+    const int64_t units = fp8 ? (p.H + 511) / 512 : ((p.H / 8) + kStepVecs - 1) / kStepVecs;
+    int64_t steps = 1;
+    split_rows(p.T, units, (int64_t)num_sms * 32, fp8 ? kFp8MinSegs : (p.tile_ready ? kPublishMinSegs : kMinSegs),
+               &p.segs, &steps);
+    p.seg_len = (int)(fp8 ? steps : steps * kStepVecs);
+    const int64_t items = p.T * p.segs;
     if (payload == SEP_PAYLOAD_BF16) {
         const int64_t smem = (int64_t)kBulkStages * p.H * 2;
         if (kBulkDispatch && p.tile_ready == nullptr && smem <= kBulkMaxSmem) {

@@ -1,0 +1,258 @@
+// Expert parallelism across ranks over peer memory (StreamEP README, "What's
+// in the box": intranode dispatch / combine on NVLink; the "DeepEP MoE
+// dispatch/combine" blog, "一轮 DeepEP 数据流": each rank sends its tokens to
+// the ranks that own their experts, the receiver lays them out by local expert,
+// and combine brings the expert outputs back to the source token).
+//
+// Rank r (of R) holds its own tokens and routing; owner o = rank o holds
+// experts [o*E/R, (o+1)*E/R).  Owner o's pool is expert-major and
+// BLOCK_M-padded over its own experts; inside expert e the rows are ordered by
+// (source rank, token, slot), the stable order the single-GPU layout gives to
+// the concatenation of all ranks' tokens in rank order.  So with counts[r][e]
+// the valid assignments of rank r to expert e (exchanged between ranks):
+//   N_e        = sum_r counts[r][e],  tau_e = ceil(N_e / B)
+//   gboff[e]   = sum of tau over owner(e)'s experts before e   (tiles)
+//   row(r,t,j) = gboff[e]*B + sum_{r' < r} counts[r'][e] + s
+// where s is the assignment's stable index among rank r's assignments to e,
+// which the rank's own layout already holds: its local row is
+// loff_r[e]*B + s.  The plan is therefore one shift per (rank, expert),
+//   delta_r[e] = gboff[e]*B + sum_{r' < r} counts[r'][e] - loff_r[e]*B,
+// computed on the host from the exchanged counts (sep_ep_plan).
+//
+// The dispatch writes each token row straight into the owner's pool through
+// the owner's pointer (a peer pointer on another GPU, plain stores over
+// NVLink; no TMA, no multicast) together with the owner's receive map
+// (token, rank, slot); the owner marks its own padding rows.  The combine
+// gathers each token's k rows from the owners' expert-output pools the same
+// way (peer loads) and reduces them exactly as the single-GPU combine does.
+#include <cuda_bf16.h>
+
+#include "sep_internal.cuh"
+
+namespace sep {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kUnroll = 4;
+constexpr int kRowBatch = 4;
+
+__device__ __forceinline__ uint4 ld_stream(const uint4 *ptr)
+{
+    uint4 v;
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "l"(ptr));
+    return v;
+}
+
+// Global row of assignment (t, j) of this rank in its owner's pool, and the
+// owner; -1 for a masked assignment or (with *err set) a row outside the
+// owner's pool or an owner outside the group.
+template <typename P>
+__device__ __forceinline__ int64_t owner_row(const P &p, int64_t a, int *owner)
+{
+    const int local = __ldg(p.src_pool_row + a);
+    if (local < 0)
+        return -1;
+    const int e = __ldg(p.tile_expert + local / p.B);
+    const int o = e / p.E_loc;
+    const int64_t row = (int64_t)local + __ldg(p.delta + e);
+    if (o >= p.R || row < 0 || row >= p.pool_rows[o]) {
+        atomicExch(p.error, 1u);
+        return -1;
+    }
+    *owner = o;
+    return row;
+}
+
+// bf16 dispatch into the owners' pools: a work item is (token, segment).
+__global__ void __launch_bounds__(kWarps * 32) ep_dispatch_kernel(EpDispatchParams p)
+{
+    grid_dependency_wait();
+    allow_dependents();
+    const int lane = threadIdx.x & 31;
+    const int V = p.H / 8;
+    const int64_t items = p.T * p.segs;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t it = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items; it += nwarps) {
+        const int64_t t = it / p.segs;
+        const int s = (int)(it - t * p.segs);
+        const int v_begin = s * p.seg_len;
+        const int v_end = min(V, v_begin + p.seg_len);
+        int my_owner = 0;
+        const int64_t my_row = lane < p.k ? owner_row(p, t * p.k + lane, &my_owner) : -1;
+        uint4 *my_dst = my_row >= 0 ? static_cast<uint4 *>(p.pools[my_owner]) + my_row * V : nullptr;
+        if (s == 0 && my_row >= 0) {                     // the owner's receive map, once per assignment
+            if (p.recv_token[my_owner])
+                p.recv_token[my_owner][my_row] = (int32_t)t;
+            if (p.recv_rank[my_owner])
+                p.recv_rank[my_owner][my_row] = p.rank;
+            if (p.recv_slot[my_owner])
+                p.recv_slot[my_owner][my_row] = lane;
+        }
+        const uint4 *src = static_cast<const uint4 *>(p.x) + t * V;
+        for (int v0 = v_begin; v0 < v_end; v0 += 32 * kUnroll) {
+            uint4 buf[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int v = v0 + u * 32 + lane;
+                buf[u] = v < v_end ? ld_stream(src + v) : make_uint4(0, 0, 0, 0);
+            }
+            for (int j = 0; j < p.k; ++j) {
+                uint4 *dst = reinterpret_cast<uint4 *>(
+                    __shfl_sync(kFullMask, reinterpret_cast<unsigned long long>(my_dst), j));
+                if (dst == nullptr)
+                    continue;                            // warp-uniform
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v < v_end)
+                        dst[v] = buf[u];
+                }
+            }
+        }
+    }
+}
+
+// Owner side: -1 in the receive map on the padding rows of its pool.
+__global__ void __launch_bounds__(256) ep_mark_padding_kernel(EpPaddingParams p)
+{
+    grid_dependency_wait();
+    allow_dependents();
+    const int64_t n = p.pool_rows;
+    for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < n; r += (int64_t)gridDim.x * blockDim.x) {
+        const int tile = (int)(r / p.B);
+        int lo = 0, hi = p.E_loc;                        // expert e with block_offset[e] <= tile < block_offset[e+1]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldg(p.block_offset + mid) <= tile)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        const int64_t slot = r - (int64_t)__ldg(p.block_offset + lo) * p.B;
+        if (slot >= __ldg(p.expert_counts + lo)) {
+            if (p.recv_token)
+                p.recv_token[r] = -1;
+            if (p.recv_rank)
+                p.recv_rank[r] = -1;
+            if (p.recv_slot)
+                p.recv_slot[r] = -1;
+        }
+    }
+}
+
+__device__ __forceinline__ void accumulate_word(float &lo, float &hi, uint32_t word, float w)
+{
+    lo = __fadd_rn(lo, __fmul_rn(w, __uint_as_float(word << 16)));
+    hi = __fadd_rn(hi, __fmul_rn(w, __uint_as_float(word & 0xffff0000u)));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    const uint32_t l = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+    const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+    return l | (h << 16);
+}
+
+// Combine from the owners' expert outputs: a warp owns (token, segment); the
+// k row pointers and weights are broadcast into registers once; fp32 sums in
+// ascending j, as the single-GPU combine.
+__global__ void __launch_bounds__(kWarps * 32) ep_combine_kernel(EpCombineParams p)
+{
+    grid_dependency_wait();
+    allow_dependents();
+    const int lane = threadIdx.x & 31;
+    const int V = p.H / 8;
+    const int64_t items = p.T * p.segs;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t it = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items; it += nwarps) {
+        const int64_t t = it / p.segs;
+        const int s = (int)(it - t * p.segs);
+        const int v_begin = s * p.seg_len;
+        const int v_end = min(V, v_begin + p.seg_len);
+        int my_owner = 0;
+        const int64_t my_row = lane < p.k ? owner_row(p, t * p.k + lane, &my_owner) : -1;
+        const uint4 *my_src = my_row >= 0 ? static_cast<const uint4 *>(p.y_pools[my_owner]) + my_row * V : nullptr;
+        const float my_w = lane < p.k ? __ldg(p.w + t * p.k + lane) : 0.f;
+        uint4 *out = static_cast<uint4 *>(p.out) + t * V;
+        for (int v0 = v_begin; v0 < v_end; v0 += 32) {
+            const int v = v0 + lane;
+            const bool act = v < v_end;
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int j0 = 0; j0 < p.k; j0 += kRowBatch) {
+                uint4 buf[kRowBatch];
+                const uint4 *src[kRowBatch];
+#pragma unroll
+                for (int u = 0; u < kRowBatch; ++u) {
+                    const int j = j0 + u;
+                    src[u] = reinterpret_cast<const uint4 *>(
+                        __shfl_sync(kFullMask, reinterpret_cast<unsigned long long>(my_src), j & 31));
+                    if (j >= p.k)
+                        src[u] = nullptr;
+                    buf[u] = (src[u] != nullptr && act) ? ld_stream(src[u] + v) : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < kRowBatch; ++u) {
+                    const float w = __shfl_sync(kFullMask, my_w, (j0 + u) & 31);
+                    if (src[u] != nullptr) {
+                        accumulate_word(acc[0], acc[1], buf[u].x, w);
+                        accumulate_word(acc[2], acc[3], buf[u].y, w);
+                        accumulate_word(acc[4], acc[5], buf[u].z, w);
+                        accumulate_word(acc[6], acc[7], buf[u].w, w);
+                    }
+                }
+            }
+            if (act)
+                out[v] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                    pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_ep_dispatch(EpDispatchParams p, cudaStream_t s, int num_sms)
+{
+    if (p.T == 0)
+        return cudaSuccess;
+    int64_t steps = 1;                                   // 128-vector steps, as the single-GPU dispatch
+    split_rows(p.T, ((p.H / 8) + 127) / 128, (int64_t)num_sms * 32, 1 << 20, &p.segs, &steps);
+    p.seg_len = (int)(steps * 128);
+    const int64_t items = p.T * p.segs;
+    return launch_kernel(ep_dispatch_kernel, dim3((int)((items + kWarps - 1) / kWarps)), dim3(kWarps * 32), 0, s, p);
+}
+
+cudaError_t launch_ep_mark_padding(const EpPaddingParams &p, cudaStream_t s, int num_sms)
+{
+    if (p.pool_rows == 0)
+        return cudaSuccess;
+    int64_t blocks = (p.pool_rows + 255) / 256;
+    if (blocks > (int64_t)num_sms * 8)
+        blocks = (int64_t)num_sms * 8;
+    return launch_kernel(ep_mark_padding_kernel, dim3((int)blocks), dim3(256), 0, s, p);
+}
+
+cudaError_t launch_ep_combine(EpCombineParams p, cudaStream_t s, int num_sms)
+{
+    if (p.T == 0)
+        return cudaSuccess;
+    int64_t steps = 1;                                   // 32-vector steps, as the single-GPU combine
+    split_rows(p.T, ((p.H / 8) + 31) / 32, (int64_t)num_sms * 32, 1, &p.segs, &steps);
+    p.seg_len = (int)(steps * 32);
+    const int64_t items = p.T * p.segs;
+    return launch_kernel(ep_combine_kernel, dim3((int)((items + kWarps - 1) / kWarps)), dim3(kWarps * 32), 0, s, p);
+}
+
+cudaError_t preload_ep_kernels()
+{
+    cudaFuncAttributes a;
+    cudaError_t e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(ep_dispatch_kernel));
+    if (e == cudaSuccess)
+        e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(ep_mark_padding_kernel));
+    if (e == cudaSuccess)
+        e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(ep_combine_kernel));
+    return e;
+}
+
+}  // namespace sep

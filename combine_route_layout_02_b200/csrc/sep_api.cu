@@ -105,6 +105,8 @@ sep_status preload_once(int dev)
         e = sep::preload_backward_kernels();
     if (e == cudaSuccess)
         e = sep::preload_scatter_kernels();
+    if (e == cudaSuccess)
+        e = sep::preload_ep_kernels();
     if (e != cudaSuccess)
         return cuda_fail(e, "loading the library's kernels");
     if (dev >= 0 && dev < 64)
@@ -206,35 +208,6 @@ sep_status create(int64_t T_cap, int k, int E, int R, int B, uint32_t flags, cud
     *out = h;
     return SEP_OK;
 }
-
-// Work items of the dispatch and combine kernels are (token, segment of a
-// row).  A row of `units` warp-steps is split so that there are at least
-// `want_warps` items and at least `min_segs` segments per row; returns the
-// segment count and the steps per segment.
-void split_rows(int64_t T, int64_t units, int64_t want_warps, int64_t min_segs, int *segs, int64_t *steps)
-{
-    int64_t n = (want_warps + T - 1) / T;
-    if (n < min_segs)
-        n = min_segs;
-    if (n > units)
-        n = units;
-    if (n < 1)
-        n = 1;
-    *steps = (units + n - 1) / n;
-    *segs = (int)((units + *steps - 1) / *steps);
-}
-
-// Row splitting.  A bf16 dispatch step is 128 vectors of 16 bytes (one pass of
-// the kernel's 4-deep unroll); without tile publication every step is its own
-// work item, so the items divide finely over the waves of CTAs (measured
-// faster than whole rows per warp).  With tile publication a row stays on one
-// warp where possible, since every item pays a fence and one arrival per row.
-// FP8 steps are 512 channels; combine steps are 32 vectors.
-constexpr int64_t kDispatchStepVecs = 128;
-constexpr int64_t kDispatchMinSegs = 1 << 20;
-constexpr int64_t kDispatchPublishMinSegs = 1;
-constexpr int64_t kDispatchFp8MinSegs = 7;
-constexpr int64_t kCombineMinSegs = 1;
 
 // A borrowed view leases the handle's row map to its consumers.
 sep_status check_not_leased(const sep_handle *h)
@@ -577,12 +550,6 @@ sep_status sep_dispatch(sep_handle *h, const void *x, int64_t hidden, int payloa
     p.seq = dispatch_seq;
     p.error_epoch = h->timeout_epoch;
     p.epoch = h->epoch;
-    // split a token row over several warps when there are too few tokens to fill the GPU
-    const int64_t units = fp8 ? (hidden + 511) / 512 : ((hidden / 8) + kDispatchStepVecs - 1) / kDispatchStepVecs;
-    int64_t steps = 1;
-    const int64_t min_segs = fp8 ? kDispatchFp8MinSegs : (tile_ready ? kDispatchPublishMinSegs : kDispatchMinSegs);
-    split_rows(h->T, units, (int64_t)num_sms * 32, min_segs, &p.segs, &steps);
-    p.seg_len = (int)(fp8 ? steps : steps * kDispatchStepVecs);
     cudaError_t e = sep::launch_dispatch(p, payload, s, num_sms);
     return e == cudaSuccess ? SEP_OK : cuda_fail(e, "dispatch launch");
 }
@@ -628,7 +595,6 @@ sep_status prepare_combine(const sep_handle *h, uint32_t layout_epoch, const voi
         return SEP_OK;
     const_cast<sep_handle *>(h)->last_stream = s;
 
-    const int num_sms = sep::device_sm_count();
     *p = sep::CombineParams{};
     p->y = y;
     p->T = h->T;
@@ -639,10 +605,6 @@ sep_status prepare_combine(const sep_handle *h, uint32_t layout_epoch, const voi
     p->out = out;
     p->error_epoch = h->timeout_epoch;
     p->epoch = h->epoch;
-    const int64_t units = ((hidden / 8) + 31) / 32;
-    int64_t steps = 1;
-    split_rows(h->T, units, (int64_t)num_sms * 32, kCombineMinSegs, &p->segs, &steps);
-    p->seg_len = (int)(steps * 32);
     return SEP_OK;
 }
 
@@ -664,7 +626,7 @@ sep_status sep_combine(const sep_handle *h, uint32_t layout_epoch, const void *y
                                     &p, &empty);
     if (st != SEP_OK || empty)
         return st;
-    cudaError_t e = sep::launch_combine(p, s, 0);
+    cudaError_t e = sep::launch_combine(p, s, sep::device_sm_count(), 0);
     return e == cudaSuccess ? SEP_OK : cuda_fail(e, "combine launch");
 }
 
@@ -692,12 +654,7 @@ sep_status sep_combine_scatter(const sep_handle *h, uint32_t layout_epoch, const
     p.out = out;
     p.num_pool_rows = h->sizes;
     p.rows_cap = needed_rows(h);
-    // a pool row splits into the dispatch's 4 KB steps
-    const int64_t units = ((hidden / 8) + kDispatchStepVecs - 1) / kDispatchStepVecs;
-    int64_t steps = 1;
-    split_rows(p.rows_cap, units, (int64_t)num_sms * 32, kDispatchMinSegs, &p.segs, &steps);
-    p.seg_len = (int)(steps * kDispatchStepVecs);
-    e = sep::launch_combine_scatter(p, s);
+    e = sep::launch_combine_scatter(p, s, num_sms);
     return e == cudaSuccess ? SEP_OK : cuda_fail(e, "scatter combine launch");
 }
 
@@ -711,7 +668,7 @@ sep_status sep_combine_grads(const sep_handle *h, uint32_t layout_epoch, const v
                                     &p, &empty);
     if (st != SEP_OK || empty)
         return st;
-    cudaError_t e = sep::launch_combine(p, s, 0);
+    cudaError_t e = sep::launch_combine(p, s, sep::device_sm_count(), 0);
     return e == cudaSuccess ? SEP_OK : cuda_fail(e, "combine_grads launch");
 }
 
@@ -745,15 +702,12 @@ sep_status sep_combine_gated(const sep_handle *h, uint32_t layout_epoch, const v
         return cuda_fail(e, "cudaMemsetAsync (status)");
     if (empty)
         return SEP_OK;
-    // a warp reduces a whole token, so a token is either reduced or left unwritten
-    p.segs = 1;
-    p.seg_len = (int)(hidden / 8);
     p.y_done = y_done;
     p.done_seq = done_seq;
     p.timeout_ns = timeout_ns ? timeout_ns : 1000000000ull;
     p.max_polls = poll_budget(p.timeout_ns);
     p.status = status;
-    e = sep::launch_combine(p, s, num_ctas);
+    e = sep::launch_combine(p, s, sep::device_sm_count(), num_ctas);
     return e == cudaSuccess ? SEP_OK : cuda_fail(e, "gated combine launch");
 }
 
@@ -807,11 +761,6 @@ sep_status sep_dispatch_grads(const sep_handle *h, uint32_t layout_epoch, const 
     p.H = (int)hidden;
     p.k = h->k;
     p.src_pool_row = h->src_pool_row;
-    // without grad_w, rows split into the forward dispatch's steps
-    const int64_t units = ((hidden / 8) + kDispatchStepVecs - 1) / kDispatchStepVecs;
-    int64_t steps = 1;
-    split_rows(h->T, units, (int64_t)num_sms * 32, kDispatchMinSegs, &p.segs, &steps);
-    p.seg_len = (int)(steps * kDispatchStepVecs);
     cudaError_t e = sep::launch_dispatch_grads(p, s, num_sms);
     return e == cudaSuccess ? SEP_OK : cuda_fail(e, "dispatch_grads launch");
 }
@@ -989,6 +938,243 @@ sep_status sep_gather_rows(const sep_recv_view *view, void *dst, int64_t dst_row
     p.indexed = v.indexed ? 1 : 0;
     const cudaError_t e = sep::launch_gather(p, static_cast<cudaStream_t>(stream), sep::device_sm_count());
     return e == cudaSuccess ? SEP_OK : cuda_fail(e, "gather launch");
+}
+
+// ------------------------------------------------------- expert parallelism
+
+
+sep_status sep_ep_plan(const int32_t *all_counts, int num_ranks, int num_experts, int block_m, int rank,
+                       int32_t *delta, int64_t *owner_rows, int32_t *owner_block_offset,
+                       int32_t *owner_expert_counts)
+{
+    if (all_counts == nullptr || delta == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "NULL all_counts or delta");
+    if (num_ranks < 1 || num_ranks > 1024 || num_experts < 1 || num_experts > 1024 ||
+        num_experts % num_ranks != 0)
+        return fail(SEP_ERR_INVALID_ARG, "need 1 <= num_ranks <= 1024, num_experts in 1..1024 divisible by num_ranks");
+    if (block_m < 1 || block_m > 1024)
+        return fail(SEP_ERR_INVALID_ARG, "block_m must be in 1..1024");
+    if (rank < 0 || rank >= num_ranks)
+        return fail(SEP_ERR_INVALID_ARG, "rank %d outside 0..%d", rank, num_ranks - 1);
+    const int R = num_ranks, E = num_experts, El = E / R, B = block_m;
+    for (int64_t i = 0; i < (int64_t)R * E; ++i)
+        if (all_counts[i] < 0)
+            return fail(SEP_ERR_INVALID_ARG, "all_counts[%lld] is negative", (long long)i);
+    int64_t loff = 0;                                    // this rank's local block offset (tiles), running over e
+    int64_t gboff = 0;                                   // owner-local block offset of e (tiles)
+    for (int e = 0; e < E; ++e) {
+        if (e % El == 0) {
+            if (e > 0 && owner_rows != nullptr)
+                owner_rows[e / El - 1] = gboff * B;
+            gboff = 0;
+        }
+        int64_t N = 0, before = 0;
+        for (int r = 0; r < R; ++r) {
+            const int64_t c = all_counts[(int64_t)r * E + e];
+            if (r < rank)
+                before += c;
+            N += c;
+        }
+        const int64_t own = all_counts[(int64_t)rank * E + e];
+        const int64_t d = gboff * B + before - loff * B;
+        if (N > INT32_MAX || d > INT32_MAX || d < INT32_MIN || (gboff + (N + B - 1) / B) * B > INT32_MAX)
+            return fail(SEP_ERR_INVALID_ARG, "counts too large for 32-bit pool rows");
+        delta[e] = (int32_t)d;
+        if (e / El == rank) {
+            if (owner_block_offset != nullptr)
+                owner_block_offset[e % El] = (int32_t)gboff;
+            if (owner_expert_counts != nullptr)
+                owner_expert_counts[e % El] = (int32_t)N;
+        }
+        gboff += (N + B - 1) / B;
+        loff += (own + B - 1) / B;
+        if (e == E - 1) {
+            if (owner_rows != nullptr)
+                owner_rows[R - 1] = gboff * B;
+        }
+        if (e / El == rank && e % El == El - 1 && owner_block_offset != nullptr)
+            owner_block_offset[El] = (int32_t)gboff;
+    }
+    return SEP_OK;
+}
+
+namespace {
+
+// Checks shared by sep_ep_dispatch and sep_ep_combine, and the rank-group
+// part of their parameters.
+struct EpCommon {
+    int64_t T;
+    int H, k, B, E_loc, R;
+    const int32_t *src_pool_row, *tile_expert, *delta;
+    uint32_t *error;
+    int64_t pool_rows[sep::kEpMaxRanks];
+};
+
+sep_status ep_common(const sep_handle *h, uint32_t layout_epoch, int64_t hidden, const int32_t *delta,
+                     const int64_t *pool_rows, uint32_t *error, EpCommon *c)
+{
+    if (h == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "NULL handle");
+    sep_status st = check_device(h);
+    if (st != SEP_OK)
+        return st;
+    if (layout_epoch != h->epoch)
+        return fail(SEP_ERR_HANDLE_MISMATCH, "handle epoch is %u, caller's routing has epoch %u",
+                    h->epoch, layout_epoch);
+    if ((st = check_not_leased(h)) != SEP_OK)
+        return st;
+    if (h->R > sep::kEpMaxRanks)
+        return fail(SEP_ERR_INVALID_ARG, "an expert-parallel group has at most %d ranks (the handle has %d owners)",
+                    sep::kEpMaxRanks, h->R);
+    if (hidden < 1 || hidden > 65536 || hidden % 8 != 0)
+        return fail(SEP_ERR_INVALID_ARG, "hidden must be a multiple of 8 in 1..65536 (got %lld)",
+                    (long long)hidden);
+    if (delta == nullptr || pool_rows == nullptr || error == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "NULL delta, pool_rows or error");
+    if (((reinterpret_cast<uintptr_t>(delta) | reinterpret_cast<uintptr_t>(error)) & 3u) != 0)
+        return fail(SEP_ERR_INVALID_ARG, "delta and error must be 4-byte aligned");
+    c->T = h->T;
+    c->H = (int)hidden;
+    c->k = h->k;
+    c->B = h->B;
+    c->E_loc = h->E / h->R;
+    c->R = h->R;
+    c->src_pool_row = h->src_pool_row;
+    c->tile_expert = h->tile_expert;
+    c->delta = delta;
+    c->error = error;
+    for (int r = 0; r < h->R; ++r) {
+        if (pool_rows[r] < 0 || pool_rows[r] > INT32_MAX)
+            return fail(SEP_ERR_INVALID_ARG, "pool_rows[%d] = %lld is outside 0..2^31-1", r, (long long)pool_rows[r]);
+        c->pool_rows[r] = pool_rows[r];
+    }
+    return SEP_OK;
+}
+
+}  // namespace
+
+sep_status sep_ep_dispatch(const sep_handle *h, uint32_t layout_epoch, const void *x, int64_t hidden, int rank,
+                           const int32_t *delta, void *const *pools, const int64_t *pool_rows,
+                           int32_t *const *recv_token, int32_t *const *recv_rank, int32_t *const *recv_slot,
+                           uint32_t *error, void *stream)
+{
+    EpCommon c;
+    sep_status st = ep_common(h, layout_epoch, hidden, delta, pool_rows, error, &c);
+    if (st != SEP_OK)
+        return st;
+    sep::EpDispatchParams p{};
+    p.T = c.T;
+    p.H = c.H;
+    p.k = c.k;
+    p.B = c.B;
+    p.E_loc = c.E_loc;
+    p.R = c.R;
+    p.src_pool_row = c.src_pool_row;
+    p.tile_expert = c.tile_expert;
+    p.delta = c.delta;
+    p.error = c.error;
+    memcpy(p.pool_rows, c.pool_rows, sizeof(p.pool_rows));
+    if (rank < 0 || rank >= h->R)
+        return fail(SEP_ERR_INVALID_ARG, "rank %d outside 0..%d", rank, h->R - 1);
+    if (pools == nullptr || (h->T > 0 && x == nullptr))
+        return fail(SEP_ERR_INVALID_ARG, "NULL pools or x");
+    if (!aligned16(x))
+        return fail(SEP_ERR_INVALID_ARG, "x must be 16-byte aligned");
+    for (int r = 0; r < h->R; ++r) {
+        if ((pool_rows[r] > 0 && pools[r] == nullptr) || !aligned16(pools[r]))
+            return fail(SEP_ERR_INVALID_ARG, "pools[%d] must be non-NULL (if it has rows) and 16-byte aligned", r);
+        p.pools[r] = pools[r];
+        p.recv_token[r] = recv_token ? recv_token[r] : nullptr;
+        p.recv_rank[r] = recv_rank ? recv_rank[r] : nullptr;
+        p.recv_slot[r] = recv_slot ? recv_slot[r] : nullptr;
+        if (((reinterpret_cast<uintptr_t>(p.recv_token[r]) | reinterpret_cast<uintptr_t>(p.recv_rank[r]) |
+              reinterpret_cast<uintptr_t>(p.recv_slot[r])) & 3u) != 0)
+            return fail(SEP_ERR_INVALID_ARG, "receive maps of rank %d must be 4-byte aligned", r);
+    }
+    p.x = x;
+    p.rank = rank;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = wait_for_release(const_cast<sep_handle *>(h), s, false)) != SEP_OK)
+        return st;
+    if (h->T == 0)
+        return SEP_OK;
+    const_cast<sep_handle *>(h)->last_stream = s;
+    const cudaError_t e = sep::launch_ep_dispatch(p, s, sep::device_sm_count());
+    return e == cudaSuccess ? SEP_OK : cuda_fail(e, "expert-parallel dispatch launch");
+}
+
+sep_status sep_ep_mark_padding(int num_local_experts, int block_m, const int32_t *owner_block_offset,
+                               const int32_t *owner_expert_counts, int64_t pool_rows, int32_t *recv_token,
+                               int32_t *recv_rank, int32_t *recv_slot, void *stream)
+{
+    if (num_local_experts < 1 || num_local_experts > 1024 || block_m < 1 || block_m > 1024)
+        return fail(SEP_ERR_INVALID_ARG, "need num_local_experts and block_m in 1..1024");
+    if (pool_rows < 0 || pool_rows > INT32_MAX)
+        return fail(SEP_ERR_INVALID_ARG, "pool_rows outside 0..2^31-1");
+    if (pool_rows > 0 && (owner_block_offset == nullptr || owner_expert_counts == nullptr))
+        return fail(SEP_ERR_INVALID_ARG, "NULL owner_block_offset or owner_expert_counts");
+    if (((reinterpret_cast<uintptr_t>(owner_block_offset) | reinterpret_cast<uintptr_t>(owner_expert_counts) |
+          reinterpret_cast<uintptr_t>(recv_token) | reinterpret_cast<uintptr_t>(recv_rank) |
+          reinterpret_cast<uintptr_t>(recv_slot)) & 3u) != 0)
+        return fail(SEP_ERR_INVALID_ARG, "arrays must be 4-byte aligned");
+    int dev = -1;
+    sep_status st = current_device(&dev);
+    if (st != SEP_OK)
+        return st;
+    if ((st = preload_once(dev)) != SEP_OK)
+        return st;
+    sep::EpPaddingParams p{};
+    p.E_loc = num_local_experts;
+    p.B = block_m;
+    p.block_offset = owner_block_offset;
+    p.expert_counts = owner_expert_counts;
+    p.pool_rows = pool_rows;
+    p.recv_token = recv_token;
+    p.recv_rank = recv_rank;
+    p.recv_slot = recv_slot;
+    const cudaError_t e = sep::launch_ep_mark_padding(p, static_cast<cudaStream_t>(stream), sep::device_sm_count());
+    return e == cudaSuccess ? SEP_OK : cuda_fail(e, "padding launch");
+}
+
+sep_status sep_ep_combine(const sep_handle *h, uint32_t layout_epoch, const void *const *y_pools,
+                          const int64_t *pool_rows, int64_t hidden, const int32_t *delta, const float *topk_weight,
+                          void *out, uint32_t *error, void *stream)
+{
+    EpCommon c;
+    sep_status st = ep_common(h, layout_epoch, hidden, delta, pool_rows, error, &c);
+    if (st != SEP_OK)
+        return st;
+    sep::EpCombineParams p{};
+    p.T = c.T;
+    p.H = c.H;
+    p.k = c.k;
+    p.B = c.B;
+    p.E_loc = c.E_loc;
+    p.R = c.R;
+    p.src_pool_row = c.src_pool_row;
+    p.tile_expert = c.tile_expert;
+    p.delta = c.delta;
+    p.error = c.error;
+    memcpy(p.pool_rows, c.pool_rows, sizeof(p.pool_rows));
+    if (y_pools == nullptr || (h->T > 0 && (topk_weight == nullptr || out == nullptr)))
+        return fail(SEP_ERR_INVALID_ARG, "NULL y_pools, topk_weight or out");
+    if (!aligned16(out) || (reinterpret_cast<uintptr_t>(topk_weight) & 3u) != 0)
+        return fail(SEP_ERR_INVALID_ARG, "out must be 16-byte aligned, topk_weight 4-byte aligned");
+    for (int r = 0; r < h->R; ++r) {
+        if ((pool_rows[r] > 0 && y_pools[r] == nullptr) || !aligned16(y_pools[r]))
+            return fail(SEP_ERR_INVALID_ARG, "y_pools[%d] must be non-NULL (if it has rows) and 16-byte aligned", r);
+        p.y_pools[r] = y_pools[r];
+    }
+    p.w = topk_weight;
+    p.out = out;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = wait_for_release(const_cast<sep_handle *>(h), s, false)) != SEP_OK)
+        return st;
+    if (h->T == 0)
+        return SEP_OK;
+    const_cast<sep_handle *>(h)->last_stream = s;
+    const cudaError_t e = sep::launch_ep_combine(p, s, sep::device_sm_count());
+    return e == cudaSuccess ? SEP_OK : cuda_fail(e, "expert-parallel combine launch");
 }
 
 void sep_handle_free(sep_handle *h)

@@ -10,6 +10,23 @@ namespace sep {
 
 constexpr unsigned kFullMask = 0xffffffffu;
 
+// Work items of the row kernels are (row, segment of the row).  A row of
+// `units` warp-steps is split so that there are at least `want_warps` items
+// and at least `min_segs` segments per row (never more segments than steps);
+// returns the segment count and the steps per segment.
+inline void split_rows(int64_t rows, int64_t units, int64_t want_warps, int64_t min_segs, int *segs, int64_t *steps)
+{
+    int64_t n = rows > 0 ? (want_warps + rows - 1) / rows : 1;
+    if (n < min_segs)
+        n = min_segs;
+    if (n > units)
+        n = units;
+    if (n < 1)
+        n = 1;
+    *steps = (units + n - 1) / n;
+    *segs = (int)((units + *steps - 1) / *steps);
+}
+
 // ----------------------------------------------------------------- layout
 
 // CTA chunks of the assignment stream: CTA c of the count / assign kernels
@@ -58,7 +75,7 @@ struct DispatchParams {
     void *recv;                      // [rows][H] bf16 or e4m3
     void *recv_scales;               // [rows][H/128] f32 or u8
     int scale;                       // sep_scale
-    int segs;                        // warps sharing one token row
+    int segs;                        // warps sharing one token row (set by launch_dispatch)
     int seg_len;                     // per warp: 16-byte vectors (bf16) or 512-channel steps (fp8)
     // streaming publication (tile_ready != nullptr)
     uint32_t *tile_ready;
@@ -70,7 +87,7 @@ struct DispatchParams {
     uint32_t epoch;
 };
 
-cudaError_t launch_dispatch(const DispatchParams &p, int payload, cudaStream_t s, int num_sms);
+cudaError_t launch_dispatch(DispatchParams p, int payload, cudaStream_t s, int num_sms);
 
 // -------------------------------------------------------- backward pair
 
@@ -87,7 +104,7 @@ struct DispatchGradsParams {
     int seg_len;                     // 16-byte vectors per warp
 };
 
-cudaError_t launch_dispatch_grads(const DispatchGradsParams &p, cudaStream_t s, int num_sms);
+cudaError_t launch_dispatch_grads(DispatchGradsParams p, cudaStream_t s, int num_sms);
 cudaError_t preload_backward_kernels();
 
 // ---------------------------------------------------------------- combine
@@ -111,7 +128,8 @@ struct CombineParams {
     uint32_t *status;                // [2]: code, tokens not reduced
 };
 
-cudaError_t launch_combine(const CombineParams &p, cudaStream_t s, int num_sms);
+// num_ctas bounds the persistent grid of the gated variant (y_done != nullptr)
+cudaError_t launch_combine(CombineParams p, cudaStream_t s, int num_sms, int num_ctas);
 
 // ---------------------------------------------------- atomic-scatter combine
 
@@ -128,8 +146,58 @@ struct ScatterParams {
     int seg_len;                     // 16-byte vectors per warp
 };
 
-cudaError_t launch_combine_scatter(const ScatterParams &p, cudaStream_t s);
+cudaError_t launch_combine_scatter(ScatterParams p, cudaStream_t s, int num_sms);
 cudaError_t preload_scatter_kernels();
+
+// ------------------------------------------------- expert parallelism (ranks)
+
+// Ranks of one expert-parallel group (the per-rank pointers travel in the
+// kernel parameters, so the host can check them).
+constexpr int kEpMaxRanks = 64;
+
+struct EpDispatchParams {
+    const void *x;                   // bf16 [T][H], this rank's tokens
+    int64_t T;
+    int H, k, B, E_loc, R;
+    const int32_t *src_pool_row;     // this rank's layout: local row of (t, j)
+    const int32_t *tile_expert;      // this rank's layout: expert of each local tile
+    const int32_t *delta;            // [E] global-row shift of this rank's rows of expert e
+    int rank;
+    uint32_t *error;                 // set to 1 when a row falls outside its owner's pool
+    int segs, seg_len;               // set by launch_ep_dispatch
+    int64_t pool_rows[kEpMaxRanks];  // rows of each owner's pool
+    void *pools[kEpMaxRanks];        // owners' pools (bf16 rows; peer pointers on other GPUs)
+    int32_t *recv_token[kEpMaxRanks];   // owners' receive maps (entries may be nullptr)
+    int32_t *recv_rank[kEpMaxRanks];
+    int32_t *recv_slot[kEpMaxRanks];
+};
+
+struct EpPaddingParams {
+    int E_loc, B;
+    const int32_t *block_offset;     // [E_loc + 1] tiles, this owner's pool
+    const int32_t *expert_counts;    // [E_loc] valid rows of each expert
+    int64_t pool_rows;
+    int32_t *recv_token, *recv_rank, *recv_slot;   // this owner's maps (each may be nullptr)
+};
+
+struct EpCombineParams {
+    int64_t T;
+    int H, k, B, E_loc, R;
+    const int32_t *src_pool_row;
+    const int32_t *tile_expert;
+    const int32_t *delta;
+    const float *w;                  // [T][k]
+    void *out;                       // bf16 [T][H]
+    uint32_t *error;
+    int segs, seg_len;               // set by launch_ep_combine
+    int64_t pool_rows[kEpMaxRanks];
+    const void *y_pools[kEpMaxRanks];   // owners' expert outputs (bf16 rows)
+};
+
+cudaError_t launch_ep_dispatch(EpDispatchParams p, cudaStream_t s, int num_sms);
+cudaError_t launch_ep_mark_padding(const EpPaddingParams &p, cudaStream_t s, int num_sms);
+cudaError_t launch_ep_combine(EpCombineParams p, cudaStream_t s, int num_sms);
+cudaError_t preload_ep_kernels();
 
 // --------------------------------------------------------------- consumer
 

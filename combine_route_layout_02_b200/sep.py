@@ -84,6 +84,10 @@ _SIGNATURES = [
     ("sep_dispatch_grads", _i32, [_P, _u32, _P, _i64, _P, _P, _i64, _P, _i64, _P, _P]),
     ("sep_combine_grads", _i32, [_P, _u32, _P, _i64, _i64, _P, _P]),
     ("sep_combine_scatter", _i32, [_P, _u32, _P, _i64, _i64, _P, _P, _P]),
+    ("sep_ep_plan", _i32, [_P, _i32, _i32, _i32, _i32, _P, _P, _P, _P]),
+    ("sep_ep_dispatch", _i32, [_P, _u32, _P, _i64, _i32, _P, _P, _P, _P, _P, _P, _P, _P]),
+    ("sep_ep_mark_padding", _i32, [_i32, _i32, _P, _P, _i64, _P, _P, _P, _P]),
+    ("sep_ep_combine", _i32, [_P, _u32, _P, _P, _i64, _P, _P, _P, _P, _P]),
 ]
 
 
@@ -252,6 +256,62 @@ def sep_consume_tiles(handle: Handle, recv_x: torch.Tensor, tile_ready: torch.Te
     _check(_lib.sep_consume_tiles(handle.ptr, _ptr(recv_x), row_bytes, recv_x.shape[0], _ptr(tile_ready),
                                   tile_ready.numel(), dispatch_seq, _ptr(dst), num_ctas, timeout_ns,
                                   _ptr(status), _stream(stream)), "sep_consume_tiles")
+
+
+def sep_ep_plan(all_counts, rank: int, block_m: int) -> dict:
+    """Host-only plan from every rank's expert counts (numpy int32 [R, E]):
+    delta [E], owner_rows [R], owner_block_offset [E/R + 1], owner_expert_counts [E/R]."""
+    import numpy as np
+    counts = np.ascontiguousarray(np.asarray(all_counts, dtype=np.int32))
+    R, E = counts.shape
+    El = E // R if R > 0 and E % R == 0 else 1
+    delta = np.zeros(E, np.int32)
+    rows = np.zeros(R, np.int64)
+    boff = np.zeros(El + 1, np.int32)
+    ecnt = np.zeros(El, np.int32)
+    _check(_lib.sep_ep_plan(counts.ctypes.data, R, E, block_m, rank, delta.ctypes.data, rows.ctypes.data,
+                            boff.ctypes.data, ecnt.ctypes.data), "sep_ep_plan")
+    return {"delta": delta, "owner_rows": rows, "owner_block_offset": boff, "owner_expert_counts": ecnt}
+
+
+def _ptr_array(tensors):
+    arr = (ctypes.c_void_p * len(tensors))()
+    for i, t in enumerate(tensors):
+        arr[i] = None if t is None else t.data_ptr()
+    return arr
+
+
+def sep_ep_dispatch(handle: Handle, x: torch.Tensor, rank: int, delta: torch.Tensor, pools, pool_rows,
+                    error: torch.Tensor, recv_token=None, recv_rank=None, recv_slot=None,
+                    layout_epoch: int | None = None, stream=None) -> None:
+    """Rows of this rank's tokens into the owners' pools (lists of R device tensors)."""
+    if x.dtype != torch.bfloat16 or delta.dtype != torch.int32:
+        raise ValueError("x must be bf16 and delta int32")
+    R = len(pools)
+    rows = (ctypes.c_int64 * R)(*[int(r) for r in pool_rows])
+    maps = [None if m is None else _ptr_array(m) for m in (recv_token, recv_rank, recv_slot)]
+    epoch = handle.epoch if layout_epoch is None else layout_epoch
+    _check(_lib.sep_ep_dispatch(handle.ptr, epoch, _ptr(x), x.shape[1], rank, _ptr(delta), _ptr_array(pools), rows,
+                                maps[0], maps[1], maps[2], _ptr(error), _stream(stream)), "sep_ep_dispatch")
+
+
+def sep_ep_mark_padding(owner_block_offset: torch.Tensor, owner_expert_counts: torch.Tensor, block_m: int,
+                        pool_rows: int, recv_token=None, recv_rank=None, recv_slot=None, stream=None) -> None:
+    _check(_lib.sep_ep_mark_padding(owner_expert_counts.numel(), block_m, _ptr(owner_block_offset),
+                                    _ptr(owner_expert_counts), int(pool_rows), _ptr(recv_token), _ptr(recv_rank),
+                                    _ptr(recv_slot), _stream(stream)), "sep_ep_mark_padding")
+
+
+def sep_ep_combine(handle: Handle, y_pools, pool_rows, delta: torch.Tensor, topk_weight: torch.Tensor,
+                   out: torch.Tensor, error: torch.Tensor, layout_epoch: int | None = None, stream=None) -> None:
+    """out[t] = bf16(sum_j w[t,j] * y_pools[owner][row(t,j)]) from the owners' expert outputs."""
+    if out.dtype != torch.bfloat16 or topk_weight.dtype != torch.float32:
+        raise ValueError("out must be bf16 and topk_weight fp32")
+    R = len(y_pools)
+    rows = (ctypes.c_int64 * R)(*[int(r) for r in pool_rows])
+    epoch = handle.epoch if layout_epoch is None else layout_epoch
+    _check(_lib.sep_ep_combine(handle.ptr, epoch, _ptr_array(y_pools), rows, out.shape[1], _ptr(delta),
+                               _ptr(topk_weight), _ptr(out), _ptr(error), _stream(stream)), "sep_ep_combine")
 
 
 def sep_combine_scatter(handle: Handle, y_pool: torch.Tensor, topk_weight: torch.Tensor, out: torch.Tensor,

@@ -430,6 +430,88 @@ SEP_API sep_status sep_view_release(sep_handle *handle, void *const *streams, in
  */
 SEP_API sep_status sep_gather_rows(const sep_recv_view *view, void *dst, int64_t dst_rows, void *stream);
 
+/*
+ * Expert parallelism across ranks over peer memory (StreamEP README, "What's
+ * in the box": intranode dispatch / combine over NVLink; "DeepEP MoE
+ * dispatch/combine" blog, "一轮 DeepEP 数据流": tokens go to the ranks that
+ * own their experts, the receiver groups them by local expert, combine brings
+ * the expert outputs back).
+ *
+ * R ranks (at most 64); rank o owns experts [o*E/R, (o+1)*E/R).  Each rank lays
+ * out its own routing with sep_layout(num_owners = R).  Owner o's pool is
+ * expert-major and BLOCK_M-padded over its own experts, and inside an expert
+ * the rows are ordered by (source rank, token, slot): exactly owner o's segment
+ * of the single-GPU layout of all ranks' tokens concatenated in rank order.
+ * A pool is any device memory of this or a peer GPU (a peer pointer from CUDA
+ * IPC or symmetric memory); rows are written and read with plain stores and
+ * loads (no TMA, no multicast).  Between the dispatches of all ranks and the
+ * owners' expert compute, and between that and the combines, the caller
+ * synchronises the ranks (a barrier or a collective).
+ */
+
+/*
+ * sep_ep_plan — host-only: the per-rank row shift from every rank's expert
+ * counts.  Calls no CUDA function.
+ *
+ *  all_counts           host int32 [num_ranks, num_experts]: row r is rank r's
+ *                       expert_counts (exchanged between ranks, e.g. by an all-gather).
+ *  delta                host int32 [num_experts], out: a row of this rank's layout
+ *                       at local row L (expert e) goes to row L + delta[e] of its
+ *                       owner's pool.
+ *  owner_rows           host int64 [num_ranks] or NULL, out: pool rows of each owner.
+ *  owner_block_offset   host int32 [E/R + 1] or NULL, out: this rank's pool, tile
+ *                       offset of each local expert (for its grouped GEMM).
+ *  owner_expert_counts  host int32 [E/R] or NULL, out: valid rows of each local expert.
+ * SEP_ERR_INVALID_ARG for a size out of range, a negative count or a pool
+ * that would not fit 32-bit rows.
+ */
+SEP_API sep_status sep_ep_plan(const int32_t *all_counts, int num_ranks, int num_experts, int block_m, int rank,
+                               int32_t *delta, int64_t *owner_rows, int32_t *owner_block_offset,
+                               int32_t *owner_expert_counts);
+
+/*
+ * sep_ep_dispatch — copies this rank's token rows into their owners' pools
+ * (bf16), and writes each owner's receive map entry: recv_token = source
+ * token, recv_rank = this rank, recv_slot = top-k slot.
+ *
+ *  handle, layout_epoch  this rank's layout (num_owners = R) and its epoch.
+ *  rank                  this rank (0..R-1).
+ *  delta                 device int32 [E]: sep_ep_plan's delta for this rank.
+ *  pools, pool_rows      host arrays [R]: each owner's pool (device bf16
+ *                        [pool_rows[o], hidden], 16-byte aligned) and its rows.
+ *  recv_token, recv_rank, recv_slot
+ *                        host arrays [R] of device int32 [pool_rows[o]] maps, or
+ *                        NULL (an entry may be NULL too).
+ *  error                 device uint32: set to 1 when a row falls outside its
+ *                        owner's pool (the write is skipped; a wrong delta or a
+ *                        short pool is never written past).
+ */
+SEP_API sep_status sep_ep_dispatch(const sep_handle *handle, uint32_t layout_epoch, const void *x, int64_t hidden,
+                                   int rank, const int32_t *delta, void *const *pools, const int64_t *pool_rows,
+                                   int32_t *const *recv_token, int32_t *const *recv_rank, int32_t *const *recv_slot,
+                                   uint32_t *error, void *stream);
+
+/*
+ * sep_ep_mark_padding — owner side: -1 in the receive maps (each may be NULL)
+ * on the padding rows of this owner's pool, from sep_ep_plan's
+ * owner_block_offset and owner_expert_counts (device copies).  Touches no
+ * valid row, so it may run while other ranks dispatch.
+ */
+SEP_API sep_status sep_ep_mark_padding(int num_local_experts, int block_m, const int32_t *owner_block_offset,
+                                       const int32_t *owner_expert_counts, int64_t pool_rows, int32_t *recv_token,
+                                       int32_t *recv_rank, int32_t *recv_slot, void *stream);
+
+/*
+ * sep_ep_combine — out[t] = bf16( sum over valid j, ascending, of
+ * topk_weight[t, j] * y_pools[owner][row(t, j)] ) with fp32 products and sums:
+ * sep_combine over the owners' expert-output pools (host array [R] of device
+ * bf16 [pool_rows[o], hidden], 16-byte aligned).  Other arguments as
+ * sep_ep_dispatch.
+ */
+SEP_API sep_status sep_ep_combine(const sep_handle *handle, uint32_t layout_epoch, const void *const *y_pools,
+                                  const int64_t *pool_rows, int64_t hidden, const int32_t *delta,
+                                  const float *topk_weight, void *out, uint32_t *error, void *stream);
+
 /* Frees the handle.  Its device memory is released stream-ordered on the
  * stream of the last call that used it; the caller must have ordered every
  * other stream that used the handle before that point.  NULL is a no-op; a
