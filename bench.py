@@ -56,7 +56,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--consumer-ctas", type=int, default=64)
     ap.add_argument("--gate-ctas", type=int, default=0,
-                    help="CTAs of the gated combine in the combine_gate measurement (0: the consumer's)")
+                    help="CTAs of the gated combine in the combine_gate measurement (0: one per SM)")
     ap.add_argument("--no-graph", action="store_true",
                     help="skip timing the step replayed from a CUDA graph (non-streaming workloads)")
     ap.add_argument("--no-extras", action="store_true",
@@ -738,7 +738,7 @@ def gate_compare(args, w, h, x, idx, wt, recv, dev, steps=50):
     st_g = torch.zeros(2, dtype=torch.int32, device=dev)
     seq = _gate_seq                                      # advances across calls: tile_ready may reuse an address
     ctas = args.consumer_ctas
-    gctas = args.gate_ctas or ctas
+    gctas = args.gate_ctas or torch.cuda.get_device_properties(dev).multi_processor_count
 
     def serial():
         seq[0] += 1

@@ -347,7 +347,8 @@ __global__ void __launch_bounds__(kWarps * 32) layout_assign_kernel(LayoutParams
 //      ceil(n_e / BLOCK_M) over experts follows in shared memory; CTA 0
 //      writes the counts, offsets, sizes and owner arrays
 //   C  the warp counts of A become cursors and the chunk is walked again
-//   D  tile tables and padding rows, experts spread over CTAs
+//   D  tile tables and padding rows, one warp per expert
+// A routing small enough for one CTA chunk skips the table and the barrier.
 // The barrier arrives with atom.release and waits with ld.acquire, bounded; a
 // barrier that gives up records the epoch in the handle's timeout word and the
 // kernel returns (sep_handle_sync reports it).  The counter is never reset:
@@ -405,6 +406,8 @@ __device__ __forceinline__ bool grid_barrier(const LayoutParams &p, unsigned *co
     return *s_flag != 0;
 }
 
+constexpr int64_t kSingleCtaMaxNa = 1024;     // routings this small run as one CTA chunk
+
 constexpr int kFusedThreads = kWarps * 32;
 constexpr int kRedInts = 1024;               // per reduction table: row groups x padded experts
 
@@ -441,6 +444,18 @@ __global__ void __launch_bounds__(kFusedThreads) layout_fused_kernel(LayoutParam
     if (__any_sync(kFullMask, bad) && lane == 0)
         atomicMax(p.bad_epoch, p.epoch);
     __syncthreads();
+    if (G == 1) {
+        // one chunk: the totals are this CTA's own counts; no table, no grid barrier
+        for (int e = tid; e < E; e += blockDim.x) {
+            int sum = 0;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w)
+                sum += s_cnt[w * E + e];
+            s_tot[e] = sum;
+            s_pre[e] = 0;
+        }
+        __syncthreads();
+    } else {
     for (int e = tid; e < hs; e += blockDim.x) {
         int sum = 0;
         if (e < E) {
@@ -502,6 +517,7 @@ __global__ void __launch_bounds__(kFusedThreads) layout_fused_kernel(LayoutParam
             }
             __syncthreads();
         }
+    }
     }
 
     // tile offsets over experts (each thread a run of experts), in shared memory
@@ -596,17 +612,18 @@ __global__ void __launch_bounds__(kFusedThreads) layout_fused_kernel(LayoutParam
         }
     }
 
-    // D. tile tables and padding rows; experts spread over CTAs
-    for (int e = c; e < E; e += G) {
+    // D. tile tables and padding rows; one warp per expert, experts spread over
+    // the warps of all CTAs
+    for (int e = c * kWarps + warp; e < E; e += G * kWarps) {
         const int t0 = s_off[e], t1 = s_off[e + 1];
         const int n = s_tot[e];
-        for (int i = tid; i < t1 - t0; i += blockDim.x) {
+        for (int i = lane; i < t1 - t0; i += 32) {
             p.tile_expert[t0 + i] = e;
             p.pool_arrival_target[t0 + i] = min(p.B, n - i * p.B);
             p.pool_arrival_count[t0 + i] = 0u;
         }
         const int64_t r1 = (int64_t)t1 * p.B;
-        for (int64_t row = (int64_t)t0 * p.B + n + tid; row < r1; row += blockDim.x) {
+        for (int64_t row = (int64_t)t0 * p.B + n + lane; row < r1; row += 32) {
             p.pool_recv_token[row] = -1;
             p.pool_recv_slot[row] = -1;
         }
@@ -683,6 +700,11 @@ cudaError_t launch_layout_t(const LayoutParams &p, cudaStream_t s)
 
 int layout_rounds_for(int64_t Na)
 {
+    // small routings: one CTA chunk, which needs neither the chunk table nor the
+    // grid barrier (measured: 256 assignments, 17.6 -> 15.4 us per step; at
+    // 2048 assignments and 256 experts one CTA is slower than eight)
+    if (Na <= kSingleCtaMaxNa)
+        return (int)(Na > 0 ? (Na + 32LL * kWarps - 1) / (32LL * kWarps) : 1);
     // at most 128 CTA chunks of 8 warps; 1..64 rounds of 32 assignments per warp
     const int64_t per_round = 32LL * kWarps * 128;
     int64_t r = (Na + per_round - 1) / per_round;
