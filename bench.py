@@ -59,6 +59,8 @@ def parse_args(argv=None):
                     help="CTAs of the gated combine in the combine_gate measurement (0: one per SM)")
     ap.add_argument("--no-graph", action="store_true",
                     help="skip timing the step replayed from a CUDA graph (non-streaming workloads)")
+    ap.add_argument("--extras", default="borrowed,backward,gate,scatter,ep",
+                    help="comma list of the measurements taken after the timed region")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the borrowed-receive, backward-pair, combine-gate and scatter-combine measurements")
     return ap.parse_args(argv)
@@ -482,15 +484,20 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
         e2e_mode = "pipelined: two buffer sets, uploads / kernels / downloads on three streams"
     (e2e_ms,) = reduce_max([e2e_local], world, dev)
     peaks = load_peaks()
+    extras = set() if args.no_extras else set(args.extras.split(","))
+
+    def want(name):
+        return name in extras
+
     borrowed = (borrow_compare(args, w, h, x, idx, recv, dev)
-                if (w.payload == "bf16" and not w.streaming and not args.no_extras) else None)
+                if (w.payload == "bf16" and not w.streaming and want("borrowed")) else None)
     backward = (backward_compare(w, h, idx, wt, y, None if flush is None else flush.zero_, peaks["hbm_gbs"])
-                if w.payload == "bf16" and not args.no_extras else None)
-    gate = gate_compare(args, w, h, x, idx, wt, recv, dev) if w.payload == "bf16" and not args.no_extras else None
+                if w.payload == "bf16" and want("backward") else None)
+    gate = gate_compare(args, w, h, x, idx, wt, recv, dev) if w.payload == "bf16" and want("gate") else None
     scatter = (scatter_compare(w, h, idx, wt, y, None if flush is None else flush.zero_, peaks["hbm_gbs"])
-               if not args.no_extras else None)
+               if want("scatter") else None)
     ep = (ep_compare(w, dev, None if flush is None else flush.zero_, peaks["hbm_gbs"])
-          if w.payload == "bf16" and not w.streaming and not args.no_extras and w.T % w.R == 0 else None)
+          if w.payload == "bf16" and not w.streaming and want("ep") and w.T % w.R == 0 else None)
     sep.sep_handle_free(h)
 
     ab = algorithmic_bytes(w)
