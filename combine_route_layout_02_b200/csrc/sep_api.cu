@@ -1177,6 +1177,52 @@ sep_status sep_ep_combine(const sep_handle *h, uint32_t layout_epoch, const void
     return e == cudaSuccess ? SEP_OK : cuda_fail(e, "expert-parallel combine launch");
 }
 
+sep_status sep_ep_buffer_alloc(int64_t bytes, void **ptr, void *ipc_handle)
+{
+    if (ptr == nullptr || ipc_handle == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "NULL ptr or ipc_handle");
+    if (bytes < 1)
+        return fail(SEP_ERR_INVALID_ARG, "bytes must be positive");
+    *ptr = nullptr;
+    void *p = nullptr;
+    cudaError_t e = cudaMalloc(&p, (size_t)bytes);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaMalloc (expert-parallel buffer)");
+    cudaIpcMemHandle_t hd;
+    e = cudaIpcGetMemHandle(&hd, p);
+    if (e != cudaSuccess) {
+        cudaFree(p);
+        return cuda_fail(e, "cudaIpcGetMemHandle");
+    }
+    static_assert(sizeof(cudaIpcMemHandle_t) == SEP_IPC_HANDLE_BYTES, "IPC handle size");
+    memcpy(ipc_handle, &hd, sizeof(hd));
+    *ptr = p;
+    return SEP_OK;
+}
+
+sep_status sep_ep_buffer_open(const void *ipc_handle, void **ptr)
+{
+    if (ptr == nullptr || ipc_handle == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "NULL ptr or ipc_handle");
+    *ptr = nullptr;
+    cudaIpcMemHandle_t hd;
+    memcpy(&hd, ipc_handle, sizeof(hd));
+    void *p = nullptr;
+    const cudaError_t e = cudaIpcOpenMemHandle(&p, hd, cudaIpcMemLazyEnablePeerAccess);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaIpcOpenMemHandle");
+    *ptr = p;
+    return SEP_OK;
+}
+
+sep_status sep_ep_buffer_close(void *ptr, int opened)
+{
+    if (ptr == nullptr)
+        return SEP_OK;
+    const cudaError_t e = opened ? cudaIpcCloseMemHandle(ptr) : cudaFree(ptr);
+    return e == cudaSuccess ? SEP_OK : cuda_fail(e, opened ? "cudaIpcCloseMemHandle" : "cudaFree");
+}
+
 void sep_handle_free(sep_handle *h)
 {
     if (h == nullptr)

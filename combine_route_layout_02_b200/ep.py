@@ -1,0 +1,133 @@
+"""Expert parallelism across processes: the host side around the EP kernels.
+
+One process per rank (normally one per GPU; several may share one GPU).  Rank
+o owns experts [o*E/R, (o+1)*E/R).  Each step:
+
+1. the rank lays out its own routing (``sep_layout`` with num_owners = R);
+2. the ranks exchange their expert counts (an all-gather of E integers, the
+   one collective of the path) and each computes its plan (``sep_ep_plan``);
+3. each owner marks the padding rows of its pool; a barrier;
+4. each rank writes its token rows straight into the owners' pools through
+   their pointers (``sep_ep_dispatch``); a barrier;
+5. the owners compute their experts' outputs into their shared y buffers;
+   a barrier;
+6. each rank reads its tokens' k output rows from the owners' y buffers and
+   reduces them (``sep_ep_combine``); a barrier before the buffers are reused.
+
+The pools, y buffers and receive maps are allocated by the library and shared
+by CUDA IPC (plain device memory mapped into every peer; no multicast).  The
+barriers follow a device synchronisation, so no kernel ever waits on another
+process's kernel.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+from . import sep as _sep
+
+
+def _pool_rows_cap(world: int, max_tokens: int, top_k: int, num_local_experts: int, block_m: int) -> int:
+    """Rows of an owner's pool that hold any routing: every assignment of every
+    rank on this owner, plus at most block_m - 1 padding rows per local expert."""
+    n = world * max_tokens * top_k
+    rows = n + min(num_local_experts, n) * (block_m - 1)
+    return max((rows + block_m - 1) // block_m * block_m, block_m)
+
+
+class EPGroup:
+    """Dispatch and combine across the ranks of a torch.distributed group."""
+
+    def __init__(self, num_experts: int, top_k: int, block_m: int, hidden: int, max_tokens: int, group=None):
+        self.group = group
+        self.rank = dist.get_rank(group)
+        self.world = dist.get_world_size(group)
+        if num_experts % self.world != 0:
+            raise ValueError("num_experts must be divisible by the number of ranks")
+        self.E, self.k, self.B, self.H = num_experts, top_k, block_m, hidden
+        self.E_loc = num_experts // self.world
+        self.rows_cap = _pool_rows_cap(self.world, max_tokens, top_k, self.E_loc, block_m)
+        self.cpu_collectives = dist.get_backend(group) != "nccl"
+        own = [_sep.sep_ep_buffer_alloc(self.rows_cap * hidden * 2),   # pool
+               _sep.sep_ep_buffer_alloc(self.rows_cap * hidden * 2),   # expert outputs y
+               _sep.sep_ep_buffer_alloc(3 * self.rows_cap * 4)]        # receive maps: token, rank, slot
+        handles = [None] * self.world
+        dist.all_gather_object(handles, [b.handle for b in own], group=group)
+        self.buffers = []                                # [rank] -> [pool, y, maps]
+        for r in range(self.world):
+            if r == self.rank:
+                self.buffers.append(own)
+            else:
+                self.buffers.append([_sep.sep_ep_buffer_open(h, b.nbytes) for h, b in zip(handles[r], own)])
+        shape = (self.rows_cap, hidden)
+        self.pools = [bufs[0].tensor(shape, torch.bfloat16) for bufs in self.buffers]
+        self.ys = [bufs[1].tensor(shape, torch.bfloat16) for bufs in self.buffers]
+        maps = [bufs[2].tensor((3, self.rows_cap), torch.int32) for bufs in self.buffers]
+        self.recv_token = [m[0] for m in maps]
+        self.recv_rank = [m[1] for m in maps]
+        self.recv_slot = [m[2] for m in maps]
+        self.handle = _sep.sep_handle_create(max_tokens, top_k, num_experts, self.world, block_m)
+        self.error = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.plan = None
+        self._barrier()
+
+    def _barrier(self):
+        torch.cuda.synchronize()                         # this process's kernels are done first
+        dist.barrier(group=self.group)
+
+    def _all_counts(self) -> np.ndarray:
+        mine = self.handle.view("expert_counts").to(torch.int32)
+        if self.cpu_collectives:
+            mine = mine.cpu()
+        out = [torch.zeros_like(mine) for _ in range(self.world)]
+        dist.all_gather(out, mine, group=self.group)
+        return torch.stack(out).cpu().numpy()
+
+    def dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor):
+        """Steps 1-4; returns this owner's received rows [P_o, H] (a view of its
+        pool) and receive maps (token, rank, slot), each [P_o]."""
+        _sep.sep_layout(topk_idx, self.E, self.world, self.B, handle=self.handle)
+        plan = _sep.sep_ep_plan(self._all_counts(), self.rank, self.B)
+        rows = [int(v) for v in plan["owner_rows"]]
+        if max(rows) > self.rows_cap:
+            raise RuntimeError(f"an owner needs {max(rows)} pool rows, the group holds {self.rows_cap}")
+        self.plan = plan
+        self.rows = rows
+        self.delta = torch.from_numpy(plan["delta"]).cuda()
+        _sep.sep_ep_mark_padding(torch.from_numpy(plan["owner_block_offset"]).cuda(),
+                                 torch.from_numpy(plan["owner_expert_counts"]).cuda(), self.B, rows[self.rank],
+                                 self.recv_token[self.rank], self.recv_rank[self.rank], self.recv_slot[self.rank])
+        self._barrier()                                  # every owner ready, the last step's readers done
+        _sep.sep_ep_dispatch(self.handle, x, self.rank, self.delta, self.pools, rows, self.error,
+                             recv_token=self.recv_token, recv_rank=self.recv_rank, recv_slot=self.recv_slot)
+        self._barrier()                                  # every row has landed
+        P = rows[self.rank]
+        return (self.pools[self.rank][:P], self.recv_token[self.rank][:P], self.recv_rank[self.rank][:P],
+                self.recv_slot[self.rank][:P])
+
+    def expert_output(self) -> torch.Tensor:
+        """This owner's y buffer [P_o, H], to be filled with its experts' outputs
+        (row r of y is the output for row r of the received pool)."""
+        return self.ys[self.rank][: self.rows[self.rank]]
+
+    def combine(self, topk_weight: torch.Tensor, out: torch.Tensor, y_is_pool: bool = False) -> None:
+        """Step 6: out[t] = bf16(sum_j w[t, j] * y_owner[row(t, j)]).  With
+        y_is_pool the received rows themselves are the outputs (identity experts)."""
+        self._barrier()                                  # every owner's outputs are written
+        ys = self.pools if y_is_pool else self.ys
+        _sep.sep_ep_combine(self.handle, ys, self.rows, self.delta, topk_weight, out, self.error)
+        self._barrier()                                  # before the next step reuses the buffers
+        if int(self.error.item()) != 0:
+            raise RuntimeError("a row fell outside its owner's pool")
+
+    def close(self) -> None:
+        self._barrier()
+        for r, bufs in enumerate(self.buffers):
+            if r != self.rank:
+                for b in bufs:
+                    b.close()
+        self._barrier()                                  # every peer has unmapped this rank's buffers
+        for b in self.buffers[self.rank]:
+            b.close()
+        _sep.sep_handle_free(self.handle)

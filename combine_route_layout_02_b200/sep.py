@@ -88,6 +88,9 @@ _SIGNATURES = [
     ("sep_ep_dispatch", _i32, [_P, _u32, _P, _i64, _i32, _P, _P, _P, _P, _P, _P, _P, _P]),
     ("sep_ep_mark_padding", _i32, [_i32, _i32, _P, _P, _i64, _P, _P, _P, _P]),
     ("sep_ep_combine", _i32, [_P, _u32, _P, _P, _i64, _P, _P, _P, _P, _P]),
+    ("sep_ep_buffer_alloc", _i32, [_i64, ctypes.POINTER(_P), _P]),
+    ("sep_ep_buffer_open", _i32, [_P, ctypes.POINTER(_P)]),
+    ("sep_ep_buffer_close", _i32, [_P, _i32]),
 ]
 
 
@@ -312,6 +315,51 @@ def sep_ep_combine(handle: Handle, y_pools, pool_rows, delta: torch.Tensor, topk
     epoch = handle.epoch if layout_epoch is None else layout_epoch
     _check(_lib.sep_ep_combine(handle.ptr, epoch, _ptr_array(y_pools), rows, out.shape[1], _ptr(delta),
                                _ptr(topk_weight), _ptr(out), _ptr(error), _stream(stream)), "sep_ep_combine")
+
+
+IPC_HANDLE_BYTES = 64
+
+
+class SharedBuffer:
+    """A device buffer shared between the processes of a group (CUDA IPC): either
+    allocated here (``opened`` False) or mapped from another process's handle."""
+
+    def __init__(self, ptr: int, nbytes: int, handle: bytes, opened: bool):
+        self.ptr, self.nbytes, self.handle, self.opened = ptr, nbytes, handle, opened
+
+    def tensor(self, shape, dtype: torch.dtype) -> torch.Tensor:
+        """A torch view of the buffer (no copy)."""
+        typestr = {torch.bfloat16: "<V2", torch.int32: "<i4", torch.float32: "<f4", torch.uint8: "|u1"}[dtype]
+        n = 1
+        for d in shape:
+            n *= d
+        if n * torch.empty((), dtype=dtype).element_size() > self.nbytes:
+            raise ValueError("view larger than the buffer")
+        if dtype == torch.bfloat16:          # torch has no bf16 typestr: view int16 storage as bf16
+            t = torch.as_tensor(_DeviceArray(self.ptr, shape, "<i2"), device="cuda")
+            return t.view(torch.bfloat16)
+        return torch.as_tensor(_DeviceArray(self.ptr, shape, typestr), device="cuda")
+
+    def close(self) -> None:
+        if self.ptr:
+            _check(_lib.sep_ep_buffer_close(ctypes.c_void_p(self.ptr), 1 if self.opened else 0), "sep_ep_buffer_close")
+            self.ptr = 0
+
+
+def sep_ep_buffer_alloc(nbytes: int) -> SharedBuffer:
+    ptr = ctypes.c_void_p()
+    hd = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    _check(_lib.sep_ep_buffer_alloc(int(nbytes), ctypes.byref(ptr), hd), "sep_ep_buffer_alloc")
+    return SharedBuffer(ptr.value, int(nbytes), hd.raw, False)
+
+
+def sep_ep_buffer_open(handle: bytes, nbytes: int) -> SharedBuffer:
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise ValueError("an IPC handle has 64 bytes")
+    ptr = ctypes.c_void_p()
+    _check(_lib.sep_ep_buffer_open(ctypes.create_string_buffer(handle, IPC_HANDLE_BYTES), ctypes.byref(ptr)),
+           "sep_ep_buffer_open")
+    return SharedBuffer(ptr.value, int(nbytes), handle, True)
 
 
 def sep_combine_scatter(handle: Handle, y_pool: torch.Tensor, topk_weight: torch.Tensor, out: torch.Tensor,

@@ -512,6 +512,26 @@ SEP_API sep_status sep_ep_combine(const sep_handle *handle, uint32_t layout_epoc
                                   const int64_t *pool_rows, int64_t hidden, const int32_t *delta,
                                   const float *topk_weight, void *out, uint32_t *error, void *stream);
 
+/*
+ * Buffers shared across the processes of an expert-parallel group (CUDA IPC;
+ * plain device memory mapped into the peers, no multicast object).  No
+ * counterpart on the pages: they are the plumbing a multi-process group needs
+ * to hand each other pool pointers.
+ *
+ * sep_ep_buffer_alloc   cudaMalloc of `bytes` on the current device; writes the
+ *                       SEP_IPC_HANDLE_BYTES-byte handle other processes open.
+ * sep_ep_buffer_open    maps a handle from another process (on this device or a
+ *                       peer) and returns its device pointer.  A process cannot
+ *                       open its own handle: it uses its own pointer.
+ * sep_ep_buffer_close   opened = 1: unmaps a buffer from sep_ep_buffer_open;
+ *                       opened = 0: frees one from sep_ep_buffer_alloc (after
+ *                       every peer has closed it).  Both synchronise the device.
+ */
+#define SEP_IPC_HANDLE_BYTES 64
+SEP_API sep_status sep_ep_buffer_alloc(int64_t bytes, void **ptr, void *ipc_handle);
+SEP_API sep_status sep_ep_buffer_open(const void *ipc_handle, void **ptr);
+SEP_API sep_status sep_ep_buffer_close(void *ptr, int opened);
+
 /* Frees the handle.  Its device memory is released stream-ordered on the
  * stream of the last call that used it; the caller must have ordered every
  * other stream that used the handle before that point.  NULL is a no-op; a

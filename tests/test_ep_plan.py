@@ -105,7 +105,7 @@ def _worker(rank, world, port, out, E, B, k, Ts):
 def test_two_ranks_exchange_counts_and_agree_on_the_plan():
     world, E, B, k, Ts = 2, 16, 16, 4, [61, 38]
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_worker, args=(world, port, out, E, B, k, Ts), nprocs=world, join=True)
         res = dict(out)
