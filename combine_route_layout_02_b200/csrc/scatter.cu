@@ -95,10 +95,11 @@ cudaError_t launch_combine_scatter(ScatterParams p, cudaStream_t s, int num_sms)
 {
     if (p.rows_cap == 0)
         return cudaSuccess;
-    // a pool row splits into 128-vector steps, one work item each
+    // a pool row splits into steps of 32 * kUnroll vectors, one work item each
     int64_t steps = 1;
-    split_rows(p.rows_cap, ((p.H / 8) + 127) / 128, (int64_t)num_sms * 32, 1 << 20, &p.segs, &steps);
-    p.seg_len = (int)(steps * 128);
+    split_rows(p.rows_cap, ((p.H / 8) + 32 * kUnroll - 1) / (32 * kUnroll), (int64_t)num_sms * 32, 1 << 20, &p.segs,
+               &steps);
+    p.seg_len = (int)(steps * 32 * kUnroll);
     const int64_t items = p.rows_cap * p.segs;
     if (items == 0)
         return cudaSuccess;
