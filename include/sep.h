@@ -23,7 +23,9 @@
  * pool_recv_token < 0 and are never read or written.
  *
  * Logical owners ("ranks") are contiguous expert ranges: owner r holds experts
- * [r*E/R, (r+1)*E/R).  Everything runs on one GPU; there is no communication.
+ * [r*E/R, (r+1)*E/R).  The core calls run on one GPU with no communication;
+ * the sep_ep_* calls extend dispatch and combine to owners that are separate
+ * processes (one per GPU), whose pools are reached through peer pointers.
  *
  * Errors: every entry point returns a sep_status; SEP_OK means the work was
  * enqueued.  On any other status nothing was enqueued (except SEP_ERR_CUDA,
