@@ -504,6 +504,7 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
         torch.cuda.synchronize()
         barrier(world)
         e2e_local = mean([a.elapsed_time(b) for a, b in e2e_ev])
+        copies_local = 0.0                               # not measured one step at a time
         e2e_mode = "one step at a time (the consumer occupies a side stream)"
     else:
         nb = 2
@@ -520,7 +521,7 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
         ev_cmp = [torch.cuda.Event() for _ in range(nb)]
         ev_out = [torch.cuda.Event() for _ in range(nb)]
 
-        def e2e_step(i):
+        def e2e_step(i, kernels=True):
             b = i % nb
             S, hb = sets[b], handles[b]
             s_in.wait_event(ev_cmp[b])                   # step i-nb has finished with these inputs
@@ -531,10 +532,11 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
             ev_in[b].record(s_in)
             s_cmp.wait_event(ev_in[b])
             s_cmp.wait_event(ev_out[b])                  # step i-nb's output has been downloaded
-            sep.sep_layout(S["idx"], w.E, w.R, w.B, handle=hb, stream=s_cmp)
-            sep.sep_dispatch(hb, S["x"], S["recv"], payload=w.payload, scale=w.scale, recv_scales=S["scales"],
-                             stream=s_cmp)
-            sep.sep_combine(hb, S["y"], S["wt"], S["out"], stream=s_cmp)
+            if kernels:
+                sep.sep_layout(S["idx"], w.E, w.R, w.B, handle=hb, stream=s_cmp)
+                sep.sep_dispatch(hb, S["x"], S["recv"], payload=w.payload, scale=w.scale,
+                                 recv_scales=S["scales"], stream=s_cmp)
+                sep.sep_combine(hb, S["y"], S["wt"], S["out"], stream=s_cmp)
             ev_cmp[b].record(s_cmp)
             s_out.wait_event(ev_cmp[b])
             with torch.cuda.stream(s_out):
@@ -553,10 +555,20 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
         torch.cuda.synchronize()
         barrier(world)
         e2e_local = t0.elapsed_time(t1) / args.e2e_steps
+        # the same pipeline with the kernels left out: the host-link floor of a step
+        for i in range(4):
+            e2e_step(i, kernels=False)
+        torch.cuda.synchronize()
+        t0.record(s_in)
+        for i in range(args.e2e_steps):
+            e2e_step(i, kernels=False)
+        t1.record(s_out)
+        torch.cuda.synchronize()
+        copies_local = t0.elapsed_time(t1) / args.e2e_steps
         for hb in handles[1:]:
             sep.sep_handle_free(hb)
         e2e_mode = "pipelined: two buffer sets, uploads / kernels / downloads on three streams"
-    (e2e_ms,) = reduce_max([e2e_local], world, dev)
+    (e2e_ms, copies_ms) = reduce_max([e2e_local, copies_local], world, dev)
     peaks = load_peaks()
     extras = set() if args.no_extras else set(args.extras.split(","))
 
@@ -625,6 +637,7 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
                      "traffic": traffic},
         "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "mode": e2e_mode,
+                "copies_only_ms_per_step": copies_ms or None,
                 "l2": "not flushed: every step uploads its inputs and the step's working set cycles the L2"},
         "gpu_launches": launches,
         **({"graph_replay": {"ms_per_step": graph_ms, "value": world * T / (graph_ms * 1e-3),
