@@ -13,6 +13,13 @@ seeded bf16 pool).  Inputs are resident in HBM before timing; the L2 is flushed
 (a 2 x L2 write, then read back so no dirty line of the flush is written back
 inside the step) before every timed step, outside the events.
 
+After the timed steps, on the same data: the phase split (its own loop, with
+events between the kernels), a loop without the L2 flush, the step replayed
+from a CUDA graph, the end-to-end pipeline through the C ABI with host copies,
+the CPU oracle (one core and every core), and the measurements chosen with
+--extras (borrowed receive, backward pair, combine gate, scatter combine,
+expert parallelism emulated on one GPU).
+
 Multi-GPU (torchrun): every rank runs the same workload on its own token shard
 (its own seed), with no collective on the data path (weak scaling); the step
 time is the maximum over ranks.  Rank 0 prints one JSON line.
@@ -22,7 +29,6 @@ from __future__ import annotations
 import argparse
 import hashlib
 import re
-import glob
 import json
 import os
 import statistics

@@ -115,3 +115,25 @@ def test_two_ranks_exchange_counts_and_agree_on_the_plan():
         _check_rank(r, idx, plan["delta"], Ts, lay_all, E, world, B)
         _check_owner(r, plan, lay_all, E, world, B)
         np.testing.assert_array_equal(plan["owner_rows"], res[0][1]["owner_rows"])   # every rank sees the same sizes
+
+
+def test_group_pool_capacity_holds_the_worst_routing():
+    """EPGroup sizes every owner's pool for the worst case: every assignment of
+    every rank on one owner, spread so each of its experts wastes BLOCK_M - 1
+    padding rows.  The plan's owner sizes must never exceed it."""
+    from combine_route_layout_02_b200.ep import _pool_rows_cap
+    rng = np.random.default_rng(11)
+    for _ in range(200):
+        R = int(rng.choice([1, 2, 4, 8]))
+        El = int(rng.integers(1, 9))
+        E, B, k = R * El, int(rng.choice([1, 16, 128])), int(rng.integers(1, 9))
+        max_tokens = int(rng.integers(1, 200))
+        cap = _pool_rows_cap(R, max_tokens, k, El, B)
+        counts = np.zeros((R, E), np.int32)
+        for r in range(R):                               # all of rank r's assignments, on owner 0's experts
+            n = max_tokens * k
+            split = rng.multinomial(n, np.ones(El) / El)
+            counts[r, :El] = split
+        plan = sep.sep_ep_plan(counts, 0, B)
+        assert plan["owner_rows"].max() <= cap
+        assert cap % B == 0
