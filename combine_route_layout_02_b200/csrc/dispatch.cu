@@ -115,136 +115,6 @@ __global__ void __launch_bounds__(kWarps * 32) dispatch_bf16_kernel(DispatchPara
     }
 }
 
-// ---------------------------------------------------------------- bulk copy
-//
-// bf16 dispatch through the TMA unit (non-streaming only): a CTA is one warp
-// whose lane 0 bulk-loads x[t] into one stage of a shared-memory ring
-// (cp.async.bulk global->shared, completion on an mbarrier), then issues k
-// bulk stores from that stage to the token's pool rows (cp.async.bulk
-// shared->global, one bulk group per token).  A stage is refilled once the
-// stores of the token before have finished reading it.  Every wait is bounded;
-// a wait that gives up records the layout epoch in the handle's timeout word
-// (reported by sep_handle_sync), drains the copies it issued and returns.
-constexpr bool kBulkDispatch = false;
-constexpr int kBulkStages = 4;
-constexpr int kBulkMaxSmem = 96 * 1024;
-
-__device__ __forceinline__ uint32_t smem_u32(const void *ptr)
-{
-    return static_cast<uint32_t>(__cvta_generic_to_shared(ptr));
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ uint64_t now_ns()
-{
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// true once the barrier's phase `parity` completed; false after ~limit_ns
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint64_t limit_ns)
-{
-    const uint64_t t0 = now_ns();
-    for (uint32_t it = 0; it < (1u << 24); ++it) {
-        if (mbar_try_wait(bar, parity))
-            return true;
-        if (now_ns() - t0 > limit_ns)
-            return false;
-    }
-    return false;
-}
-
-__device__ __forceinline__ void bulk_load(uint32_t dst_smem, const void *src, uint32_t bytes, uint32_t bar)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(dst_smem), "l"(src), "r"(bytes), "r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void bulk_store(void *dst, uint32_t src_smem, uint32_t bytes)
-{
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
-                 ::"l"(dst), "r"(src_smem), "r"(bytes) : "memory");
-}
-
-__global__ void __launch_bounds__(32) dispatch_bf16_bulk_kernel(DispatchParams p)
-{
-    extern __shared__ __align__(128) uint8_t stage_mem[];
-    __shared__ __align__(8) uint64_t bars[kBulkStages];
-    grid_dependency_wait();
-    allow_dependents();
-    const int lane = threadIdx.x;
-    const bool leader = lane == 0;                       // lane 0 drives the copies
-    const uint32_t row_bytes = (uint32_t)p.H * 2u;
-    const int64_t n = p.T > blockIdx.x ? (p.T - 1 - blockIdx.x) / gridDim.x + 1 : 0;   // this CTA's tokens
-    const uint8_t *x = static_cast<const uint8_t *>(p.x);
-    uint8_t *recv = static_cast<uint8_t *>(p.recv);
-    const uint32_t base = smem_u32(stage_mem);
-    auto token = [&](int64_t i) { return (int64_t)blockIdx.x + i * gridDim.x; };
-
-    int64_t loaded = n < kBulkStages ? n : kBulkStages;  // loads issued so far
-    if (leader) {
-        for (int s = 0; s < kBulkStages; ++s)
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[s])));
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        for (int64_t i = 0; i < loaded; ++i)
-            bulk_load(base + (uint32_t)i * row_bytes, x + token(i) * row_bytes, row_bytes, smem_u32(&bars[i]));
-    }
-    int64_t waited = 0;                                  // loads whose completion was observed
-    bool ok = true;
-    for (int64_t i = 0; i < n; ++i) {
-        const int s = (int)(i % kBulkStages);
-        const int64_t t = token(i);
-        const int my_row = lane < p.k ? __ldg(p.src_pool_row + t * p.k + lane) : -1;
-        int got = 1;
-        if (leader)
-            got = mbar_wait_bounded(smem_u32(&bars[s]), (uint32_t)((i / kBulkStages) & 1), 100000000ull);
-        if (!__shfl_sync(kFullMask, got, 0)) {
-            ok = false;
-            break;
-        }
-        waited = i + 1;
-        for (int j = 0; j < p.k; ++j) {
-            const int row = __shfl_sync(kFullMask, my_row, j);
-            if (leader && row >= 0)
-                bulk_store(recv + (int64_t)row * row_bytes, base + (uint32_t)s * row_bytes, row_bytes);
-        }
-        if (leader) {
-            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-            // refill the previous stage once the stores of token i-1 have read it
-            if (i >= 1 && loaded < n) {
-                asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-                const int ps = (int)((i - 1) % kBulkStages);
-                bulk_load(base + (uint32_t)ps * row_bytes, x + token(loaded) * row_bytes, row_bytes,
-                          smem_u32(&bars[ps]));
-            }
-        }
-        if (i >= 1 && loaded < n)
-            ++loaded;                                    // every lane keeps the same count
-    }
-    if (leader) {
-        if (!ok) {
-            atomicMax(p.error_epoch, p.epoch);
-            // let the loads already issued land before the CTA's shared memory goes away
-            for (int64_t i = waited; i < loaded; ++i)
-                mbar_wait_bounded(smem_u32(&bars[i % kBulkStages]), (uint32_t)((i / kBulkStages) & 1),
-                                  100000000ull);
-        }
-        asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-    }
-}
-
 // Smallest E with 448 * 2^E >= amax (0 for amax == 0), clamped to [-127, 127].
 // amax = m * 2^x with m in [1, 2): 448 = 1.75 * 2^8, so E = x - 8 when
 // m <= 1.75 (mantissa field <= 0x600000) and x - 7 otherwise.  Every subnormal
@@ -410,25 +280,6 @@ cudaError_t launch_dispatch(DispatchParams p, int payload, cudaStream_t s, int n
     p.seg_len = (int)(fp8 ? steps : steps * kStepVecs);
     const int64_t items = p.T * p.segs;
     if (payload == SEP_PAYLOAD_BF16) {
-        const int64_t smem = (int64_t)kBulkStages * p.H * 2;
-        if (kBulkDispatch && p.tile_ready == nullptr && smem <= kBulkMaxSmem) {
-            static int attr_set = 0;
-            if (!attr_set) {
-                cudaError_t e = cudaFuncSetAttribute(dispatch_bf16_bulk_kernel,
-                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kBulkMaxSmem);
-                if (e != cudaSuccess)
-                    return e;
-                attr_set = 1;
-            }
-            int per_sm = 0;
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dispatch_bf16_bulk_kernel, 32, (size_t)smem) !=
-                    cudaSuccess || per_sm < 1)
-                per_sm = 1;
-            const int64_t want = p.T;
-            const int64_t cap = (int64_t)num_sms * per_sm;
-            return launch_kernel(dispatch_bf16_bulk_kernel, dim3((int)(want < cap ? want : cap)), dim3(32),
-                                 (size_t)smem, s, p);
-        }
         if (p.tile_ready != nullptr)
             return launch_kernel(dispatch_bf16_kernel<4, true>, dim3(blocks_for(0, items, num_sms)),
                                  dim3(kWarps * 32), 0, s, p);
@@ -441,7 +292,6 @@ cudaError_t launch_dispatch(DispatchParams p, int payload, cudaStream_t s, int n
 cudaError_t preload_dispatch_kernels()
 {
     const void *k[] = {
-        reinterpret_cast<const void *>(dispatch_bf16_bulk_kernel),
         reinterpret_cast<const void *>(dispatch_bf16_kernel<4, false>),
         reinterpret_cast<const void *>(dispatch_bf16_kernel<4, true>),
         reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_F32, false>),
