@@ -95,3 +95,32 @@ def test_noalloc_rejects_sizes_beyond_its_limits():
     la.max_pool_rows = 10
     small = lib.sep_layout_noalloc(ctypes.c_void_p(16), 4, 100, 2, 8, 2, 16, ctypes.byref(la), None)
     assert small == sep.SEP_ERR_CAPACITY
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("T,k,E,R,B,masked", [(0, 4, 8, 2, 16, 0.0), (1, 1, 1, 1, 1, 0.0), (333, 3, 12, 4, 5, 0.3),
+                                               (2048, 8, 256, 32, 64, 0.1), (9000, 6, 96, 8, 128, 0.0)])
+def test_noalloc_layout_equals_the_oracle(T, k, E, R, B, masked):
+    """Shapes up to the limits (E = 256), a ragged BLOCK_M, masked entries and an
+    empty routing, each against the oracle directly."""
+    import oracle
+    rng = np.random.default_rng(T * 7 + E)
+    idx = rng.integers(0, E, size=(T, k)).astype(np.int32)
+    idx[rng.random((T, k)) < masked] = -1
+    lay = oracle.layout(idx, E, R, B)
+    out = _outputs(T, k, E, R, B)
+    sep.sep_layout_noalloc(torch.from_numpy(idx).cuda(), E, R, B, out)
+    torch.cuda.synchronize()
+    assert out["status"].cpu().tolist() == [0, 0]
+    P, NT = lay.num_pool_rows, lay.num_tiles
+    np.testing.assert_array_equal(out["sizes"].cpu().numpy(), [P, NT])
+    np.testing.assert_array_equal(out["expert_counts"].cpu().numpy(), lay.expert_counts)
+    np.testing.assert_array_equal(out["owner_counts"].cpu().numpy(), lay.owner_counts)
+    np.testing.assert_array_equal(out["expert_pool_block_offset"].cpu().numpy(), lay.expert_pool_block_offset)
+    np.testing.assert_array_equal(out["owner_pool_row_offset"].cpu().numpy(), lay.owner_pool_row_offset)
+    np.testing.assert_array_equal(out["tile_expert"][:NT].cpu().numpy(), lay.tile_expert)
+    np.testing.assert_array_equal(out["pool_arrival_target"][:NT].cpu().numpy(), lay.pool_arrival_target)
+    if T:
+        np.testing.assert_array_equal(out["src_pool_row"].cpu().numpy(), lay.src_pool_row)
+    np.testing.assert_array_equal(out["pool_recv_token"][:P].cpu().numpy(), lay.pool_recv_token)
+    np.testing.assert_array_equal(out["pool_recv_slot"][:P].cpu().numpy(), lay.pool_recv_slot)
