@@ -20,6 +20,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
+#include "fp8_quant.cuh"
 #include "sep_internal.cuh"
 
 namespace sep {
@@ -115,38 +116,6 @@ __global__ void __launch_bounds__(kWarps * 32) dispatch_bf16_kernel(DispatchPara
     }
 }
 
-// Smallest E with 448 * 2^E >= amax (0 for amax == 0), clamped to [-127, 127].
-// amax = m * 2^x with m in [1, 2): 448 = 1.75 * 2^8, so E = x - 8 when
-// m <= 1.75 (mantissa field <= 0x600000) and x - 7 otherwise.  Every subnormal
-// amax is below 448 * 2^-134 and clamps to -127.
-__device__ __forceinline__ int ue8m0_exponent(float amax)
-{
-    const uint32_t u = __float_as_uint(amax);
-    if (u == 0u)
-        return 0;
-    const int ex = (int)(u >> 23);
-    if (ex == 0)
-        return -127;
-    const int e = ex - 127 - 8 + ((u & 0x7fffffu) > 0x600000u ? 1 : 0);
-    return e < -127 ? -127 : (e > 127 ? 127 : e);
-}
-
-// 2^e as fp32 for e in [-127, 127] (2^-127 is subnormal).
-__device__ __forceinline__ float exp2_int(int e)
-{
-    return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00400000u);
-}
-
-__device__ __forceinline__ void bf16x8_to_f32(const uint4 &v, float *f)
-{
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        f[2 * i] = __uint_as_float(w[i] << 16);
-        f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-    }
-}
-
 // fp8: a work item is (token, segment of seg_len 512-channel iterations).
 template <int SCALE, bool PUBLISH>
 __global__ void __launch_bounds__(kWarps * 32) dispatch_fp8_kernel(DispatchParams p)
@@ -179,38 +148,9 @@ __global__ void __launch_bounds__(kWarps * 32) dispatch_fp8_kernel(DispatchParam
                 for (int q = 0; q < 16; ++q)
                     f[q] = 0.f;
             }
-            float amax = 0.f;
-#pragma unroll
-            for (int q = 0; q < 16; ++q)
-                amax = fmaxf(amax, fabsf(f[q]));
-            amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 1));
-            amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 2));
-            amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 4));
-
-            float scale_f = 1.f, inv = 1.f;
-            int expo = 0;
-            if (SCALE == SEP_SCALE_F32) {
-                scale_f = amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
-            } else {
-                expo = ue8m0_exponent(amax);
-                scale_f = exp2_int(expo);
-                inv = exp2_int(-expo);                    // exact: x * 2^-E == x / 2^E
-            }
-            uint32_t packed[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                float a[4];
-#pragma unroll
-                for (int r = 0; r < 4; ++r)
-                    a[r] = SCALE == SEP_SCALE_F32 ? __fdiv_rn(f[4 * q + r], scale_f)
-                                                  : __fmul_rn(f[4 * q + r], inv);
-                const __nv_fp8x2_storage_t lo =
-                    __nv_cvt_float2_to_fp8x2(make_float2(a[0], a[1]), __NV_SATFINITE, __NV_E4M3);
-                const __nv_fp8x2_storage_t hi =
-                    __nv_cvt_float2_to_fp8x2(make_float2(a[2], a[3]), __NV_SATFINITE, __NV_E4M3);
-                packed[q] = (uint32_t)lo | ((uint32_t)hi << 16);
-            }
-            const uint4 codes = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            float scale_f;
+            int expo;
+            const uint4 codes = quantize_lane16<SCALE>(f, scale_f, expo);
             const int g = c0 / 128;
             for (int j = 0; j < p.k; ++j) {
                 const int row = __shfl_sync(kFullMask, my_row, j);

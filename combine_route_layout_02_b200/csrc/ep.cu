@@ -27,6 +27,7 @@
 // way (peer loads) and reduces them exactly as the single-GPU combine does.
 #include <cuda_bf16.h>
 
+#include "fp8_quant.cuh"
 #include "sep_internal.cuh"
 
 namespace sep {
@@ -108,6 +109,78 @@ __global__ void __launch_bounds__(kWarps * 32) ep_dispatch_kernel(EpDispatchPara
                     const int v = v0 + u * 32 + lane;
                     if (v < v_end)
                         dst[v] = buf[u];
+                }
+            }
+        }
+    }
+}
+
+// FP8 dispatch into the owners' pools: a work item is (token, segment of
+// 512-channel iterations); each token is quantised once (the single-GPU
+// kernel's arithmetic) and its codes and scales stored to the k owners' rows.
+template <int SCALE>
+__global__ void __launch_bounds__(kWarps * 32) ep_dispatch_fp8_kernel(EpDispatchParams p)
+{
+    grid_dependency_wait();
+    allow_dependents();
+    const int lane = threadIdx.x & 31;
+    const int H = p.H;
+    const int G = H / 128;
+    const int iters = (H + 511) / 512;
+    const int64_t items = p.T * p.segs;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t it = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items; it += nwarps) {
+        const int64_t t = it / p.segs;
+        const int s = (int)(it - t * p.segs);
+        const int i_begin = s * p.seg_len;
+        const int i_end = min(iters, i_begin + p.seg_len);
+        int my_owner = 0;
+        const int64_t my_row = lane < p.k ? owner_row(p, t * p.k + lane, &my_owner) : -1;
+        uint8_t *my_codes = my_row >= 0 ? static_cast<uint8_t *>(p.pools[my_owner]) + my_row * H : nullptr;
+        uint8_t *my_scales = my_row >= 0 ? static_cast<uint8_t *>(p.scales[my_owner]) +
+                                               my_row * G * (SCALE == SEP_SCALE_UE8M0 ? 1 : 4)
+                                         : nullptr;
+        if (s == 0 && my_row >= 0) {                     // the owner's receive map, once per assignment
+            if (p.recv_token[my_owner])
+                p.recv_token[my_owner][my_row] = (int32_t)t;
+            if (p.recv_rank[my_owner])
+                p.recv_rank[my_owner][my_row] = p.rank;
+            if (p.recv_slot[my_owner])
+                p.recv_slot[my_owner][my_row] = lane;
+        }
+        const __nv_bfloat16 *xrow = static_cast<const __nv_bfloat16 *>(p.x) + t * H;
+        for (int i = i_begin; i < i_end; ++i) {
+            const int c0 = i * 512 + lane * 16;          // H % 128 == 0: whole groups are in or out
+            const bool active = c0 < H;
+            float f[16];
+            if (active) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(xrow + c0);
+                bf16x8_to_f32(ld_stream(src), f);
+                bf16x8_to_f32(ld_stream(src + 1), f + 8);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 16; ++q)
+                    f[q] = 0.f;
+            }
+            float scale_f;
+            int expo;
+            const uint4 codes = quantize_lane16<SCALE>(f, scale_f, expo);
+            const int g = c0 / 128;
+            for (int j = 0; j < p.k; ++j) {
+                uint8_t *dst = reinterpret_cast<uint8_t *>(
+                    __shfl_sync(kFullMask, reinterpret_cast<unsigned long long>(my_codes), j));
+                uint8_t *sc = reinterpret_cast<uint8_t *>(
+                    __shfl_sync(kFullMask, reinterpret_cast<unsigned long long>(my_scales), j));
+                if (dst == nullptr)
+                    continue;                            // warp-uniform
+                if (active) {
+                    *reinterpret_cast<uint4 *>(dst + c0) = codes;
+                    if ((lane & 7) == 0) {
+                        if (SCALE == SEP_SCALE_UE8M0)
+                            sc[g] = (uint8_t)(expo + 127);
+                        else
+                            reinterpret_cast<float *>(sc)[g] = scale_f;
+                    }
                 }
             }
         }
@@ -223,6 +296,24 @@ cudaError_t launch_ep_dispatch(EpDispatchParams p, cudaStream_t s, int num_sms)
     return launch_kernel(ep_dispatch_kernel, dim3((int)((items + kWarps - 1) / kWarps)), dim3(kWarps * 32), 0, s, p);
 }
 
+cudaError_t launch_ep_dispatch_fp8(EpDispatchParams p, cudaStream_t s, int num_sms)
+{
+    if (p.T == 0)
+        return cudaSuccess;
+    int64_t steps = 1;                                   // 512-channel steps, up to 7 warps a row
+    split_rows(p.T, (p.H + 511) / 512, (int64_t)num_sms * 32, 7, &p.segs, &steps);
+    p.seg_len = (int)steps;
+    const dim3 grid((int)((p.T * p.segs + kWarps - 1) / kWarps)), block(kWarps * 32);
+    switch (p.scale) {
+    case SEP_SCALE_F32:
+        return launch_kernel(ep_dispatch_fp8_kernel<SEP_SCALE_F32>, grid, block, 0, s, p);
+    case SEP_SCALE_UE8M0:
+        return launch_kernel(ep_dispatch_fp8_kernel<SEP_SCALE_UE8M0>, grid, block, 0, s, p);
+    default:
+        return launch_kernel(ep_dispatch_fp8_kernel<SEP_SCALE_F32_POW2>, grid, block, 0, s, p);
+    }
+}
+
 cudaError_t launch_ep_mark_padding(const EpPaddingParams &p, cudaStream_t s, int num_sms)
 {
     if (p.pool_rows == 0)
@@ -252,6 +343,12 @@ cudaError_t preload_ep_kernels()
         e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(ep_mark_padding_kernel));
     if (e == cudaSuccess)
         e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(ep_combine_kernel));
+    if (e == cudaSuccess)
+        e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(ep_dispatch_fp8_kernel<SEP_SCALE_F32>));
+    if (e == cudaSuccess)
+        e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(ep_dispatch_fp8_kernel<SEP_SCALE_UE8M0>));
+    if (e == cudaSuccess)
+        e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(ep_dispatch_fp8_kernel<SEP_SCALE_F32_POW2>));
     return e;
 }
 

@@ -1103,6 +1103,66 @@ sep_status sep_ep_dispatch(const sep_handle *h, uint32_t layout_epoch, const voi
     return e == cudaSuccess ? SEP_OK : cuda_fail(e, "expert-parallel dispatch launch");
 }
 
+sep_status sep_ep_dispatch_fp8(const sep_handle *h, uint32_t layout_epoch, const void *x, int64_t hidden, int rank,
+                               int scale, const int32_t *delta, void *const *pools, void *const *scales,
+                               const int64_t *pool_rows, int32_t *const *recv_token, int32_t *const *recv_rank,
+                               int32_t *const *recv_slot, uint32_t *error, void *stream)
+{
+    EpCommon c;
+    sep_status st = ep_common(h, layout_epoch, hidden, delta, pool_rows, error, &c);
+    if (st != SEP_OK)
+        return st;
+    if (rank < 0 || rank >= h->R)
+        return fail(SEP_ERR_INVALID_ARG, "rank %d outside 0..%d", rank, h->R - 1);
+    if (hidden % 128 != 0)
+        return fail(SEP_ERR_INVALID_ARG, "the FP8 payload needs hidden to be a multiple of 128 (got %lld)",
+                    (long long)hidden);
+    if (scale != SEP_SCALE_F32 && scale != SEP_SCALE_UE8M0 && scale != SEP_SCALE_F32_POW2)
+        return fail(SEP_ERR_INVALID_ARG, "the FP8 payload needs an fp32, UE8M0 or power-of-two fp32 scale");
+    if (pools == nullptr || scales == nullptr || (h->T > 0 && x == nullptr))
+        return fail(SEP_ERR_INVALID_ARG, "NULL pools, scales or x");
+    if (!aligned16(x))
+        return fail(SEP_ERR_INVALID_ARG, "x must be 16-byte aligned");
+    sep::EpDispatchParams p{};
+    p.T = c.T;
+    p.H = c.H;
+    p.k = c.k;
+    p.B = c.B;
+    p.E_loc = c.E_loc;
+    p.R = c.R;
+    p.src_pool_row = c.src_pool_row;
+    p.tile_expert = c.tile_expert;
+    p.delta = c.delta;
+    p.error = c.error;
+    memcpy(p.pool_rows, c.pool_rows, sizeof(p.pool_rows));
+    const uintptr_t scale_align = scale == SEP_SCALE_UE8M0 ? 0u : 3u;
+    for (int r = 0; r < h->R; ++r) {
+        if ((pool_rows[r] > 0 && (pools[r] == nullptr || scales[r] == nullptr)) || !aligned16(pools[r]) ||
+            (reinterpret_cast<uintptr_t>(scales[r]) & scale_align) != 0)
+            return fail(SEP_ERR_INVALID_ARG, "pools[%d] / scales[%d] must be non-NULL (if it has rows), "
+                                             "16-byte and scale-size aligned", r, r);
+        p.pools[r] = pools[r];
+        p.scales[r] = scales[r];
+        p.recv_token[r] = recv_token ? recv_token[r] : nullptr;
+        p.recv_rank[r] = recv_rank ? recv_rank[r] : nullptr;
+        p.recv_slot[r] = recv_slot ? recv_slot[r] : nullptr;
+        if (((reinterpret_cast<uintptr_t>(p.recv_token[r]) | reinterpret_cast<uintptr_t>(p.recv_rank[r]) |
+              reinterpret_cast<uintptr_t>(p.recv_slot[r])) & 3u) != 0)
+            return fail(SEP_ERR_INVALID_ARG, "receive maps of rank %d must be 4-byte aligned", r);
+    }
+    p.x = x;
+    p.rank = rank;
+    p.scale = scale;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = wait_for_release(const_cast<sep_handle *>(h), s, false)) != SEP_OK)
+        return st;
+    if (h->T == 0)
+        return SEP_OK;
+    const_cast<sep_handle *>(h)->last_stream = s;
+    const cudaError_t e = sep::launch_ep_dispatch_fp8(p, s, sep::device_sm_count());
+    return e == cudaSuccess ? SEP_OK : cuda_fail(e, "expert-parallel FP8 dispatch launch");
+}
+
 sep_status sep_ep_mark_padding(int num_local_experts, int block_m, const int32_t *owner_block_offset,
                                const int32_t *owner_expert_counts, int64_t pool_rows, int32_t *recv_token,
                                int32_t *recv_rank, int32_t *recv_slot, void *stream)

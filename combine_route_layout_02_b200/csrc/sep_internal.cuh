@@ -170,6 +170,9 @@ struct EpDispatchParams {
     int32_t *recv_token[kEpMaxRanks];   // owners' receive maps (entries may be nullptr)
     int32_t *recv_rank[kEpMaxRanks];
     int32_t *recv_slot[kEpMaxRanks];
+    // FP8 payload (pools hold e4m3 codes): owners' scale arrays [rows][H/128]
+    int scale;                       // sep_scale
+    void *scales[kEpMaxRanks];
 };
 
 struct EpPaddingParams {
@@ -195,6 +198,7 @@ struct EpCombineParams {
 };
 
 cudaError_t launch_ep_dispatch(EpDispatchParams p, cudaStream_t s, int num_sms);
+cudaError_t launch_ep_dispatch_fp8(EpDispatchParams p, cudaStream_t s, int num_sms);
 cudaError_t launch_ep_mark_padding(const EpPaddingParams &p, cudaStream_t s, int num_sms);
 cudaError_t launch_ep_combine(EpCombineParams p, cudaStream_t s, int num_sms);
 cudaError_t preload_ep_kernels();

@@ -87,6 +87,7 @@ _SIGNATURES = [
     ("sep_ep_plan", _i32, [_P, _i32, _i32, _i32, _i32, _P, _P, _P, _P]),
     ("sep_ep_dispatch", _i32, [_P, _u32, _P, _i64, _i32, _P, _P, _P, _P, _P, _P, _P, _P]),
     ("sep_ep_mark_padding", _i32, [_i32, _i32, _P, _P, _i64, _P, _P, _P, _P]),
+    ("sep_ep_dispatch_fp8", _i32, [_P, _u32, _P, _i64, _i32, _i32, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     ("sep_ep_combine", _i32, [_P, _u32, _P, _P, _i64, _P, _P, _P, _P, _P]),
     ("sep_ep_buffer_alloc", _i32, [_i64, ctypes.POINTER(_P), _P]),
     ("sep_ep_buffer_open", _i32, [_P, ctypes.POINTER(_P)]),
@@ -296,6 +297,21 @@ def sep_ep_dispatch(handle: Handle, x: torch.Tensor, rank: int, delta: torch.Ten
     epoch = handle.epoch if layout_epoch is None else layout_epoch
     _check(_lib.sep_ep_dispatch(handle.ptr, epoch, _ptr(x), x.shape[1], rank, _ptr(delta), _ptr_array(pools), rows,
                                 maps[0], maps[1], maps[2], _ptr(error), _stream(stream)), "sep_ep_dispatch")
+
+
+def sep_ep_dispatch_fp8(handle: Handle, x: torch.Tensor, rank: int, delta: torch.Tensor, pools, scales, pool_rows,
+                        error: torch.Tensor, scale: str = "ue8m0", recv_token=None, recv_rank=None, recv_slot=None,
+                        layout_epoch: int | None = None, stream=None) -> None:
+    """FP8 rows (codes + per-128-channel scales) of this rank's tokens into the owners' pools."""
+    if x.dtype != torch.bfloat16 or delta.dtype != torch.int32:
+        raise ValueError("x must be bf16 and delta int32")
+    R = len(pools)
+    rows = (ctypes.c_int64 * R)(*[int(r) for r in pool_rows])
+    maps = [None if m is None else _ptr_array(m) for m in (recv_token, recv_rank, recv_slot)]
+    epoch = handle.epoch if layout_epoch is None else layout_epoch
+    _check(_lib.sep_ep_dispatch_fp8(handle.ptr, epoch, _ptr(x), x.shape[1], rank, SCALES[scale], _ptr(delta),
+                                    _ptr_array(pools), _ptr_array(scales), rows, maps[0], maps[1], maps[2],
+                                    _ptr(error), _stream(stream)), "sep_ep_dispatch_fp8")
 
 
 def sep_ep_mark_padding(owner_block_offset: torch.Tensor, owner_expert_counts: torch.Tensor, block_m: int,

@@ -494,6 +494,23 @@ SEP_API sep_status sep_ep_dispatch(const sep_handle *handle, uint32_t layout_epo
                                    uint32_t *error, void *stream);
 
 /*
+ * sep_ep_dispatch_fp8 — sep_ep_dispatch with the FP8 e4m3 payload: each token
+ * is quantised once per 128-channel group exactly as sep_dispatch does
+ * (scale = SEP_SCALE_F32, SEP_SCALE_UE8M0 or SEP_SCALE_F32_POW2), and its
+ * codes and scales are stored to the owners' rows.
+ *
+ *  pools    host array [R] of device e4m3 [pool_rows[o], hidden] (16-byte aligned).
+ *  scales   host array [R] of device [pool_rows[o], hidden / 128] fp32 or u8.
+ *  hidden   a multiple of 128.
+ * Other arguments and errors as sep_ep_dispatch.
+ */
+SEP_API sep_status sep_ep_dispatch_fp8(const sep_handle *handle, uint32_t layout_epoch, const void *x,
+                                       int64_t hidden, int rank, int scale, const int32_t *delta,
+                                       void *const *pools, void *const *scales, const int64_t *pool_rows,
+                                       int32_t *const *recv_token, int32_t *const *recv_rank,
+                                       int32_t *const *recv_slot, uint32_t *error, void *stream);
+
+/*
  * sep_ep_mark_padding — owner side: -1 in the receive maps (each may be NULL)
  * on the padding rows of this owner's pool, from sep_ep_plan's
  * owner_block_offset and owner_expert_counts (device copies).  Touches no

@@ -22,7 +22,7 @@ def test_library_is_built_for_sm100a_and_in_tree():
 
 def test_exports_match_header():
     declared = sep.declared_entry_points(HEADER)
-    assert len(declared) == 28
+    assert len(declared) == 29
     out = subprocess.run(["nm", "-D", "--defined-only", sep.library_path()], capture_output=True,
                          text=True, check=True).stdout
     exported = sorted(set(re.findall(r"\sT\s+(sep_\w+)$", out, flags=re.M)))

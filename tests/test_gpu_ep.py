@@ -117,3 +117,49 @@ def test_ep_rows_outside_a_short_pool_are_refused_on_the_device():
     assert err == 1
     short = max(rows[0] - B, 0)
     assert (bf16_bits(pools[0])[short:] == POISON_BF16).all()
+
+
+@pytest.mark.parametrize("scale", ["ue8m0", "f32", "f32_pow2"])
+def test_ep_fp8_dispatch_matches_the_concatenated_oracle(scale):
+    """The FP8 payload across ranks: codes and scales in every owner's pool equal
+    the single-GPU FP8 dispatch of the concatenated tokens, bit for bit."""
+    R, E, B, k, H, Ts = 4, 16, 16, 4, 384, [100, 0, 37, 211]
+    G = H // 128
+    idx = [_routing(900 + r, Ts[r], k, E, 0.2) for r in range(R)]
+    xs = [W.random_x(Ts[r], H, seed=950 + r) for r in range(R)]
+    handles = [sep.sep_layout(torch.from_numpy(idx[r]).cuda(), E, R, B, flags=sep.SEP_LAYOUT_SYNC_COUNTS)
+               for r in range(R)]
+    try:
+        counts = np.stack([h.view("expert_counts").cpu().numpy() for h in handles]).astype(np.int32)
+        plans = [sep.sep_ep_plan(counts, r, B) for r in range(R)]
+        rows = [int(v) for v in plans[0]["owner_rows"]]
+        pools = [torch.full((rows[o] + GUARD, H), 0xA5, dtype=torch.uint8, device="cuda") for o in range(R)]
+        if scale == "ue8m0":
+            scales = [torch.full((rows[o] + GUARD, G), 0xA5, dtype=torch.uint8, device="cuda") for o in range(R)]
+        else:
+            scales = [torch.full((rows[o] + GUARD, G), 0x7FC00ABC, dtype=torch.int32, device="cuda").view(torch.float32)
+                      for o in range(R)]
+        tok = [torch.full((rows[o] + GUARD,), -7, dtype=torch.int32, device="cuda") for o in range(R)]
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        for r in range(R):
+            sep.sep_ep_dispatch_fp8(handles[r], xs[r].cuda(), r, torch.from_numpy(plans[r]["delta"]).cuda(), pools,
+                                    scales, rows, err, scale=scale, recv_token=tok)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        lay = oracle.layout(np.concatenate(idx), E, R, B)
+        codes, scl = oracle.dispatch_fp8(torch.cat(xs), lay, scale)
+        off = lay.owner_pool_row_offset
+        for o in range(R):
+            seg = slice(off[o], off[o + 1])
+            valid = lay.pool_recv_token[seg] >= 0
+            got = pools[o].cpu().numpy()
+            np.testing.assert_array_equal(got[:rows[o]][valid], codes[seg][valid])
+            assert (got[:rows[o]][~valid] == 0xA5).all() and (got[rows[o]:] == 0xA5).all()
+            gs = scales[o].cpu().numpy()
+            if scale == "ue8m0":
+                np.testing.assert_array_equal(gs[:rows[o]][valid], scl[seg][valid])
+            else:
+                np.testing.assert_array_equal(gs[:rows[o]][valid].view(np.uint32), scl[seg][valid].view(np.uint32))
+    finally:
+        for h in handles:
+            sep.sep_handle_free(h)
