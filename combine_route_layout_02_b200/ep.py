@@ -14,7 +14,9 @@ o owns experts [o*E/R, (o+1)*E/R).  Each step:
 6. each rank reads its tokens' k output rows from the owners' y buffers and
    reduces them (``sep_ep_combine``); a barrier before the buffers are reused.
 
-The pools, y buffers and receive maps are allocated by the library and shared
+The dispatch may carry the bf16 rows or the FP8 e4m3 payload with its
+per-128-channel scales.  The pools, y buffers, scales and receive maps are
+allocated by the library and shared
 by CUDA IPC (plain device memory mapped into every peer; no multicast).  The
 barriers follow a device synchronisation, so no kernel ever waits on another
 process's kernel.
@@ -49,12 +51,14 @@ class EPGroup:
         self.E_loc = num_experts // self.world
         self.rows_cap = _pool_rows_cap(self.world, max_tokens, top_k, self.E_loc, block_m)
         self.cpu_collectives = dist.get_backend(group) != "nccl"
-        own = [_sep.sep_ep_buffer_alloc(self.rows_cap * hidden * 2),   # pool
+        self.G = max(hidden // 128, 1)
+        own = [_sep.sep_ep_buffer_alloc(self.rows_cap * hidden * 2),   # pool (bf16 rows, or e4m3 codes)
                _sep.sep_ep_buffer_alloc(self.rows_cap * hidden * 2),   # expert outputs y
-               _sep.sep_ep_buffer_alloc(3 * self.rows_cap * 4)]        # receive maps: token, rank, slot
+               _sep.sep_ep_buffer_alloc(3 * self.rows_cap * 4),        # receive maps: token, rank, slot
+               _sep.sep_ep_buffer_alloc(self.rows_cap * self.G * 4)]   # FP8 scales (fp32 or u8)
         handles = [None] * self.world
         dist.all_gather_object(handles, [b.handle for b in own], group=group)
-        self.buffers = []                                # [rank] -> [pool, y, maps]
+        self.buffers = []                                # [rank] -> [pool, y, maps, scales]
         for r in range(self.world):
             if r == self.rank:
                 self.buffers.append(own)
@@ -64,6 +68,9 @@ class EPGroup:
         self.pools = [bufs[0].tensor(shape, torch.bfloat16) for bufs in self.buffers]
         self.ys = [bufs[1].tensor(shape, torch.bfloat16) for bufs in self.buffers]
         maps = [bufs[2].tensor((3, self.rows_cap), torch.int32) for bufs in self.buffers]
+        self.codes = [bufs[0].tensor((self.rows_cap, hidden), torch.uint8) for bufs in self.buffers]
+        self.scales_f32 = [bufs[3].tensor((self.rows_cap, self.G), torch.float32) for bufs in self.buffers]
+        self.scales_u8 = [bufs[3].tensor((self.rows_cap, self.G), torch.uint8) for bufs in self.buffers]
         self.recv_token = [m[0] for m in maps]
         self.recv_rank = [m[1] for m in maps]
         self.recv_slot = [m[2] for m in maps]
@@ -84,9 +91,11 @@ class EPGroup:
         dist.all_gather(out, mine, group=self.group)
         return torch.stack(out).cpu().numpy()
 
-    def dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor):
-        """Steps 1-4; returns this owner's received rows [P_o, H] (a view of its
-        pool) and receive maps (token, rank, slot), each [P_o]."""
+    def dispatch(self, x: torch.Tensor, topk_idx: torch.Tensor, payload: str = "bf16", scale: str = "none"):
+        """Steps 1-4; returns this owner's received rows (a view of its pool:
+        bf16 [P_o, H], or with payload="fp8" the pair of e4m3 codes [P_o, H] as
+        bytes and scales [P_o, H/128], fp32 or u8) and receive maps (token,
+        rank, slot), each [P_o]."""
         _sep.sep_layout(topk_idx, self.E, self.world, self.B, handle=self.handle)
         plan = _sep.sep_ep_plan(self._all_counts(), self.rank, self.B)
         rows = [int(v) for v in plan["owner_rows"]]
@@ -99,11 +108,19 @@ class EPGroup:
                                  torch.from_numpy(plan["owner_expert_counts"]).cuda(), self.B, rows[self.rank],
                                  self.recv_token[self.rank], self.recv_rank[self.rank], self.recv_slot[self.rank])
         self._barrier()                                  # every owner ready, the last step's readers done
-        _sep.sep_ep_dispatch(self.handle, x, self.rank, self.delta, self.pools, rows, self.error,
-                             recv_token=self.recv_token, recv_rank=self.recv_rank, recv_slot=self.recv_slot)
-        self._barrier()                                  # every row has landed
+        maps = dict(recv_token=self.recv_token, recv_rank=self.recv_rank, recv_slot=self.recv_slot)
         P = rows[self.rank]
-        return (self.pools[self.rank][:P], self.recv_token[self.rank][:P], self.recv_rank[self.rank][:P],
+        if payload == "fp8":
+            scales = self.scales_u8 if scale == "ue8m0" else self.scales_f32
+            _sep.sep_ep_dispatch_fp8(self.handle, x, self.rank, self.delta, self.codes, scales, rows, self.error,
+                                     scale=scale, **maps)
+            self._barrier()                              # every row has landed
+            received = (self.codes[self.rank][:P], scales[self.rank][:P])
+        else:
+            _sep.sep_ep_dispatch(self.handle, x, self.rank, self.delta, self.pools, rows, self.error, **maps)
+            self._barrier()                              # every row has landed
+            received = self.pools[self.rank][:P]
+        return (received, self.recv_token[self.rank][:P], self.recv_rank[self.rank][:P],
                 self.recv_slot[self.rank][:P])
 
     def expert_output(self) -> torch.Tensor:

@@ -2,8 +2,9 @@
 
 Two processes share the one GPU (each a rank; gloo carries the counts
 all-gather and the barriers), hand each other their pools by CUDA IPC and run
-two steps: identity experts (the combine reads the received rows), then
-experts that double their input (written into the shared y buffers).  The EP
+three steps: identity experts (the combine reads the received rows),
+experts that double their input (written into the shared y buffers), and an
+FP8 dispatch (codes and UE8M0 scales into the shared pools).  The EP
 kernels never wait on another process's kernel — every barrier follows a
 device synchronisation — so two ranks on one GPU are safe.  The oracle is the
 single-GPU layout, dispatch and combine of both ranks' tokens concatenated in
@@ -65,6 +66,10 @@ def _worker(rank, world, port, out):
             y2 = torch.empty_like(y1)
             g.combine(w.cuda(), y2)
             res["out_double"] = bf16_bits(y2)
+            (codes, scales), _, _, _ = g.dispatch(x.cuda(), torch.from_numpy(idx).cuda(), payload="fp8",
+                                                  scale="ue8m0")
+            res["codes"] = codes.cpu().numpy()
+            res["scales"] = scales.cpu().numpy()
             out[rank] = res
         finally:
             g.close()
@@ -105,3 +110,9 @@ def test_two_processes_dispatch_and_combine_through_ipc_pools():
     for r in range(world):
         np.testing.assert_array_equal(res[r]["out_identity"], want1[cum[r]:cum[r + 1]])
         np.testing.assert_array_equal(res[r]["out_double"], want2[cum[r]:cum[r + 1]])
+    codes, scl = oracle.dispatch_fp8(torch.cat([i[1] for i in ins]), lay, "ue8m0")
+    for o in range(world):
+        seg = slice(off[o], off[o + 1])
+        valid = lay.pool_recv_token[seg] >= 0
+        np.testing.assert_array_equal(res[o]["codes"][valid], codes[seg][valid])
+        np.testing.assert_array_equal(res[o]["scales"][valid], scl[seg][valid])
