@@ -1,0 +1,47 @@
+"""Host-side pieces of the benchmark, on CPU: the algorithmic byte model, the
+traffic lookup keyed by the kernel sources, and the argument defaults."""
+import json
+import os
+import shutil
+
+import bench
+import workloads as W
+
+
+def test_algorithmic_bytes_of_the_fp8_workloads():
+    w = W.WORKLOADS["prefill_skew"]                       # FP8 codes + fp32 scales
+    Na, T, H = w.n_assign, w.T, w.H
+    ab = bench.algorithmic_bytes(w)
+    assert ab["dispatch"] == T * H * 2 + Na * H + Na * (H // 128) * 4 + 4 * Na
+    assert ab["combine"] == Na * H * 2 + T * H * 2 + 8 * Na
+    d = W.WORKLOADS["decode"]                             # FP8 codes + UE8M0 bytes
+    ab = bench.algorithmic_bytes(d)
+    assert ab["dispatch"] == d.T * d.H * 2 + d.n_assign * d.H + d.n_assign * (d.H // 128) + 4 * d.n_assign
+    s = W.WORKLOADS["streaming"]
+    assert bench.algorithmic_bytes(s)["consumer"] == 2 * s.n_assign * s.H * 2
+
+
+def test_traffic_is_reported_only_for_the_profiled_sources(tmp_path, monkeypatch):
+    root = tmp_path / "repo"
+    csrc = root / "combine_route_layout_02_b200" / "csrc"
+    shutil.copytree(os.path.join(bench.ROOT, "combine_route_layout_02_b200", "csrc"), csrc,
+                    ignore=shutil.ignore_patterns("*.o", "*.so"))
+    (root / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    h = bench.kernel_source_hash("dispatch")
+    table = {"train8k": {"dispatch": {"bytes_per_launch": 123.0, "source_hash": h}}}
+    (root / "profiles" / "dram_traffic.json").write_text(json.dumps(table))
+    assert bench.profiled_traffic("train8k", "dispatch") == 123.0
+    assert bench.profiled_traffic("train8k", "combine") is None
+    assert bench.profiled_traffic("decode", "dispatch") is None
+    # an unrelated file changing keeps the figure; the kernel's own file changing drops it
+    (csrc / "scatter.cu").write_text((csrc / "scatter.cu").read_text() + "\n// edit\n")
+    assert bench.profiled_traffic("train8k", "dispatch") == 123.0
+    (csrc / "dispatch.cu").write_text((csrc / "dispatch.cu").read_text() + "\n// edit\n")
+    assert bench.profiled_traffic("train8k", "dispatch") is None
+
+
+def test_argument_defaults():
+    a = bench.parse_args([])
+    assert a.extras.split(",") == ["borrowed", "backward", "gate", "scatter", "ep"]
+    assert not a.no_graph and not a.no_extras and a.gate_ctas == 0 and a.consumer_ctas == 64
