@@ -98,3 +98,20 @@ def test_no_cpu_fallback_in_the_binding():
 
 def test_launch_counter_starts_without_gpu_work():
     assert sep.sep_launch_count() >= 0
+
+
+def test_expert_parallel_calls_reject_bad_arguments_before_any_cuda_call():
+    lib = sep.library()
+    assert lib.sep_ep_dispatch(None, 0, None, 8, 0, None, None, None, None, None, None, None, None) == \
+        sep.SEP_ERR_INVALID_ARG
+    assert lib.sep_ep_dispatch_fp8(None, 0, None, 128, 0, 2, None, None, None, None, None, None, None, None,
+                                   None) == sep.SEP_ERR_INVALID_ARG
+    assert lib.sep_ep_combine(None, 0, None, None, 8, None, None, None, None, None) == sep.SEP_ERR_INVALID_ARG
+    assert lib.sep_ep_mark_padding(0, 16, None, None, 0, None, None, None, None) == sep.SEP_ERR_INVALID_ARG
+    assert lib.sep_ep_mark_padding(4, 0, None, None, 0, None, None, None, None) == sep.SEP_ERR_INVALID_ARG
+    assert lib.sep_ep_mark_padding(4, 16, None, None, 64, None, None, None, None) == sep.SEP_ERR_INVALID_ARG
+    ptr = ctypes.c_void_p()
+    assert lib.sep_ep_buffer_alloc(0, ctypes.byref(ptr), ctypes.create_string_buffer(64)) == sep.SEP_ERR_INVALID_ARG
+    assert lib.sep_ep_buffer_alloc(64, None, None) == sep.SEP_ERR_INVALID_ARG
+    assert lib.sep_ep_buffer_open(None, ctypes.byref(ptr)) == sep.SEP_ERR_INVALID_ARG
+    assert lib.sep_ep_buffer_close(None, 1) == sep.SEP_OK
