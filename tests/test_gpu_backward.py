@@ -100,7 +100,7 @@ def test_backward_pair_extreme_routings(kind):
     _check_backward(idx, 16, 4, 32, 264, seed=62)          # H = 264: a ragged last 16-byte column block
 
 
-@pytest.mark.parametrize("T,k,H", [(1, 1, 8), (5, 3, 24), (300, 9, 136), (64, 32, 64)])
+@pytest.mark.parametrize("T,k,H", [(1, 1, 8), (5, 3, 24), (300, 9, 136), (64, 32, 64), (40, 4, 65536)])
 def test_backward_pair_shapes(T, k, H):
     g = torch.Generator().manual_seed(T * 100 + k)
     idx = torch.randint(-1, 40, (T, k), generator=g, dtype=torch.int32)

@@ -103,14 +103,14 @@ def test_expert_count_range(E, R):
     run_bf16_path(idx, W.random_x(T, 8, seed=E), W.random_weights(T, k, seed=E), E, R, 8)
 
 
-@pytest.mark.parametrize("H", [8, 24, 264, 4104, 16384])
+@pytest.mark.parametrize("H", [8, 24, 264, 4104, 16384, 65536])
 def test_hidden_sizes_bf16(H):
     T, k, E = 97, 3, 12
     idx = W.edge_routing("uniform", T, k, E, 3, seed=H)
     run_bf16_path(idx, W.random_x(T, H, seed=H), W.random_weights(T, k, seed=H), E, 3, 16)
 
 
-@pytest.mark.parametrize("H", [128, 384, 640, 16384])
+@pytest.mark.parametrize("H", [128, 384, 640, 16384, 65536])
 @pytest.mark.parametrize("scale", ["f32", "ue8m0", "f32_pow2"])
 def test_hidden_sizes_fp8(H, scale):
     T, k, E = 61, 4, 16

@@ -79,3 +79,10 @@ def test_scatter_combine_on_an_unsynced_layout():
     w = W.scaled(W.WORKLOADS["train8k"], 700)
     d = W.make_inputs(w, with_x=False)
     _check_scatter(d["topk_idx"], d["topk_weight"], w.E, w.R, w.B, w.H, seed=34, sync=False)
+
+
+def test_scatter_combine_largest_hidden():
+    """H = 65536, the largest the ABI accepts: 8192 16-byte vectors per row."""
+    idx = W.edge_routing("uniform", 40, 4, 16, 4, seed=34)
+    wts = W.random_weights(40, 4, seed=35)
+    _check_scatter(idx, wts, 16, 4, 32, 65536, seed=36)
