@@ -1058,7 +1058,7 @@ sep_status sep_ep_dispatch(const sep_handle *h, uint32_t layout_epoch, const voi
                            int32_t *const *recv_token, int32_t *const *recv_rank, int32_t *const *recv_slot,
                            uint32_t *error, void *stream)
 {
-    EpCommon c;
+    EpCommon c{};
     sep_status st = ep_common(h, layout_epoch, hidden, delta, pool_rows, error, &c);
     if (st != SEP_OK)
         return st;
@@ -1108,7 +1108,7 @@ sep_status sep_ep_dispatch_fp8(const sep_handle *h, uint32_t layout_epoch, const
                                const int64_t *pool_rows, int32_t *const *recv_token, int32_t *const *recv_rank,
                                int32_t *const *recv_slot, uint32_t *error, void *stream)
 {
-    EpCommon c;
+    EpCommon c{};
     sep_status st = ep_common(h, layout_epoch, hidden, delta, pool_rows, error, &c);
     if (st != SEP_OK)
         return st;
@@ -1200,7 +1200,7 @@ sep_status sep_ep_combine(const sep_handle *h, uint32_t layout_epoch, const void
                           const int64_t *pool_rows, int64_t hidden, const int32_t *delta, const float *topk_weight,
                           void *out, uint32_t *error, void *stream)
 {
-    EpCommon c;
+    EpCommon c{};
     sep_status st = ep_common(h, layout_epoch, hidden, delta, pool_rows, error, &c);
     if (st != SEP_OK)
         return st;
