@@ -767,9 +767,12 @@ def ep_compare(w, dev, flush, peak_gbs, steps=100):
     one GPU: the workload's T tokens split into R rank shards of T/R (own
     seeds), each rank laid out alone, the counts planned, then every rank's
     dispatch into the owners' pools and every rank's combine from them (the
-    kernels a multi-GPU group runs with peer pointers).  Against the
-    single-GPU dispatch + combine of the same tokens concatenated (same rows,
-    same bytes).  Layouts and the plan are outside the timed region in both."""
+    kernels a multi-GPU group runs with peer pointers), timed two ways: the
+    ranks one after another on one stream, and each rank on its own stream
+    with a join (the group's barrier) between the dispatches and the combines.
+    Against the single-GPU dispatch + combine of the same tokens concatenated
+    (same rows, same bytes).  Layouts and the plan are outside the timed
+    region in all three."""
     import numpy as np
     import torch
     import combine_route_layout_02_b200 as sep
@@ -792,6 +795,26 @@ def ep_compare(w, dev, flush, peak_gbs, steps=100):
         for r in range(R):
             sep.sep_ep_combine(hs[r], pools, rows, deltas[r], ws[r], outs[r], err)
 
+    streams = [torch.cuda.Stream(device=dev) for _ in range(R)]
+
+    def join(main):
+        for st in streams:                               # the group's barrier: every rank's kernels done
+            main.wait_stream(st)
+        for st in streams:
+            st.wait_stream(main)
+
+    def ep_concurrent_step():
+        main = torch.cuda.current_stream()
+        for st in streams:
+            st.wait_stream(main)
+        for r in range(R):
+            sep.sep_ep_dispatch(hs[r], xs[r], r, deltas[r], pools, rows, err, stream=streams[r])
+        join(main)
+        for r in range(R):
+            sep.sep_ep_combine(hs[r], pools, rows, deltas[r], ws[r], outs[r], err, stream=streams[r])
+        for st in streams:
+            main.wait_stream(st)
+
     idx_cat = torch.cat([sd["topk_idx"] for sd in shards]).to(dev)
     x_cat = torch.cat([sd["x"] for sd in shards]).to(dev)
     w_cat = torch.cat([sd["topk_weight"] for sd in shards]).to(dev)
@@ -804,16 +827,21 @@ def ep_compare(w, dev, flush, peak_gbs, steps=100):
         sep.sep_combine(h1, pool1, w_cat, out1)
 
     ep_us = _time_arm(ep_step, steps, flush)
+    ep_conc_us = _time_arm(ep_concurrent_step, steps, flush)
     single_us = _time_arm(single_step, steps, flush)
     assert int(err.item()) == 0, "a row fell outside its owner's pool"
     for h in hs + [h1]:
         sep.sep_handle_free(h)
     b = algorithmic_bytes(replace(w, T=R * Tr))
     moved = b["dispatch"] + b["combine"]
-    return {"ranks": R, "tokens_per_rank": Tr, "ep_us": ep_us, "single_gpu_us": single_us,
+    return {"ranks": R, "tokens_per_rank": Tr, "ep_us": ep_us, "ep_concurrent_us": ep_conc_us,
+            "single_gpu_us": single_us,
             "ep_gbs": moved / (ep_us * 1e-6) / 1e9, "ep_frac": moved / (ep_us * 1e-6) / 1e9 / peak_gbs,
+            "ep_concurrent_frac": moved / (ep_conc_us * 1e-6) / 1e9 / peak_gbs,
             "note": "R ranks emulated on one GPU (2R launches: every rank's dispatch, then every rank's combine, "
-                    "into / from the owners' pools); single_gpu is the same tokens' dispatch + combine; "
+                    "into / from the owners' pools); ep_us runs them one after another on one stream, "
+                    "ep_concurrent_us runs each rank on its own stream with a join between the dispatches and "
+                    "the combines (the group's barrier); single_gpu is the same tokens' dispatch + combine; "
                     "layouts outside the timed region; L2 flushed before every step"}
 
 
