@@ -45,3 +45,21 @@ def test_argument_defaults():
     a = bench.parse_args([])
     assert a.extras.split(",") == ["borrowed", "backward", "gate", "scatter", "ep"]
     assert not a.no_graph and not a.no_extras and a.gate_ctas == 0 and a.consumer_ctas == 64
+
+
+def test_reference_arm_line_on_the_host_cores():
+    """`--impl reference` times the oracle on the host cores (no GPU): rank 0
+    prints the contract's line with the cpu_baseline description and a zero-copy
+    e2e; any other rank does no work."""
+    args = bench.parse_args(["--impl", "reference", "--workload", "tiny", "--steps", "2", "--warmup", "1"])
+    assert bench.run_reference(args, rank=1) is None
+    res = bench.run_reference(args, rank=0)
+    assert res["impl"] == "reference" and res["metric"] == bench.METRIC and res["unit"] == "tokens/s"
+    assert res["value"] > 0 and res["ms_per_step"] > 0 and res["higher_is_better"] is True
+    assert (res["steps"], res["warmup"], res["n_gpus"]) == (2, 1, 1)
+    cb = res["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == res["value"] and cb["sample"]
+    assert res["e2e"] == {"value": res["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                          "d2h_bytes_per_step": 0}
+    assert res["gpu_launches"] == 0 and res["config"]["workload"] == "tiny"
+    json.dumps(res)                                       # one JSON line
