@@ -63,3 +63,18 @@ def test_reference_arm_line_on_the_host_cores():
                           "d2h_bytes_per_step": 0}
     assert res["gpu_launches"] == 0 and res["config"]["workload"] == "tiny"
     json.dumps(res)                                       # one JSON line
+
+
+def test_cpu_baseline_reports_the_oracle_on_a_bounded_sample():
+    """The cpu_baseline object of our arm's line: the oracle on one core and on
+    every core, the faster reported, both kept; bounded by the budget."""
+    import time
+    w = W.WORKLOADS["tiny"]
+    d = W.make_inputs(w)
+    t0 = time.perf_counter()
+    cb = bench.cpu_baseline(w, d, 0.5)
+    assert time.perf_counter() - t0 < 60
+    assert cb["kind"] == "oracle" and cb["unit"] == "tokens/s" and cb["value"] > 0 and cb["sample"]
+    assert cb["single_core"]["cores"] == 1 and cb["single_core"]["value"] > 0
+    assert cb["value"] == max(cb["single_core"]["value"], cb["all_cores"].get("value", 0))
+    assert cb["cores"] == (cb["all_cores"]["cores"] if cb["value"] == cb["all_cores"].get("value") else 1)
