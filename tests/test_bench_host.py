@@ -78,3 +78,61 @@ def test_cpu_baseline_reports_the_oracle_on_a_bounded_sample():
     assert cb["single_core"]["cores"] == 1 and cb["single_core"]["value"] > 0
     assert cb["value"] == max(cb["single_core"]["value"], cb["all_cores"].get("value", 0))
     assert cb["cores"] == (cb["all_cores"]["cores"] if cb["value"] == cb["all_cores"].get("value") else 1)
+
+
+class _FakeNvml:
+    """Stands in for pynvml: read-only clock queries on a fake device."""
+    NVML_CLOCK_SM = 1
+    nvmlClocksEventReasonHwSlowdown = 0x8
+    nvmlClocksEventReasonHwThermalSlowdown = 0x40
+    nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    nvmlClocksEventReasonSwPowerCap = 0x4
+    nvmlClocksEventReasonHwPowerBrakeSlowdown = 0x80
+
+    def __init__(self, clocks, reasons, fail_init=False):
+        self.clocks, self.reasons, self.fail_init = list(clocks), reasons, fail_init
+        self.opened = None
+
+    def nvmlInit(self):
+        if self.fail_init:
+            raise RuntimeError("no driver")
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        self.opened = i
+        return ("dev", i)
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        return self.clocks.pop(0) if len(self.clocks) > 1 else self.clocks[0]
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return self.reasons
+
+
+def test_clock_sampler_reads_clocks_and_reasons_from_nvml(monkeypatch):
+    import sys
+    import time
+    fake = _FakeNvml([1965, 1890, 1965, 1965], _FakeNvml.nvmlClocksEventReasonSwPowerCap)
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "3,5")
+    with bench.ClockSampler(1, period_s=0.001) as s:
+        time.sleep(0.05)
+    got = s.summary()
+    assert fake.opened == 5                               # the physical index behind device 1
+    assert got["sm_max_mhz"] == 1965 and got["sm_mhz"] == 1965 and got["samples"] >= 4
+    assert got["reasons"] == ["sw_power_cap"] and got["source"] == "nvml"
+    fake.reasons = _FakeNvml.nvmlClocksEventReasonHwThermalSlowdown | _FakeNvml.nvmlClocksEventReasonHwSlowdown
+    with bench.ClockSampler(0, period_s=0.001) as s:
+        time.sleep(0.02)
+    assert s.summary()["reasons"] == ["hw_slowdown", "hw_thermal_slowdown"]
+
+
+def test_clock_sampler_without_nvml_reports_it(monkeypatch):
+    import sys
+    monkeypatch.setitem(sys.modules, "pynvml", _FakeNvml([1965], 0, fail_init=True))
+    with bench.ClockSampler(0) as s:
+        pass
+    got = s.summary()
+    assert got["sm_mhz"] is None and got["source"] == "nvml unavailable" and got["samples"] == 0
