@@ -6,6 +6,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 import combine_route_layout_02_b200 as sep
 from combine_route_layout_02_b200 import build
@@ -115,3 +116,18 @@ def test_expert_parallel_calls_reject_bad_arguments_before_any_cuda_call():
     assert lib.sep_ep_buffer_alloc(64, None, None) == sep.SEP_ERR_INVALID_ARG
     assert lib.sep_ep_buffer_open(None, ctypes.byref(ptr)) == sep.SEP_ERR_INVALID_ARG
     assert lib.sep_ep_buffer_close(None, 1) == sep.SEP_OK
+
+
+def test_host_tensors_are_refused_not_computed():
+    """The binding has no CPU path: host tensors are refused with an error
+    before the library is called, never laid out, dispatched or combined."""
+    h = sep.Handle(ctypes.c_void_p(None))
+    idx = torch.zeros(4, 2, dtype=torch.int32)
+    x = torch.zeros(4, 16, dtype=torch.bfloat16)
+    pool = torch.zeros(64, 16, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="device tensors"):
+        sep.sep_layout(idx, 8, 2, 16)
+    with pytest.raises(ValueError, match="device tensors"):
+        sep.sep_dispatch(h, x, pool)
+    with pytest.raises(ValueError, match="device tensors"):
+        sep.sep_combine(h, pool, torch.zeros(4, 2), torch.zeros(4, 16, dtype=torch.bfloat16), layout_epoch=1)
