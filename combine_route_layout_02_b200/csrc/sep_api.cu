@@ -1294,6 +1294,9 @@ void sep_handle_free(sep_handle *h)
     int prev = -1;
     const bool switched = cudaGetDevice(&prev) == cudaSuccess && prev != h->device &&
                           cudaSetDevice(h->device) == cudaSuccess;
+    // consumers of the last borrowed view still read the row map: the free
+    // waits for the streams its release recorded
+    wait_for_release(h, h->last_stream, true);
     if (h->block != nullptr)
         cudaFreeAsync(h->block, h->last_stream);
     if (h->host_mirror != nullptr)

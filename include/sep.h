@@ -552,9 +552,10 @@ SEP_API sep_status sep_ep_buffer_open(const void *ipc_handle, void **ptr);
 SEP_API sep_status sep_ep_buffer_close(void *ptr, int opened);
 
 /* Frees the handle.  Its device memory is released stream-ordered on the
- * stream of the last call that used it; the caller must have ordered every
- * other stream that used the handle before that point.  NULL is a no-op; a
- * handle with an active borrowed view is not freed (release the view first). */
+ * stream of the last call that used it, after the streams the last
+ * sep_view_release named; the caller must have ordered every other stream
+ * that used the handle before that point.  NULL is a no-op; a handle with an
+ * active borrowed view is not freed (release the view first). */
 SEP_API void sep_handle_free(sep_handle *handle);
 
 /* Message for the calling thread's last failed call ("" if none). */
