@@ -228,6 +228,69 @@ def test_dispatch_bf16_rows_equal_source_tokens():
 
 # ------------------------------------------------------------- fp8 pins
 
+def _fp8_dispatch_case(seed=21, T=24, k=4, E=6, R=2, B=4, H=384):
+    """A routing with masked entries and duplicate experts inside a token's top-k."""
+    rng = np.random.default_rng(seed)
+    idx = rng.integers(-1, E, size=(T, k))
+    idx[0] = [2, 2, -1, 2][:k]                   # the same expert three times, one masked entry
+    idx[1] = -1                                  # a token with no assignment
+    lay = oracle.layout(idx, E, R, B)
+    x = W.random_x(T, H, seed=seed + 1)
+    x[3, :128] = 0                               # an all-zero group
+    x[5] *= 300.0                                # groups that saturate
+    return lay, x
+
+
+@pytest.mark.parametrize("scale", ["f32", "ue8m0", "f32_pow2"])
+def test_dispatch_fp8_rows_equal_quantised_source_tokens(scale):
+    """FP8 dispatch places each token's codes and per-group scales, quantised once,
+    into every pool row of that token (low-latency kernels article, "FP8 and
+    Quantization Support": the scales travel with the payload rows).  Each valid
+    row is checked against the separately pinned single-row quantiser of its
+    source token; padding rows stay untouched."""
+    lay, x = _fp8_dispatch_case()
+    xu = oracle.as_u16(x)
+    codes, scales = oracle.dispatch_fp8(x, lay, scale)
+    P = lay.num_pool_rows
+    assert codes.shape == (P, x.shape[1]) and scales.shape == (P, x.shape[1] // 128)
+    assert (lay.src_pool_row < 0).any() and len(set(lay.src_pool_row[0][lay.src_pool_row[0] >= 0])) == 3
+    for row in range(P):
+        t = lay.pool_recv_token[row]
+        if t < 0:
+            assert (codes[row] == 0).all() and (scales[row] == 0).all()
+            continue
+        want_c, want_s = oracle.quant_row(xu[t], scale)
+        np.testing.assert_array_equal(codes[row], want_c)
+        np.testing.assert_array_equal(scales[row], want_s)
+    # every valid (t, j) reaches a row holding token t's quantisation
+    for t in range(lay.T):
+        for j in range(lay.k):
+            r = lay.src_pool_row[t, j]
+            if r >= 0:
+                np.testing.assert_array_equal(codes[r], oracle.quant_row(xu[t], scale)[0])
+
+
+def test_dequant_rows_follow_the_format_and_the_group_scales():
+    """decode(code) times its own 128-channel group's scale, from the e4m3 value
+    table of the format definition and the scale encodings (fp32 value or UE8M0
+    byte b meaning 2^(b-127))."""
+    rng = np.random.default_rng(31)
+    rows, H = 5, 512
+    codes = rng.integers(0, 256, size=(rows, H)).astype(np.uint8)
+    codes[codes == 0x7f] = 0x7e
+    codes[codes == 0xff] = 0xfe
+    su = rng.integers(100, 150, size=(rows, H // 128)).astype(np.uint8)
+    sf = rng.uniform(0.01, 3.0, size=(rows, H // 128)).astype(np.float32)
+    tab = _TABLE[codes.astype(np.int64)]
+    got_u = oracle.dequant_rows(codes, su, "ue8m0")
+    want_u = (tab * np.repeat(2.0 ** (su.astype(np.float64) - 127), 128, axis=1)).astype(np.float32)
+    np.testing.assert_array_equal(got_u, want_u)
+    got_f = oracle.dequant_rows(codes, sf, "f32")
+    want_f = (tab.astype(np.float32) * np.repeat(sf, 128, axis=1)).astype(np.float32)
+    np.testing.assert_array_equal(got_f, want_f)
+
+
+
 def test_e4m3_decode_matches_format_and_torch():
     g = _golden("e4m3_codes.json")
     dec = oracle.e4m3_decode(np.arange(256))
@@ -405,6 +468,20 @@ def _pins_fail(L) -> bool:
             for i, c in gq[scale]["nonzero_codes"].items():
                 want[int(i)] = int(c, 16)
             np.testing.assert_array_equal(codes, want)
+        lay8, x8 = _fp8_dispatch_case()
+        x8u = oracle.as_u16(x8)
+        for scale in ("f32", "ue8m0"):
+            codes, scales = oracle.dispatch_fp8(x8, lay8, scale, L=L)
+            for row in range(lay8.num_pool_rows):
+                t = lay8.pool_recv_token[row]
+                if t >= 0:
+                    want_c, want_s = oracle.quant_row(x8u[t], scale)
+                    np.testing.assert_array_equal(codes[row], want_c)
+                    np.testing.assert_array_equal(scales[row], want_s)
+            deq = oracle.dequant_rows(codes, scales, scale, L=L)
+            sc = scales.astype(np.float64) if scale == "f32" else 2.0 ** (scales.astype(np.float64) - 127)
+            want = (_TABLE[codes.astype(np.int64)] * np.repeat(sc, 128, axis=1)).astype(np.float32)
+            np.testing.assert_array_equal(deq, want)
         for a in [448.0, 896.0, 7.0, 1e-3]:
             E = oracle.ue8m0_exponent(a, L=L)
             assert 448.0 * 2.0 ** E >= a and 448.0 * 2.0 ** (E - 1) < a
@@ -436,6 +513,20 @@ MUTANTS = [
     ("float prod = topk_weight[t * k + j] *", "float prod = topk_weight[t * k + (k - 1 - j)] *"),  # wrong operand
     ("if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u)))",
      "if (lower >= 0x8000u)"),                                                            # ties away in bf16
+    # FP8 dispatch: scales placed at the token's index instead of the pool row's
+    ("memcpy(recv_scales_u8 + (int64_t)row * G, su_tmp, (size_t)G);",
+     "memcpy(recv_scales_u8 + (int64_t)t * G, su_tmp, (size_t)G);"),
+    ("memcpy(recv_scales_f32 + (int64_t)row * G, sf_tmp, (size_t)G * sizeof(float));",
+     "memcpy(recv_scales_f32 + (int64_t)t * G, sf_tmp, (size_t)G * sizeof(float));"),
+    # FP8 dispatch: codes written only for the first top-k slot
+    ("memcpy(recv + (int64_t)row * H, codes_tmp, (size_t)H);",
+     "if (j == 0) memcpy(recv + (int64_t)row * H, codes_tmp, (size_t)H);"),
+    # FP8 dispatch: a group's scale taken from the wrong group
+    ("memcpy(recv_scales_f32 + (int64_t)row * G, sf_tmp, (size_t)G * sizeof(float));",
+     "memcpy(recv_scales_f32 + (int64_t)row * G, sf_tmp + 1, (size_t)(G - 1) * sizeof(float));"),
+    # dequantisation: wrong 128-channel group, wrong UE8M0 bias
+    ("scales_f32[r * G + h / 128];", "scales_f32[r * G + h / 256];"),
+    ("(int)scales_u8[r * G + h / 128] - 127)", "(int)scales_u8[r * G + h / 128] - 128)"),
 ]
 
 
