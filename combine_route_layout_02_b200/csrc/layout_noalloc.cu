@@ -11,6 +11,7 @@
 // and stable assignment, split by two bounded grid barriers) restated for
 // caller-owned outputs; it writes no arrival counters, owner token counts or
 // token-owner flags (those belong to a handle).
+#include <atomic>
 #include <cstring>
 
 #include "sep_internal.cuh"
@@ -241,8 +242,10 @@ __global__ void __launch_bounds__(kWarps * 32) layout_noalloc_kernel(NoAllocPara
     }
 }
 
-// Device address of the scratch array, looked up once per device.
-int32_t *g_scratch_addr[64] = {nullptr};
+// Device address of the scratch array, looked up once per device.  Threads
+// that make their first call at the same time may both look it up; they store
+// the same value, and the atomics make that well defined.
+std::atomic<int32_t *> g_scratch_addr[64] = {};
 
 bool aligned(const void *ptr, uintptr_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
 
@@ -292,7 +295,8 @@ extern "C" sep_status sep_layout_noalloc(const void *topk_idx, int idx_bytes, in
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || dev < 0 || dev >= 64)
         return set_error(SEP_ERR_CUDA, "sep_layout_noalloc: cudaGetDevice failed");
-    if (g_scratch_addr[dev] == nullptr) {
+    int32_t *scratch = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (scratch == nullptr) {
         // set-up, once per device with that device current: the array's device
         // address (host code only sees a host-side stand-in for it) and the
         // kernels loaded now rather than lazily at a later launch
@@ -304,9 +308,9 @@ extern "C" sep_status sep_layout_noalloc(const void *topk_idx, int idx_bytes, in
         if (cudaFuncGetAttributes(&fa, reinterpret_cast<const void *>(layout_noalloc_kernel<int>)) != cudaSuccess ||
             cudaFuncGetAttributes(&fa, reinterpret_cast<const void *>(layout_noalloc_kernel<long long>)) != cudaSuccess)
             return set_error(SEP_ERR_CUDA, "sep_layout_noalloc: loading its kernels failed");
-        g_scratch_addr[dev] = static_cast<int32_t *>(addr);
+        scratch = static_cast<int32_t *>(addr);
+        g_scratch_addr[dev].store(scratch, std::memory_order_release);
     }
-    int32_t *scratch = g_scratch_addr[dev];
 
     NoAllocParams p{};
     p.topk_idx = topk_idx;

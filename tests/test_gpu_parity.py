@@ -15,8 +15,8 @@ import torch
 import combine_route_layout_02_b200 as sep
 import oracle
 import workloads as W
-from gpu_harness import (POISON_BF16, bf16_bits, check_combine, check_layout, poisoned_bf16,
-                         run_bf16_path, run_fp8_path, u16_to_bf16_tensor)
+from gpu_harness import (POISON_BF16, POISON_F32_BITS, POISON_U8, bf16_bits, check_combine, check_layout,
+                         poisoned_bf16, run_bf16_path, run_fp8_path, u16_to_bf16_tensor)
 
 pytestmark = pytest.mark.gpu
 
@@ -324,6 +324,46 @@ def test_streaming_tile_ready_and_consumer():
         sep.sep_handle_free(h)
 
 
+def test_handle_free_between_consumer_and_dispatch_does_not_wait_for_the_device():
+    """A handle is freed on the host after a consumer was launched and before
+    the dispatch it waits for.  The free must not wait for the device: if it
+    did, the host would sit in it until the consumer's bounded wait gave up,
+    and the consumer would report SEP_ERR_TIMEOUT instead of copying every
+    tile."""
+    w, d = _inputs(W.WORKLOADS["streaming"], 2048, 512)
+    lay = oracle.layout(d["topk_idx"].numpy(), w.E, w.R, w.B)
+    idx = d["topk_idx"].cuda()
+    other = sep.sep_layout(idx, w.E, w.R, w.B)
+    h = sep.sep_layout(idx, w.E, w.R, w.B)
+    freed = False
+    try:
+        info = h.info()
+        rows = info.max_pool_rows
+        x = d["x"].cuda()
+        recv = poisoned_bf16(rows, w.H)
+        dst = poisoned_bf16(rows, w.H)
+        tile_ready = torch.zeros(info.max_tiles, dtype=torch.int32, device="cuda")
+        status = torch.zeros(2, dtype=torch.int32, device="cuda")
+        main = torch.cuda.current_stream()
+        side = torch.cuda.Stream()
+        torch.cuda.synchronize()
+        side.wait_stream(main)
+        sep.sep_consume_tiles(h, recv, tile_ready, 5, dst, status, num_ctas=16, stream=side)
+        sep.sep_handle_free(other)                     # between the consumer and its producer
+        freed = True
+        sep.sep_dispatch(h, x, recv, tile_ready=tile_ready, dispatch_seq=5, stream=main)
+        main.wait_stream(side)
+        torch.cuda.synchronize()
+        assert status.cpu().tolist() == [0, 0]
+        want = oracle.dispatch_bf16(d["x"], lay)
+        valid = lay.pool_recv_token >= 0
+        np.testing.assert_array_equal(bf16_bits(dst)[:lay.num_pool_rows][valid], want[valid])
+    finally:
+        if not freed:
+            sep.sep_handle_free(other)
+        sep.sep_handle_free(h)
+
+
 def test_streaming_fp8_publishes_every_tile():
     w, d = _inputs(W.WORKLOADS["decode"], 256)
     lay = oracle.layout(d["topk_idx"].numpy(), w.E, w.R, w.B)
@@ -388,36 +428,38 @@ def test_full_train8k_bench_configuration():
 
 
 @pytest.mark.slow
-def test_full_prefill_skew_bench_configuration_sampled():
+def test_full_prefill_skew_bench_configuration():
+    """T=16384, H=7168, E=256 in 8 owners, Zipf(1.2)-skewed top-8, BLOCK_M=128,
+    FP8 with fp32 scales, in the benchmark's launch configuration (unsynced
+    layout, worst-case buffers): every valid row's codes and scales, and every
+    token's combine output, compared with the oracle."""
     w = W.WORKLOADS["prefill_skew"]
     d = W.make_inputs(w)
     lay = oracle.layout(d["topk_idx"].numpy(), w.E, w.R, w.B)
-    h = sep.sep_layout(d["topk_idx"].cuda(), w.E, w.R, w.B)
+    h = sep.sep_layout(d["topk_idx"].cuda(), w.E, w.R, w.B, flags=0)
     try:
         check_layout(h, lay)
         info = h.info()
-        rows, G = info.max_pool_rows, w.H // 128
-        recv = torch.empty(rows, w.H, dtype=torch.uint8, device="cuda")
-        scales = torch.empty(rows, G, dtype=torch.float32, device="cuda")
+        rows, G, P = info.max_pool_rows, w.H // 128, lay.num_pool_rows
+        recv = torch.full((rows, w.H), POISON_U8, dtype=torch.uint8, device="cuda")
+        scales = torch.full((rows, G), POISON_F32_BITS, dtype=torch.int32, device="cuda").view(torch.float32)
         sep.sep_dispatch(h, d["x"].cuda(), recv, payload="fp8", scale="f32", recv_scales=scales)
-        rng = np.random.default_rng(0)
-        sample = np.sort(rng.choice(w.T, 512, replace=False))
-        sample = np.unique(np.concatenate([sample, [0, w.T - 1]]))
-        xs = oracle.as_u16(d["x"])
-        codes_gpu, scales_gpu = recv.cpu().numpy(), scales.cpu().numpy()
-        for t in sample:
-            codes, sc = oracle.quant_row(xs[t], "f32")
-            for r in lay.src_pool_row[t]:
-                np.testing.assert_array_equal(codes_gpu[r], codes)
-                np.testing.assert_array_equal(scales_gpu[r].view(np.uint32), sc.view(np.uint32))
-        # combine over a seeded bf16 pool (rows repeat a 61-row table)
-        table = oracle.as_u16(W.random_x(61, w.H, seed=77))
-        y = np.take(table, np.arange(info.max_pool_rows) % 61, axis=0)
+        valid = lay.pool_recv_token >= 0
+        codes_gpu = recv[:P].cpu().numpy()
+        scales_gpu = scales[:P].cpu().numpy()
+        del recv, scales
+        want_codes, want_scales = oracle.dispatch_fp8(d["x"], lay, "f32")
+        np.testing.assert_array_equal(codes_gpu[valid], want_codes[valid])
+        np.testing.assert_array_equal(scales_gpu[valid].view(np.uint32), want_scales[valid].view(np.uint32))
+        assert (codes_gpu[~valid] == POISON_U8).all(), "a padding row was written"
+        del codes_gpu, scales_gpu, want_codes, want_scales
+        # combine over a seeded bf16 pool (rows repeat a 61-row table), every token
+        table = W.random_x(61, w.H, seed=77)
+        y = table[torch.arange(rows) % 61].contiguous()
         out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device="cuda")
-        sep.sep_combine(h, u16_to_bf16_tensor(y).cuda(), d["topk_weight"].cuda(), out)
-        sub = oracle.Layout(**{**lay.__dict__, "T": len(sample), "src_pool_row": np.ascontiguousarray(lay.src_pool_row[sample])})
-        want = oracle.combine(y, d["topk_weight"].numpy()[sample], sub)
-        check_combine(bf16_bits(out)[sample], want)
+        sep.sep_combine(h, y.cuda(), d["topk_weight"].cuda(), out)
+        want = oracle.combine(y, d["topk_weight"].numpy(), lay)
+        check_combine(bf16_bits(out), want)
     finally:
         sep.sep_handle_free(h)
 

@@ -8,6 +8,14 @@ an 8-bit significand), each of the k - 1 additions rounds a partial sum whose
 magnitude is at most S = sum_j |w_j y_j|, and the oracle's own result carries
 one bf16 rounding; so |scatter - oracle| <= (2k + 1) * 2^-8 * S, with 2% slack
 for second-order terms.
+
+That worst case is loose: the roundings rarely line up.  A second, empirical
+ceiling catches a regression well inside it.  A CPU simulation of the same
+arithmetic (N(0,1) rows, renormalised weights, products and partial sums
+rounded to bf16, the k terms added in a random order) puts the 99.9th
+percentile of |scatter - oracle| / (2^-8 * S) at 2.0 to 2.3 for k <= 8 and its
+mean at 0.31 to 0.34; the tests require the 99.9th percentile to stay at or
+below 3 and the mean at or below 0.6, and print what they observe.
 """
 import numpy as np
 import pytest
@@ -21,14 +29,18 @@ from gpu_harness import bf16_bits, poisoned_bf16
 pytestmark = pytest.mark.gpu
 
 
-def _bound(y_bits, w, lay):
+P999_CEILING, MEAN_CEILING = 3.0, 0.6       # in units of 2^-8 * S (see above)
+
+
+def _abs_sum(y_bits, w, lay):
+    """S = sum_j |w_j y_j| per output element."""
     y = oracle.bf16_to_f32(y_bits).astype(np.float64)
     rows = lay.src_pool_row
     S = np.zeros((lay.T, y.shape[1]))
     for j in range(lay.k):
         ok = rows[:, j] >= 0
         S[ok] += np.abs(w[ok, j, None].astype(np.float64) * y[rows[ok, j]])
-    return (2 * lay.k + 1) * 2.0 ** -8 * S * 1.02
+    return S
 
 
 def _check_scatter(idx, w, E, R, B, H, seed, sync=True):
@@ -46,9 +58,19 @@ def _check_scatter(idx, w, E, R, B, H, seed, sync=True):
         got = oracle.bf16_to_f32(bf16_bits(out)).astype(np.float64)
         want = oracle.bf16_to_f32(oracle.combine(oracle.as_u16(y), w.numpy(), lay)).astype(np.float64)
         err = np.abs(got - want)
-        bound = _bound(oracle.as_u16(y), w.numpy(), lay)
+        S = _abs_sum(oracle.as_u16(y), w.numpy(), lay)
+        bound = (2 * lay.k + 1) * 2.0 ** -8 * S * 1.02
         assert np.isfinite(got).all()
         assert (err <= bound).all(), f"max err {err.max()}, worst excess {(err - bound).max()}"
+        nz = S > 0
+        assert (err[~nz] == 0).all()                    # tokens with nothing to add stay exactly zero
+        if nz.any():
+            ratio = err[nz] / (2.0 ** -8 * S[nz])
+            p999, mean = float(np.quantile(ratio, 0.999)), float(ratio.mean())
+            print(f"scatter error / (2^-8 S): p99.9 {p999:.3f}, mean {mean:.3f}, max {ratio.max():.3f} "
+                  f"(worst-case bound {2 * lay.k + 1})")
+            assert p999 <= P999_CEILING, f"99.9th percentile {p999:.3f} above {P999_CEILING}"
+            assert mean <= MEAN_CEILING, f"mean {mean:.3f} above {MEAN_CEILING}"
         return err.max()
     finally:
         sep.sep_handle_free(h)

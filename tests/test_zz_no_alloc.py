@@ -124,3 +124,63 @@ def test_noalloc_layout_equals_the_oracle(T, k, E, R, B, masked):
         np.testing.assert_array_equal(out["src_pool_row"].cpu().numpy(), lay.src_pool_row)
     np.testing.assert_array_equal(out["pool_recv_token"][:P].cpu().numpy(), lay.pool_recv_token)
     np.testing.assert_array_equal(out["pool_recv_slot"][:P].cpu().numpy(), lay.pool_recv_slot)
+
+
+def test_noalloc_wrapper_rejects_short_or_mistyped_arrays():
+    """The C ABI receives only pointers, so the binding checks every output
+    array's type and length before the call (CPU tensors: nothing reaches the
+    library)."""
+    T, k, E, R, B = 16, 2, 8, 2, 4
+    idx = torch.zeros(T, k, dtype=torch.int32)
+    good = {
+        "expert_counts": torch.zeros(E, dtype=torch.int32), "owner_counts": torch.zeros(R, dtype=torch.int32),
+        "expert_pool_block_offset": torch.zeros(E + 1, dtype=torch.int32),
+        "owner_pool_row_offset": torch.zeros(R + 1, dtype=torch.int32),
+        "tile_expert": torch.zeros(64, dtype=torch.int32), "pool_arrival_target": torch.zeros(64, dtype=torch.int32),
+        "src_pool_row": torch.zeros(T, k, dtype=torch.int32), "pool_recv_token": torch.zeros(256, dtype=torch.int32),
+        "pool_recv_slot": torch.zeros(256, dtype=torch.int32), "sizes": torch.zeros(2, dtype=torch.int64),
+        "status": torch.zeros(2, dtype=torch.int32),
+    }
+    for name, bad in [("expert_counts", torch.zeros(E - 1, dtype=torch.int32)),
+                      ("expert_pool_block_offset", torch.zeros(E, dtype=torch.int32)),
+                      ("owner_pool_row_offset", torch.zeros(R, dtype=torch.int32)),
+                      ("src_pool_row", torch.zeros(T * k - 1, dtype=torch.int32)),
+                      ("sizes", torch.zeros(2, dtype=torch.int32)),
+                      ("status", torch.zeros(1, dtype=torch.int32)),
+                      ("owner_counts", torch.zeros(R, dtype=torch.int64))]:
+        with pytest.raises(ValueError, match=name):
+            sep.sep_layout_noalloc(idx, E, R, B, {**good, name: bad})
+    missing = dict(good)
+    del missing["pool_recv_slot"]
+    with pytest.raises(ValueError, match="pool_recv_slot"):
+        sep.sep_layout_noalloc(idx, E, R, B, missing)
+    with pytest.raises(ValueError, match="device"):               # well-formed, but host memory
+        sep.sep_layout_noalloc(idx, E, R, B, good)
+
+
+@pytest.mark.gpu
+def test_noalloc_reports_an_expert_id_out_of_range():
+    """An id equal to num_experts is skipped before any memory access and
+    reported in status[0]; every output equals the oracle's layout of the same
+    routing with that entry masked."""
+    import oracle
+    T, k, E, R, B = 300, 4, 16, 4, 8
+    rng = np.random.default_rng(5)
+    idx = rng.integers(0, E, size=(T, k)).astype(np.int32)
+    idx[17, 2] = E
+    idx[250, 0] = E
+    masked = idx.copy()
+    masked[masked >= E] = -1
+    lay = oracle.layout(masked, E, R, B)
+    out = _outputs(T, k, E, R, B)
+    sep.sep_layout_noalloc(torch.from_numpy(idx).cuda(), E, R, B, out)
+    torch.cuda.synchronize()
+    assert out["status"].cpu().tolist() == [1, 0]
+    P, NT = lay.num_pool_rows, lay.num_tiles
+    np.testing.assert_array_equal(out["sizes"].cpu().numpy(), [P, NT])
+    np.testing.assert_array_equal(out["expert_counts"].cpu().numpy(), lay.expert_counts)
+    np.testing.assert_array_equal(out["src_pool_row"].cpu().numpy(), lay.src_pool_row)
+    np.testing.assert_array_equal(out["pool_recv_token"][:P].cpu().numpy(), lay.pool_recv_token)
+    np.testing.assert_array_equal(out["pool_recv_slot"][:P].cpu().numpy(), lay.pool_recv_slot)
+    np.testing.assert_array_equal(out["tile_expert"][:NT].cpu().numpy(), lay.tile_expert)
+    np.testing.assert_array_equal(out["expert_pool_block_offset"].cpu().numpy(), lay.expert_pool_block_offset)
