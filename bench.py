@@ -67,6 +67,10 @@ def parse_args(argv=None):
                     help="skip timing the step replayed from a CUDA graph (non-streaming workloads)")
     ap.add_argument("--extras", default="borrowed,backward,gate,scatter,ep",
                     help="comma list of the measurements taken after the timed region")
+    ap.add_argument("--profile-case", default=None,
+                    choices=["layout", "layout_dispatch", "dispatch", "combine", "consumer", "gated", "gather",
+                             "scatter", "backward", "ep"],
+                    help="run one kernel family a few times, its producers finished first (for ncu); no timing")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the borrowed-receive, backward-pair, combine-gate and scatter-combine measurements")
     return ap.parse_args(argv)
@@ -156,7 +160,7 @@ class ClockSampler:
                ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
                ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown")]
 
-    def __init__(self, device_index: int, period_s: float = 0.005):
+    def __init__(self, device_index: int, period_s: float = 0.002):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self._stop = threading.Event()
         self._period = period_s
@@ -375,6 +379,14 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
         # starting while the first drains (programmatic dependent launch)
         if ev is not None:
             ev[0].record(main)
+        if not w.streaming and not phases:
+            # layout and dispatch in one call (one launch when the routing is small)
+            sep.sep_layout_dispatch(idxs, xs, recv, w.E, w.R, w.B, payload=w.payload, scale=w.scale,
+                                    recv_scales=scales, handle=h)
+            sep.sep_combine(h, y, wts, out)
+            if ev is not None:
+                ev[3].record(main)
+            return
         sep.sep_layout(idxs, w.E, w.R, w.B, handle=h)
         epoch = h.epoch
         if ev is not None and phases:
@@ -411,14 +423,17 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
     phase_events = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(n_phase)]
     barrier(world)
     torch.cuda.synchronize()
+    # the clock record spans the timed steps and the phase and warm loops after
+    # them (the same kernels back to back), so it holds more than the one or two
+    # samples a short timed region leaves
     sampler = ClockSampler(local)
+    sampler.__enter__()
     launches_before = sep.sep_launch_count()
-    with sampler:
-        for i in range(args.steps):
-            if flush is not None:
-                flush.zero_()
-            step(events[i])
-        torch.cuda.synchronize()
+    for i in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+        step(events[i])
+    torch.cuda.synchronize()
     launches = sep.sep_launch_count() - launches_before
     barrier(world)
     if w.streaming:
@@ -434,12 +449,14 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
     if w.streaming:
         assert status.cpu().tolist() == [0, 0], f"consumer status {status.cpu().tolist()}"
 
-    # the same step with the L2 left warm between steps (reported beside the flushed number)
-    n_warm = min(args.steps, 500)
+    # the same step with the L2 left warm between steps (reported beside the flushed
+    # number); at least 500 steps, which also gives the clock record tens of samples
+    n_warm = max(min(args.steps, 2000), 500)
     warm_events = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(n_warm)]
     for i in range(n_warm):
         step(warm_events[i])
     torch.cuda.synchronize()
+    sampler.__exit__(None, None, None)
     barrier(world)
     if w.streaming:
         assert status.cpu().tolist() == [0, 0], f"consumer status {status.cpu().tolist()}"
@@ -539,9 +556,8 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
             s_cmp.wait_event(ev_in[b])
             s_cmp.wait_event(ev_out[b])                  # step i-nb's output has been downloaded
             if kernels:
-                sep.sep_layout(S["idx"], w.E, w.R, w.B, handle=hb, stream=s_cmp)
-                sep.sep_dispatch(hb, S["x"], S["recv"], payload=w.payload, scale=w.scale,
-                                 recv_scales=S["scales"], stream=s_cmp)
+                sep.sep_layout_dispatch(S["idx"], S["x"], S["recv"], w.E, w.R, w.B, payload=w.payload,
+                                        scale=w.scale, recv_scales=S["scales"], handle=hb, stream=s_cmp)
                 sep.sep_combine(hb, S["y"], S["wt"], S["out"], stream=s_cmp)
             ev_cmp[b].record(s_cmp)
             s_out.wait_event(ev_cmp[b])
@@ -1003,9 +1019,115 @@ def run_reference(args, rank: int) -> dict | None:
     }
 
 
+def profile_case(args) -> int:
+    """One kernel family of the path on the workload's inputs, launched `steps`
+    times after `warmup` untimed launches, with every kernel it waits for
+    finished before it starts (a profiler serialises kernels, so a consumer
+    launched before its producer would only wait out its bound).  For ncu
+    captures of one kernel (-k, -c); prints one line, no measurement."""
+    import torch
+    import combine_route_layout_02_b200 as sep
+    w = W.WORKLOADS[args.workload]
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(0)
+    d = W.make_inputs(w)
+    x, idx, wt = d["x"].to(dev), d["topk_idx"].to(dev), d["topk_weight"].to(dev)
+    h = sep.sep_layout(idx, w.E, w.R, w.B, flags=sep.SEP_LAYOUT_SYNC_COUNTS)
+    info = h.info()
+    rows = info.max_pool_rows
+    recv, scales = sep.alloc_pool(h, w.H, w.payload, w.scale, rows=rows)
+    out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
+    y = (recv if w.payload == "bf16" else
+         W.random_x(61, w.H, seed=w.seed + 7).to(dev)[torch.arange(rows, device=dev) % 61].contiguous())
+    case = args.profile_case
+    n = args.warmup + args.steps
+    status = torch.zeros(2, dtype=torch.int32, device=dev)
+    if case in ("consumer", "gated"):
+        tile_ready = torch.zeros(info.max_tiles, dtype=torch.int32, device=dev)
+        dst = torch.empty_like(recv)
+        y_done = torch.zeros(w.T, dtype=torch.int32, device=dev)
+        st2 = torch.zeros(2, dtype=torch.int32, device=dev)
+        for i in range(n):
+            sep.sep_dispatch(h, x, recv, tile_ready=tile_ready, dispatch_seq=i + 1)
+            torch.cuda.synchronize()                     # every tile is published before the consumer starts
+            if case == "consumer":
+                sep.sep_consume_tiles(h, recv, tile_ready, i + 1, dst, status, num_ctas=args.consumer_ctas)
+            else:
+                sep.sep_consume_tiles_stamp(h, recv, tile_ready, i + 1, dst, status, y_done, i + 1,
+                                            num_ctas=args.consumer_ctas)
+                torch.cuda.synchronize()                 # every token is stamped before the gated combine
+                sep.sep_combine_gated(h, dst, wt, out, y_done, i + 1, st2,
+                                      num_ctas=args.gate_ctas or torch.cuda.get_device_properties(dev)
+                                      .multi_processor_count)
+            torch.cuda.synchronize()
+            assert status.cpu().tolist() == [0, 0] and st2.cpu().tolist() == [0, 0]
+    elif case == "ep":
+        R, Tr = w.R, w.T // w.R
+        shards = [W.make_inputs(replace(w, T=Tr, seed=w.seed + 7919 * (r + 1))) for r in range(R)]
+        hs = [sep.sep_layout(sd["topk_idx"].to(dev), w.E, R, w.B) for sd in shards]
+        counts = torch.stack([hh.view("expert_counts") for hh in hs]).to(torch.int32).contiguous()
+        plans = [sep.sep_ep_plan_device(counts, r, w.B) for r in range(R)]
+        owner_rows = [int(v) for v in plans[0]["owner_rows"].cpu()]
+        cap = [max(v, w.B) for v in owner_rows]
+        pools = [torch.empty(c, w.H, dtype=torch.bfloat16, device=dev) for c in cap]
+        maps = [torch.full((c,), -1, dtype=torch.int32, device=dev) for c in cap]
+        ready = [torch.zeros(c // w.B, dtype=torch.int32, device=dev) for c in cap]
+        arrival = [torch.zeros(c // w.B, dtype=torch.int32, device=dev) for c in cap]
+        dsts = [torch.empty_like(pl) for pl in pools]
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+        xs = [sd["x"].to(dev) for sd in shards]
+        ws = [sd["topk_weight"].to(dev) for sd in shards]
+        outs = [torch.empty(Tr, w.H, dtype=torch.bfloat16, device=dev) for _ in range(R)]
+        for o in range(R):
+            sep.sep_ep_mark_padding(plans[o]["owner_block_offset"], plans[o]["owner_expert_counts"], w.B, cap[o],
+                                    maps[o])
+        for i in range(n):
+            for r in range(R):
+                sep.sep_ep_plan_device(counts, r, w.B)
+                sep.sep_ep_dispatch_publish(hs[r], xs[r], r, plans[r], pools, cap, ready, arrival, i + 1, err,
+                                            recv_token=maps)
+            for o in range(R):                           # every tile already published
+                sep.sep_ep_consume_tiles(plans[o]["owner_block_offset"], pools[o], maps[o], ready[o], arrival[o],
+                                         i + 1, dsts[o], status, w.B, num_ctas=args.consumer_ctas)
+            for r in range(R):
+                sep.sep_ep_combine(hs[r], dsts, cap, plans[r]["delta"], ws[r], outs[r], err)
+            torch.cuda.synchronize()
+            assert status.cpu().tolist() == [0, 0] and int(err.item()) == 0
+        for hh in hs:
+            sep.sep_handle_free(hh)
+    else:
+        view_dst = torch.empty(info.num_pool_rows, w.H, dtype=torch.bfloat16, device=dev) if case == "gather" else None
+        grad_y = torch.empty_like(recv) if case == "backward" and w.payload == "bf16" else None
+        grad_w = torch.empty(w.T, w.k, dtype=torch.float32, device=dev)
+        for _ in range(n):
+            if case == "layout":
+                sep.sep_layout(idx, w.E, w.R, w.B, handle=h)
+            elif case == "layout_dispatch":
+                sep.sep_layout_dispatch(idx, x, recv, w.E, w.R, w.B, payload=w.payload, scale=w.scale,
+                                        recv_scales=scales, handle=h)
+            elif case == "dispatch":
+                sep.sep_dispatch(h, x, recv, payload=w.payload, scale=w.scale, recv_scales=scales)
+            elif case == "combine":
+                sep.sep_combine(h, y, wt, out)
+            elif case == "scatter":
+                sep.sep_combine_scatter(h, y, wt, out)
+            elif case == "backward":
+                sep.sep_dispatch_grads(h, out, wt, grad_y, y_pool=y, grad_w=grad_w)
+                sep.sep_combine_grads(h, grad_y, out)
+            elif case == "gather":
+                sep.sep_gather_rows(sep.sep_dispatch_borrow(h, x), view_dst)
+                sep.sep_view_release(h, [torch.cuda.current_stream()])
+        torch.cuda.synchronize()
+    sep.sep_handle_free(h)
+    print(f"profile case {case} on {w.name}: {n} rounds done", flush=True)
+    return 0
+
+
 def main(argv=None) -> int:
     args = parse_args(argv)
     rank, world, local = dist_env()
+    if args.profile_case is not None:
+        return profile_case(args)
     if args.impl == "reference":
         res = run_reference(args, rank)
         if res is not None:

@@ -33,6 +33,13 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *ptr)
     return v;
 }
 
+__device__ __forceinline__ unsigned ld_acquire_sys(const unsigned *ptr)
+{
+    unsigned v;
+    asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ uint64_t global_time_ns()
 {
     uint64_t t;
@@ -41,11 +48,13 @@ __device__ __forceinline__ uint64_t global_time_ns()
 }
 
 // 1 once tile_ready[tile] has reached seq; 0 if this or another CTA gave up.
+template <bool SYS>
 __device__ int wait_tile(const ConsumeParams &p, int tile)
 {
     const uint64_t t0 = global_time_ns();
     for (uint32_t polls = 0;; ++polls) {
-        if ((int32_t)(ld_acquire_gpu(p.tile_ready + tile) - p.seq) >= 0)
+        const unsigned v = SYS ? ld_acquire_sys(p.tile_ready + tile) : ld_acquire_gpu(p.tile_ready + tile);
+        if ((int32_t)(v - p.seq) >= 0)
             return 1;
         if (*reinterpret_cast<volatile const uint32_t *>(p.abort_flag) != 0u)
             return 0;
@@ -86,6 +95,8 @@ __device__ void stamp_tokens(const ConsumeParams &p, int tile)
     }
 }
 
+// SYS: an expert-parallel owner's pool, written by other GPUs' dispatches.
+template <bool SYS>
 __global__ void __launch_bounds__(kThreads) consume_tiles_kernel(ConsumeParams p)
 {
     __shared__ int s_off[kMaxExperts + 1];
@@ -106,15 +117,23 @@ __global__ void __launch_bounds__(kThreads) consume_tiles_kernel(ConsumeParams p
             if (pos++ % gridDim.x != blockIdx.x)
                 continue;
             const int tile = s_off[e] + i;
+            if (SYS && tile >= p.max_tiles) {            // a plan larger than the owner's arrays
+                if (threadIdx.x == 0) {
+                    atomicCAS(p.status, 0u, (uint32_t)SEP_ERR_CAPACITY);
+                    atomicAdd(p.status + 1, 1u);
+                }
+                continue;
+            }
             if (threadIdx.x == 0)
-                s_go = wait_tile(p, tile);
+                s_go = wait_tile<SYS>(p, tile);
             __syncthreads();
             const int go = s_go;
             if (go) {
                 const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
                 for (int r = warp; r < p.B; r += kThreads / 32) {
                     const int64_t row = (int64_t)tile * p.B + r;
-                    if (__ldg(p.pool_recv_token + row) < 0)
+                    const int tok = SYS ? __ldcg(p.pool_recv_token + row) : __ldg(p.pool_recv_token + row);
+                    if (tok < 0)
                         continue;                        // padding: never read
                     const uint4 *src = reinterpret_cast<const uint4 *>(p.src) + row * vecs;
                     uint4 *dst = reinterpret_cast<uint4 *>(p.dst) + row * vecs;
@@ -141,6 +160,8 @@ __global__ void __launch_bounds__(kThreads) consume_tiles_kernel(ConsumeParams p
             __syncthreads();
             if (go && p.y_done)
                 stamp_tokens(p, tile);
+            if (SYS && go && threadIdx.x == 0)
+                p.arrival_count[tile] = 0u;              // complete: no more arrivals this step
         }
     }
 }
@@ -150,14 +171,20 @@ __global__ void __launch_bounds__(kThreads) consume_tiles_kernel(ConsumeParams p
 cudaError_t launch_consume(const ConsumeParams &p, int num_ctas, cudaStream_t s)
 {
     count_launch();
-    consume_tiles_kernel<<<num_ctas, kThreads, 0, s>>>(p);
+    if (p.arrival_count != nullptr)
+        consume_tiles_kernel<true><<<num_ctas, kThreads, 0, s>>>(p);
+    else
+        consume_tiles_kernel<false><<<num_ctas, kThreads, 0, s>>>(p);
     return cudaGetLastError();
 }
 
 cudaError_t preload_consumer_kernels()
 {
     cudaFuncAttributes a;
-    return cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(consume_tiles_kernel));
+    cudaError_t e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(consume_tiles_kernel<false>));
+    if (e == cudaSuccess)
+        e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(consume_tiles_kernel<true>));
+    return e;
 }
 
 }  // namespace sep

@@ -22,7 +22,19 @@
 // The dispatch writes each token row straight into the owner's pool through
 // the owner's pointer (a peer pointer on another GPU, plain stores over
 // NVLink; no TMA, no multicast) together with the owner's receive map
-// (token, rank, slot); the owner marks its own padding rows.  The combine
+// (token, rank, slot); the owner marks its own padding rows.
+//
+// The plan can also be computed on the GPU from the exchanged counts
+// (ep_plan_kernel), so a step needs no copy to the host.  With publication
+// (StreamEP README, "Streaming dispatch in one paragraph": the receiver counts
+// arrivals per tile and release-stores dispatch_seq at system scope once the
+// tile is complete, so the owner starts on a tile as soon as it is whole) a
+// warp owns whole rows; after its stores it fences at system scope, and lane j
+// adds one arrival to its row's tile in the owner's memory (atom.add.acq_rel
+// .sys); the arrival that reaches the tile's valid-row count (from N_e and the
+// expert's first tile, both from the plan) release-stores seq into the
+// owner's tile_ready (st.release.sys).  The owner's consumer acquires at system
+// scope and zeroes each tile's counter after copying it.  The combine
 // gathers each token's k rows from the owners' expert-output pools the same
 // way (peer loads) and reduces them exactly as the single-GPU combine does.
 #include <cuda_bf16.h>
@@ -64,6 +76,37 @@ __device__ __forceinline__ int64_t owner_row(const P &p, int64_t a, int *owner)
     }
     *owner = o;
     return row;
+}
+
+__device__ __forceinline__ unsigned atom_add_acq_rel_sys(unsigned *ptr, unsigned v)
+{
+    unsigned old;
+    asm volatile("atom.acq_rel.sys.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(ptr), "r"(v) : "memory");
+    return old;
+}
+
+__device__ __forceinline__ void st_release_sys(unsigned *ptr, unsigned v)
+{
+    asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+}
+
+// After the warp's stores of token t's rows (whole rows: one warp per token):
+// one arrival per row on its owner tile; the arrival that completes the tile
+// publishes it.
+__device__ __forceinline__ void ep_publish_rows(const EpDispatchParams &p, int64_t a, int64_t my_row, int my_owner,
+                                                int lane)
+{
+    __threadfence_system();
+    __syncwarp();
+    if (lane < p.k && my_row >= 0) {
+        const int local = __ldg(p.src_pool_row + a);
+        const int e = __ldg(p.tile_expert + local / p.B);
+        const int tile = (int)(my_row / p.B);
+        const int left = __ldg(p.expert_rows + e) - (tile - __ldg(p.expert_tile_offset + e)) * p.B;
+        const unsigned need = (unsigned)(left < p.B ? left : p.B);
+        if (atom_add_acq_rel_sys(p.arrival_count[my_owner] + tile, 1u) + 1u == need)
+            st_release_sys(p.tile_ready[my_owner] + tile, p.seq);
+    }
 }
 
 // bf16 dispatch into the owners' pools: a work item is (token, segment).
@@ -112,6 +155,8 @@ __global__ void __launch_bounds__(kWarps * 32) ep_dispatch_kernel(EpDispatchPara
                 }
             }
         }
+        if (p.tile_ready[0] != nullptr)                  // publication: segs == 1, whole rows
+            ep_publish_rows(p, t * p.k + lane, my_row, my_owner, lane);
     }
 }
 
@@ -184,6 +229,101 @@ __global__ void __launch_bounds__(kWarps * 32) ep_dispatch_fp8_kernel(EpDispatch
                 }
             }
         }
+        if (p.tile_ready[0] != nullptr)                  // publication: segs == 1, whole rows
+            ep_publish_rows(p, t * p.k + lane, my_row, my_owner, lane);
+    }
+}
+
+// The plan on the GPU: one CTA, thread e computes expert e's totals (as the
+// host sep_ep_plan does: N_e, the rows of earlier ranks, this rank's own
+// local block offset and the owner-local global block offset), with two
+// block scans over experts (tiles of N_e, tiles of this rank's own counts).
+constexpr int kPlanThreads = 1024;
+
+__device__ __forceinline__ long long block_exclusive_scan(long long v, long long *s_warp, long long *total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    long long incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long n = __shfl_up_sync(kFullMask, incl, o);
+        if (lane >= o)
+            incl += n;
+    }
+    if (lane == 31)
+        s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const long long w = lane < (int)(blockDim.x >> 5) ? s_warp[lane] : 0;
+        long long wi = w;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long n = __shfl_up_sync(kFullMask, wi, o);
+            if (lane >= o)
+                wi += n;
+        }
+        s_warp[lane] = wi - w;
+        if (lane == 31)
+            s_warp[32] = wi;
+    }
+    __syncthreads();
+    const long long ex = s_warp[warp] + incl - v;
+    *total = s_warp[32];
+    __syncthreads();                                     // s_warp is reused by the next scan
+    return ex;
+}
+
+__global__ void __launch_bounds__(kPlanThreads) ep_plan_kernel(EpPlanParams p)
+{
+    __shared__ long long s_warp[33];
+    __shared__ long long s_gtile[kPlanThreads + 1];      // exclusive scan of tau over all experts
+    const int e = threadIdx.x;
+    const int E = p.E, R = p.R, B = p.B, El = E / R;
+    long long N = 0, before = 0, own = 0;
+    bool bad = false;
+    if (e < E) {
+        for (int r = 0; r < R; ++r) {
+            const long long c = p.all_counts[(int64_t)r * E + e];
+            bad |= c < 0;
+            if (r < p.rank)
+                before += c;
+            N += c;
+        }
+        own = p.all_counts[(int64_t)p.rank * E + e];
+    }
+    const long long tau = e < E && N > 0 ? (N + B - 1) / B : 0;
+    const long long own_tau = e < E && own > 0 ? (own + B - 1) / B : 0;
+    long long total;
+    const long long gex = block_exclusive_scan(tau, s_warp, &total);
+    s_gtile[e] = gex;
+    if (e == 0)
+        s_gtile[kPlanThreads] = total;
+    const long long loff = block_exclusive_scan(own_tau, s_warp, &total);
+    __syncthreads();
+    if (e < E) {
+        const int o = e / El;
+        const long long gboff = gex - s_gtile[o * El];  // tiles before e inside its owner's pool
+        const long long d = gboff * B + before - loff * B;
+        if (bad || N > INT32_MAX || d > INT32_MAX || d < INT32_MIN || (gboff + tau) * B > INT32_MAX)
+            atomicExch(p.error, 1u);
+        p.delta[e] = (int32_t)d;
+        if (p.expert_rows)
+            p.expert_rows[e] = (int32_t)N;
+        if (p.expert_tile_offset)
+            p.expert_tile_offset[e] = (int32_t)gboff;
+        if (o == p.rank) {
+            if (p.owner_block_offset) {
+                p.owner_block_offset[e % El] = (int32_t)gboff;
+                if (e % El == El - 1)
+                    p.owner_block_offset[El] = (int32_t)(gboff + tau);
+            }
+            if (p.owner_expert_counts)
+                p.owner_expert_counts[e % El] = (int32_t)N;
+        }
+    }
+    if (p.owner_rows && e < R) {
+        const long long end = (e + 1) * El < E ? s_gtile[(e + 1) * El] : s_gtile[kPlanThreads];
+        p.owner_rows[e] = (end - s_gtile[e * El]) * B;
     }
 }
 
@@ -285,6 +425,11 @@ __global__ void __launch_bounds__(kWarps * 32) ep_combine_kernel(EpCombineParams
 
 }  // namespace
 
+cudaError_t launch_ep_plan(const EpPlanParams &p, cudaStream_t s)
+{
+    return launch_kernel(ep_plan_kernel, dim3(1), dim3(kPlanThreads), 0, s, p);
+}
+
 cudaError_t launch_ep_dispatch(EpDispatchParams p, cudaStream_t s, int num_sms)
 {
     if (p.T == 0)
@@ -292,6 +437,10 @@ cudaError_t launch_ep_dispatch(EpDispatchParams p, cudaStream_t s, int num_sms)
     int64_t steps = 1;                                   // 128-vector steps, as the single-GPU dispatch
     split_rows(p.T, ((p.H / 8) + 127) / 128, (int64_t)num_sms * 32, 1 << 20, &p.segs, &steps);
     p.seg_len = (int)(steps * 128);
+    if (p.tile_ready[0] != nullptr) {                    // publication counts whole rows: one warp a row
+        p.segs = 1;
+        p.seg_len = p.H / 8;
+    }
     const int64_t items = p.T * p.segs;
     return launch_kernel(ep_dispatch_kernel, dim3((int)((items + kWarps - 1) / kWarps)), dim3(kWarps * 32), 0, s, p);
 }
@@ -303,6 +452,10 @@ cudaError_t launch_ep_dispatch_fp8(EpDispatchParams p, cudaStream_t s, int num_s
     int64_t steps = 1;                                   // 512-channel steps, up to 7 warps a row
     split_rows(p.T, (p.H + 511) / 512, (int64_t)num_sms * 32, 7, &p.segs, &steps);
     p.seg_len = (int)steps;
+    if (p.tile_ready[0] != nullptr) {                    // publication counts whole rows: one warp a row
+        p.segs = 1;
+        p.seg_len = (p.H + 511) / 512;
+    }
     const dim3 grid((int)((p.T * p.segs + kWarps - 1) / kWarps)), block(kWarps * 32);
     switch (p.scale) {
     case SEP_SCALE_F32:
@@ -339,6 +492,8 @@ cudaError_t preload_ep_kernels()
 {
     cudaFuncAttributes a;
     cudaError_t e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(ep_dispatch_kernel));
+    if (e == cudaSuccess)
+        e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(ep_plan_kernel));
     if (e == cudaSuccess)
         e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(ep_mark_padding_kernel));
     if (e == cudaSuccess)

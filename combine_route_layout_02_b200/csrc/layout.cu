@@ -28,6 +28,9 @@
 //           plus the number of lower lanes holding that expert.  Also writes
 //           the tile tables and marks padding rows, experts spread over CTAs.
 // The result is the unique stable order and needs no atomics on the data path.
+#include <atomic>
+
+#include "fp8_quant.cuh"
 #include "sep_internal.cuh"
 
 namespace sep {
@@ -377,13 +380,13 @@ __device__ __forceinline__ uint64_t global_ns()
 // 2^32 is a multiple of the window, so the counter may wrap.
 constexpr unsigned kBarrierWindow = 4096;
 
-// All CTAs arrive on *counter; false (in every thread of the CTA) if the
+// CTAs 0..G-1 arrive on *counter; false (in every thread of the CTA) if the
 // window did not fill within the limit.
-__device__ __forceinline__ bool grid_barrier(const LayoutParams &p, unsigned *counter, int *s_flag)
+__device__ __forceinline__ bool grid_barrier(const LayoutParams &p, unsigned *counter, int *s_flag, int c, int G)
 {
     __syncthreads();
     if (threadIdx.x == 0) {
-        const unsigned add = blockIdx.x == 0 ? kBarrierWindow - (gridDim.x - 1) : 1u;
+        const unsigned add = c == 0 ? kBarrierWindow - (unsigned)(G - 1) : 1u;
         unsigned old;
         asm volatile("atom.release.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(counter), "r"(add) : "memory");
         const unsigned target = (old & ~(kBarrierWindow - 1)) + kBarrierWindow;
@@ -411,12 +414,13 @@ constexpr int64_t kSingleCtaMaxNa = 1024;     // routings this small run as one 
 constexpr int kFusedThreads = kWarps * 32;
 constexpr int kRedInts = 1024;               // per reduction table: row groups x padded experts
 
+// Chunk c of the G = p.num_wchunks chunks of the layout, run by one CTA
+// (phases A to D above).  sm: the dynamic shared memory of
+// layout_smem_bytes(); false if its grid barrier gave up.
 template <typename IdxT>
-__global__ void __launch_bounds__(kFusedThreads) layout_fused_kernel(LayoutParams p)
+__device__ bool layout_chunk(const LayoutParams &p, const int c, const int G, int32_t *sm, int &s_flag,
+                             int *s_part)
 {
-    extern __shared__ __align__(16) int32_t sm[];
-    __shared__ int s_flag;
-    __shared__ int s_part[kWarps];
     const int E = p.E, nc = p.num_wchunks;
     const int hs = (E + 3) & ~3;                         // padded row stride of the chunk table
     int32_t *s_red = sm;                                 // [2][kRedInts], read and written as int4: first
@@ -426,9 +430,7 @@ __global__ void __launch_bounds__(kFusedThreads) layout_fused_kernel(LayoutParam
     int32_t *s_pre = s_tot + E;                          // [E]
     int32_t *s_own = s_pre + E;                          // [R]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = blockIdx.x, G = gridDim.x;
     const IdxT *idx = static_cast<const IdxT *>(p.topk_idx);
-    allow_dependents();
     unsigned *counter = p.barrier_words;
     if (c == 0)
         for (int r = tid; r < p.R; r += blockDim.x)
@@ -465,8 +467,8 @@ __global__ void __launch_bounds__(kFusedThreads) layout_fused_kernel(LayoutParam
         }
         p.wchunk_hist[(int64_t)c * hs + e] = sum;
     }
-    if (!grid_barrier(p, counter, &s_flag))
-        return;
+    if (!grid_barrier(p, counter, &s_flag, c, G))
+        return false;
 
     // B. totals and this chunk's prefix, from the whole table
     {
@@ -652,6 +654,244 @@ __global__ void __launch_bounds__(kFusedThreads) layout_fused_kernel(LayoutParam
             if (s_own[r])
                 atomicAdd(&p.owner_token_counts[r], s_own[r]);
     }
+    return true;
+}
+
+size_t layout_smem_bytes(const LayoutParams &p)
+{
+    return (size_t)(kWarps * p.E + 3 * p.E + 1 + 2 * kRedInts + p.R) * sizeof(int32_t);
+}
+
+template <typename IdxT>
+__global__ void __launch_bounds__(kFusedThreads) layout_fused_kernel(LayoutParams p)
+{
+    extern __shared__ __align__(16) int32_t sm[];
+    __shared__ int s_flag;
+    __shared__ int s_part[kWarps];
+    allow_dependents();
+    layout_chunk<IdxT>(p, blockIdx.x, gridDim.x, sm, s_flag, s_part);
+}
+
+// ------------------------------------------- layout and dispatch, one launch
+//
+// For small routings (a decode step): one cooperative launch runs the layout
+// in its first nc = num_wchunks CTAs (exactly as above, its grid barrier among
+// those CTAs) and the dispatch in the other CTAs.  A dispatch warp loads its
+// items of x, and for FP8 quantises them, into registers while the layout is
+// still running; it then waits for the layout and stores the items to the
+// token's pool rows.  Items: one 16-byte vector per lane of a 32-vector step
+// of a bf16 row, or 16 channels per lane of a 512-channel step of an FP8 row
+// (the quantisation of the separate FP8 dispatch kernel, shared through
+// fp8_quant.cuh), at most kLdMaxItems per warp.
+//
+// The wait is on barrier_words[kDoneWord], a counter that is never reset.  Every CTA
+// arrives once on entry and every layout CTA once more when its chunk is
+// written; CTA 0's entry adds kBarrierWindow - (G - 1) - nc, so one launch
+// moves the counter by exactly one window, every entry arrival learns the
+// launch's window from the old value it returns, and the layout is complete
+// when the counter reaches the window's end.  As with the layout's own
+// barrier, nothing depends on host state, so a CUDA graph may replay the
+// launch.  The waits are bounded (%globaltimer and a poll budget); one that
+// gives up records the epoch in the handle's timeout word and its CTA stores
+// nothing.  Every arrival is unconditional, so the counter stays on its
+// window grid whatever happens.
+
+constexpr int kLdMaxItems = 4;
+constexpr int kLdItemsPerWarp = 2;   // preferred items per warp when the grid fits
+constexpr unsigned kDonePollNs = 256;
+
+__device__ __forceinline__ unsigned atom_add_release_u32(unsigned *ptr, unsigned v)
+{
+    unsigned old;
+    asm volatile("atom.release.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(ptr), "r"(v) : "memory");
+    return old;
+}
+
+__device__ __forceinline__ uint4 ld_nc_v4(const uint4 *ptr)
+{
+    uint4 v;
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+        : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+        : "l"(ptr));
+    return v;
+}
+
+// SCALE: SEP_SCALE_NONE for the bf16 payload, else the FP8 scale format.
+template <typename IdxT, int SCALE>
+__global__ void __launch_bounds__(kFusedThreads) layout_dispatch_kernel(LayoutParams p, DispatchParams d)
+{
+    extern __shared__ __align__(16) int32_t sm[];
+    __shared__ int s_flag;
+    __shared__ int s_part[kWarps];
+    __shared__ unsigned s_base;
+    allow_dependents();
+    const int c = blockIdx.x, G = gridDim.x, nc = p.num_wchunks;
+    unsigned *done = p.barrier_words + kDoneWord;
+    if (threadIdx.x == 0) {
+        const unsigned add = c == 0 ? kBarrierWindow - (unsigned)(G - 1) - (unsigned)nc : 1u;
+        s_base = atom_add_release_u32(done, add) & ~(kBarrierWindow - 1);
+    }
+    if (c < nc) {
+        layout_chunk<IdxT>(p, c, nc, sm, s_flag, s_part);
+        __syncthreads();                                 // every thread's layout writes precede the arrival
+        if (threadIdx.x == 0) {
+            __threadfence();
+            atom_add_release_u32(done, 1u);
+        }
+        return;
+    }
+
+    constexpr bool FP8 = SCALE != SEP_SCALE_NONE;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int H = d.H, V = H / 8, G8 = H / 128;
+    const int per_row = FP8 ? (H + 511) / 512 : (V + 31) / 32;
+    const int64_t items = d.T * per_row;
+    const int64_t nw = (int64_t)(G - nc) * kWarps;
+    const int64_t gw = (int64_t)(c - nc) * kWarps + warp;
+    uint4 val[kLdMaxItems];
+    float sf[kLdMaxItems];
+    int ex[kLdMaxItems];
+#pragma unroll
+    for (int m = 0; m < kLdMaxItems; ++m) {
+        const int64_t it = gw + m * nw;
+        val[m] = make_uint4(0u, 0u, 0u, 0u);
+        sf[m] = 1.f;
+        ex[m] = 0;
+        if (it < items) {                                // warp-uniform
+            const int64_t t = it / per_row;
+            const int st = (int)(it - t * per_row);
+            if (!FP8) {
+                const int v = st * 32 + lane;
+                if (v < V)
+                    val[m] = ld_nc_v4(static_cast<const uint4 *>(d.x) + t * V + v);
+            } else {
+                const int c0 = st * 512 + lane * 16;
+                float f[16];
+                if (c0 < H) {
+                    const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(d.x) +
+                                                                       t * H + c0);
+                    bf16x8_to_f32(ld_nc_v4(src), f);
+                    bf16x8_to_f32(ld_nc_v4(src + 1), f + 8);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q)
+                        f[q] = 0.f;
+                }
+                val[m] = quantize_lane16<FP8 ? SCALE : SEP_SCALE_F32>(f, sf[m], ex[m]);
+            }
+        }
+    }
+
+    // wait for every layout CTA (bounded)
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned target = s_base + kBarrierWindow;
+        bool ok = false;
+        const uint64_t t0 = global_ns();
+        for (uint32_t n = 0; n < (1u << 22); ++n) {
+            if ((int)(ld_acquire_u32(done) - target) >= 0) {
+                ok = true;
+                break;
+            }
+            if (global_ns() - t0 > 200000000ull)
+                break;
+            __nanosleep(kDonePollNs);
+        }
+        if (!ok)
+            atomicMax(p.timeout_epoch, p.epoch);
+        s_flag = ok ? 1 : 0;
+    }
+    __syncthreads();
+    if (!s_flag)
+        return;
+
+#pragma unroll
+    for (int m = 0; m < kLdMaxItems; ++m) {
+        const int64_t it = gw + m * nw;
+        if (it >= items)
+            break;                                       // warp-uniform
+        const int64_t t = it / per_row;
+        const int st = (int)(it - t * per_row);
+        const int my_row = lane < d.k ? __ldcg(d.src_pool_row + t * d.k + lane) : -1;
+        for (int j = 0; j < d.k; ++j) {
+            const int row = __shfl_sync(kFullMask, my_row, j);
+            if (row < 0)
+                continue;                                // warp-uniform
+            if (!FP8) {
+                const int v = st * 32 + lane;
+                if (v < V)
+                    static_cast<uint4 *>(d.recv)[(int64_t)row * V + v] = val[m];
+            } else {
+                const int c0 = st * 512 + lane * 16;
+                if (c0 < H) {
+                    *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(d.recv) + (int64_t)row * H + c0) = val[m];
+                    if ((lane & 7) == 0) {
+                        if (SCALE == SEP_SCALE_UE8M0)
+                            static_cast<uint8_t *>(d.recv_scales)[(int64_t)row * G8 + c0 / 128] =
+                                (uint8_t)(ex[m] + 127);
+                        else
+                            static_cast<float *>(d.recv_scales)[(int64_t)row * G8 + c0 / 128] = sf[m];
+                    }
+                }
+            }
+        }
+    }
+}
+
+template <typename IdxT, int SCALE>
+cudaError_t try_layout_dispatch_t(const LayoutParams &p, const DispatchParams &d, cudaStream_t s, bool *launched)
+{
+    using K = void (*)(LayoutParams, DispatchParams);
+    const K kernel = layout_dispatch_kernel<IdxT, SCALE>;
+    static std::atomic<bool> attr_set[64] = {};
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return cudaErrorInvalidDevice;
+    if (!attr_set[dev].load(std::memory_order_acquire)) {
+        const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+        if (e != cudaSuccess)
+            return e;
+        attr_set[dev].store(true, std::memory_order_release);
+    }
+    const size_t smem = layout_smem_bytes(p);
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kFusedThreads, smem) != cudaSuccess)
+        return cudaSuccess;                              // not fused: the caller launches the two kernels
+    const int per_row = SCALE != SEP_SCALE_NONE ? (d.H + 511) / 512 : (d.H / 8 + 31) / 32;
+    const int64_t items = d.T * per_row;
+    const int64_t resident = (int64_t)per_sm * sms;
+    const int nc = p.num_wchunks;
+    // two items per warp when that fits, so more warps have stores in flight
+    int64_t ctas = (items + kLdItemsPerWarp * kWarps - 1) / (kLdItemsPerWarp * kWarps);
+    if (nc + ctas > resident)
+        ctas = (items + kLdMaxItems * kWarps - 1) / (kLdMaxItems * kWarps);
+    if (ctas < 1 || nc + ctas > resident || 2 * nc + ctas >= (int64_t)kBarrierWindow)
+        return cudaSuccess;
+    LayoutParams lp = p;
+    DispatchParams dp = d;
+    void *args[] = {&lp, &dp};
+    count_launch();
+    const cudaError_t e = cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kernel), dim3((unsigned)(nc + ctas)),
+                                                      dim3(kFusedThreads), args, smem, s);
+    if (e == cudaSuccess)
+        *launched = true;
+    return e;
+}
+
+template <typename IdxT>
+cudaError_t try_layout_dispatch_idx(const LayoutParams &p, const DispatchParams &d, int payload, cudaStream_t s,
+                                    bool *launched)
+{
+    if (payload == SEP_PAYLOAD_BF16)
+        return try_layout_dispatch_t<IdxT, SEP_SCALE_NONE>(p, d, s, launched);
+    switch (d.scale) {
+    case SEP_SCALE_F32:
+        return try_layout_dispatch_t<IdxT, SEP_SCALE_F32>(p, d, s, launched);
+    case SEP_SCALE_UE8M0:
+        return try_layout_dispatch_t<IdxT, SEP_SCALE_UE8M0>(p, d, s, launched);
+    default:
+        return try_layout_dispatch_t<IdxT, SEP_SCALE_F32_POW2>(p, d, s, launched);
+    }
 }
 
 template <typename IdxT>
@@ -659,19 +899,20 @@ cudaError_t launch_layout_t(const LayoutParams &p, cudaStream_t s)
 {
     const int chunks = p.num_wchunks;
     const size_t smem_count = (size_t)kWarps * p.E * sizeof(int32_t);
-    const size_t smem_fused = (size_t)(kWarps * p.E + 3 * p.E + 1 + 2 * kRedInts + p.R) * sizeof(int32_t);
+    const size_t smem_fused = layout_smem_bytes(p);
     if (chunks > 0) {
         // single launch when every CTA can be resident at once
-        static bool attr_set[64] = {false};                  // function attributes are per device
+        // function attributes are per device; setting one twice (two threads) is harmless
+        static std::atomic<bool> attr_set[64] = {};
         int dev = 0, sms = 0, per_sm = 0;
         if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
             return cudaErrorInvalidDevice;
-        if (!attr_set[dev]) {
+        if (!attr_set[dev].load(std::memory_order_acquire)) {
             const cudaError_t e = cudaFuncSetAttribute(layout_fused_kernel<IdxT>,
                                                        cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
             if (e != cudaSuccess)
                 return e;
-            attr_set[dev] = true;
+            attr_set[dev].store(true, std::memory_order_release);
         }
         if (
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
@@ -733,9 +974,27 @@ cudaError_t launch_layout(const LayoutParams &p, int idx_bytes, cudaStream_t s)
     return idx_bytes == 8 ? launch_layout_t<long long>(p, s) : launch_layout_t<int>(p, s);
 }
 
+cudaError_t try_layout_dispatch(const LayoutParams &p, int idx_bytes, const DispatchParams &d, int payload,
+                                cudaStream_t s, bool *launched)
+{
+    *launched = false;
+    if (p.T <= 0 || p.num_wchunks < 1 || d.tile_ready != nullptr)
+        return cudaSuccess;
+    return idx_bytes == 8 ? try_layout_dispatch_idx<long long>(p, d, payload, s, launched)
+                          : try_layout_dispatch_idx<int>(p, d, payload, s, launched);
+}
+
 cudaError_t preload_layout_kernels()
 {
-    const void *k[] = {reinterpret_cast<const void *>(layout_fused_kernel<int>),
+    const void *k[] = {reinterpret_cast<const void *>(layout_dispatch_kernel<int, SEP_SCALE_NONE>),
+                       reinterpret_cast<const void *>(layout_dispatch_kernel<int, SEP_SCALE_F32>),
+                       reinterpret_cast<const void *>(layout_dispatch_kernel<int, SEP_SCALE_UE8M0>),
+                       reinterpret_cast<const void *>(layout_dispatch_kernel<int, SEP_SCALE_F32_POW2>),
+                       reinterpret_cast<const void *>(layout_dispatch_kernel<long long, SEP_SCALE_NONE>),
+                       reinterpret_cast<const void *>(layout_dispatch_kernel<long long, SEP_SCALE_F32>),
+                       reinterpret_cast<const void *>(layout_dispatch_kernel<long long, SEP_SCALE_UE8M0>),
+                       reinterpret_cast<const void *>(layout_dispatch_kernel<long long, SEP_SCALE_F32_POW2>),
+                       reinterpret_cast<const void *>(layout_fused_kernel<int>),
                        reinterpret_cast<const void *>(layout_fused_kernel<long long>),
                        reinterpret_cast<const void *>(layout_count_kernel<int>),
                        reinterpret_cast<const void *>(layout_count_kernel<long long>),

@@ -11,7 +11,9 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
+#include <vector>
 
 #include "sep_internal.cuh"
 
@@ -86,11 +88,62 @@ size_t carve(size_t *off, size_t bytes)
     return at;
 }
 
+// Pinned host words a handle reads its layout sizes and error words into.
+// One pinned slab serves many handles, so creating a handle calls no
+// cudaMallocHost and freeing one no cudaFreeHost (which synchronises the
+// device: a free between a consumer's launch and the dispatch it waits for
+// would then stall until the consumer's wait gave up).  Slabs stay until the
+// process exits.  A slot is handed back only by sep_handle_free; the one copy
+// into it (sep_handle_sync) has completed by then, since that call waits for
+// its stream.
+class MirrorPool {
+  public:
+    int64_t *take(cudaError_t *err)
+    {
+        std::lock_guard<std::mutex> lock(mu_);
+        if (free_.empty()) {
+            void *slab = nullptr;
+            *err = cudaHostAlloc(&slab, kSlots * kSlotBytes, cudaHostAllocPortable);
+            if (*err != cudaSuccess)
+                return nullptr;
+            char *b = static_cast<char *>(slab);
+            for (int i = kSlots - 1; i >= 0; --i)
+                free_.push_back(reinterpret_cast<int64_t *>(b + (size_t)i * kSlotBytes));
+        }
+        int64_t *slot = free_.back();
+        free_.pop_back();
+        *err = cudaSuccess;
+        return slot;
+    }
+    void give(int64_t *slot)
+    {
+        std::lock_guard<std::mutex> lock(mu_);
+        free_.push_back(slot);
+    }
+
+  private:
+    static constexpr int kSlots = 2048;
+    static constexpr size_t kSlotBytes = 32;
+    std::mutex mu_;
+    std::vector<int64_t *> free_;
+};
+
+MirrorPool &mirror_pool()
+{
+    static MirrorPool pool;
+    return pool;
+}
+
 // Load all kernels on this device once (see preload_* in sep_internal.cuh).
+// Threads that create their first handles at the same time serialise here.
 sep_status preload_once(int dev)
 {
-    static bool done[64] = {false};
-    if (dev >= 0 && dev < 64 && done[dev])
+    static std::atomic<bool> done[64] = {};
+    static std::mutex mu;
+    if (dev >= 0 && dev < 64 && done[dev].load(std::memory_order_acquire))
+        return SEP_OK;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 0 && dev < 64 && done[dev].load(std::memory_order_relaxed))
         return SEP_OK;
     cudaError_t e = sep::preload_layout_kernels();
     if (e == cudaSuccess)
@@ -110,7 +163,7 @@ sep_status preload_once(int dev)
     if (e != cudaSuccess)
         return cuda_fail(e, "loading the library's kernels");
     if (dev >= 0 && dev < 64)
-        done[dev] = true;
+        done[dev].store(true, std::memory_order_release);
     return SEP_OK;
 }
 
@@ -146,7 +199,7 @@ sep_status create(int64_t T_cap, int k, int E, int R, int B, uint32_t flags, cud
     const int64_t Na1 = h->Na_cap > 0 ? h->Na_cap : 1;
     size_t off = 0;
     const size_t o_sizes = carve(&off, 32);              // {P, NT}, bad_epoch, timeout_epoch: one copy to the host
-    const size_t o_bar = carve(&off, 8);
+    const size_t o_bar = carve(&off, 256);             // two counters, 128 bytes apart (own cache lines)
     const size_t o_ec = carve(&off, (size_t)E * 4);
     const size_t o_oc = carve(&off, (size_t)R * 4);
     const size_t o_otc = carve(&off, (size_t)R * 4);
@@ -168,11 +221,11 @@ sep_status create(int64_t T_cap, int k, int E, int R, int B, uint32_t flags, cud
         delete h;
         return cuda_fail(e, "cudaMallocAsync (handle storage)");
     }
-    e = cudaMallocHost(reinterpret_cast<void **>(&h->host_mirror), 32);
-    if (e != cudaSuccess) {
+    h->host_mirror = mirror_pool().take(&e);
+    if (h->host_mirror == nullptr) {
         cudaFreeAsync(h->block, s);
         delete h;
-        return cuda_fail(e, "cudaMallocHost (handle mirror)");
+        return cuda_fail(e, "cudaHostAlloc (pinned mirror slab)");
     }
     char *b = static_cast<char *>(h->block);
     h->sizes = reinterpret_cast<int64_t *>(b + o_sizes);
@@ -194,10 +247,10 @@ sep_status create(int64_t T_cap, int k, int E, int R, int B, uint32_t flags, cud
     h->wchunk_base = reinterpret_cast<int32_t *>(b + o_base);
     h->is_token_in_rank = (flags & SEP_LAYOUT_TOKEN_IN_OWNER) ? reinterpret_cast<uint8_t *>(b + o_in) : nullptr;
     h->token_arrivals = reinterpret_cast<uint32_t *>(b + o_arr);
-    e = cudaMemsetAsync(h->sizes, 0, o_bar + 8 - o_sizes, s);   // sizes, error words, barrier counters
+    e = cudaMemsetAsync(h->sizes, 0, o_bar + 256 - o_sizes, s);   // sizes, error words, barrier counters
     if (e != cudaSuccess) {
         cudaFreeAsync(h->block, s);
-        cudaFreeHost(h->host_mirror);
+        mirror_pool().give(h->host_mirror);
         delete h;
         return cuda_fail(e, "cudaMemsetAsync (handle)");
     }
@@ -253,17 +306,17 @@ sep_status set_error(sep_status st, const char *msg)
 
 int device_sm_count()
 {
-    static int cached[64] = {0};
+    static std::atomic<int> cached[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
         return 148;
-    if (cached[dev] == 0) {
-        int n = 0;
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
             n = 148;
-        cached[dev] = n;
+        cached[dev].store(n, std::memory_order_relaxed);
     }
-    return cached[dev];
+    return n;
 }
 
 int occupancy_blocks_per_sm(const void *kernel, int threads, size_t smem)
@@ -275,6 +328,8 @@ int occupancy_blocks_per_sm(const void *kernel, int threads, size_t smem)
     };
     static Entry cache[32];
     static int used = 0;
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
     for (int i = 0; i < used; ++i)
         if (cache[i].kernel == kernel && cache[i].threads == threads)
             return cache[i].blocks;
@@ -321,9 +376,16 @@ sep_status sep_handle_create(int64_t max_tokens, int top_k, int num_experts, int
                   static_cast<cudaStream_t>(stream), handle);
 }
 
-sep_status sep_layout(const void *topk_idx, int idx_bytes, int64_t num_tokens, int top_k,
-                      int num_experts, int num_owners, int block_m, uint32_t flags, void *stream,
-                      sep_handle **handle)
+}  // extern "C"
+
+namespace {
+
+// Everything sep_layout does before its launch: argument checks, the handle
+// (created, or reused and re-armed for a new routing) and the kernel
+// parameters.  Nothing is enqueued except a new handle's allocation.
+sep_status layout_begin(const void *topk_idx, int idx_bytes, int64_t num_tokens, int top_k, int num_experts,
+                        int num_owners, int block_m, uint32_t flags, cudaStream_t s, sep_handle **handle,
+                        sep::LayoutParams *out)
 {
     if (handle == nullptr)
         return fail(SEP_ERR_INVALID_ARG, "handle in/out pointer is NULL");
@@ -338,7 +400,6 @@ sep_status sep_layout(const void *topk_idx, int idx_bytes, int64_t num_tokens, i
         return fail(SEP_ERR_INVALID_ARG, "topk_idx is NULL");
     if (topk_idx != nullptr && (reinterpret_cast<uintptr_t>(topk_idx) % idx_bytes) != 0)
         return fail(SEP_ERR_INVALID_ARG, "topk_idx is not %d-byte aligned", idx_bytes);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
 
     sep_handle *h = *handle;
     if (h != nullptr) {
@@ -397,14 +458,32 @@ sep_status sep_layout(const void *topk_idx, int idx_bytes, int64_t num_tokens, i
     p.timeout_epoch = h->timeout_epoch;
     p.barrier_words = h->barrier_words;
     p.epoch = h->epoch;
+    *handle = h;
     if (p.num_wchunks > h->wchunk_cap)
         return fail(SEP_ERR_CUDA, "internal: chunk table too small");
+    *out = p;
+    return SEP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sep_status sep_layout(const void *topk_idx, int idx_bytes, int64_t num_tokens, int top_k,
+                      int num_experts, int num_owners, int block_m, uint32_t flags, void *stream,
+                      sep_handle **handle)
+{
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    sep::LayoutParams p{};
+    sep_status st = layout_begin(topk_idx, idx_bytes, num_tokens, top_k, num_experts, num_owners, block_m, flags, s,
+                                 handle, &p);
+    if (st != SEP_OK)
+        return st;
     cudaError_t e = sep::launch_layout(p, idx_bytes, s);
     if (e != cudaSuccess)
         return cuda_fail(e, "layout launch");
-    *handle = h;
     if (flags & SEP_LAYOUT_SYNC_COUNTS)
-        return sep_handle_sync(h, stream);
+        return sep_handle_sync(*handle, stream);
     return SEP_OK;
 }
 
@@ -466,6 +545,66 @@ sep_status sep_handle_sync(sep_handle *h, void *stream)
     return SEP_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Checks of a dispatch's payload arguments against a pool that must hold
+// need_rows rows (the handle-independent part of sep_dispatch's checks).
+sep_status check_payload_args(int64_t T, const void *x, int64_t hidden, int payload, int scale, const void *recv_x,
+                              const void *recv_scales, int64_t recv_capacity_rows, int64_t need_rows, bool synced)
+{
+    if (payload != SEP_PAYLOAD_BF16 && payload != SEP_PAYLOAD_FP8_E4M3)
+        return fail(SEP_ERR_INVALID_ARG, "unknown payload %d", payload);
+    const bool fp8 = payload == SEP_PAYLOAD_FP8_E4M3;
+    if (!fp8 && scale != SEP_SCALE_NONE)
+        return fail(SEP_ERR_INVALID_ARG, "bf16 payload takes SEP_SCALE_NONE");
+    if (fp8 && scale != SEP_SCALE_F32 && scale != SEP_SCALE_UE8M0 && scale != SEP_SCALE_F32_POW2)
+        return fail(SEP_ERR_INVALID_ARG, "FP8 payload needs a scale format (got %d)", scale);
+    if (hidden < 1 || hidden > 65536 || hidden % (fp8 ? 128 : 8) != 0)
+        return fail(SEP_ERR_INVALID_ARG, "hidden must be a multiple of %d in 1..65536 (got %lld)",
+                    fp8 ? 128 : 8, (long long)hidden);
+    if (T > 0 && (x == nullptr || recv_x == nullptr))
+        return fail(SEP_ERR_INVALID_ARG, "x or recv_x is NULL");
+    if (!aligned16(x) || !aligned16(recv_x))
+        return fail(SEP_ERR_INVALID_ARG, "x and recv_x must be 16-byte aligned");
+    if (fp8) {
+        if (T > 0 && recv_scales == nullptr)
+            return fail(SEP_ERR_INVALID_ARG, "recv_scales is NULL");
+        if (scale != SEP_SCALE_UE8M0 && (reinterpret_cast<uintptr_t>(recv_scales) & 3u))
+            return fail(SEP_ERR_INVALID_ARG, "fp32 recv_scales must be 4-byte aligned");
+    }
+    if (recv_capacity_rows < need_rows)
+        return fail(SEP_ERR_CAPACITY, "recv_x holds %lld rows, the layout needs %lld%s",
+                    (long long)recv_capacity_rows, (long long)need_rows,
+                    synced ? "" : " (worst case; sync the layout for the exact size)");
+    return SEP_OK;
+}
+
+sep::DispatchParams dispatch_params(const sep_handle *h, const void *x, int64_t hidden, int scale, void *recv_x,
+                                    void *recv_scales)
+{
+    sep::DispatchParams p{};
+    p.x = x;
+    p.T = h->T;
+    p.H = (int)hidden;
+    p.k = h->k;
+    p.B = h->B;
+    p.src_pool_row = h->src_pool_row;
+    p.recv = recv_x;
+    p.recv_scales = recv_scales;
+    p.scale = scale;
+    p.pool_arrival_count = h->pool_arrival_count;
+    p.pool_arrival_target = h->pool_arrival_target;
+    p.error_epoch = h->timeout_epoch;
+    p.epoch = h->epoch;
+    return p;
+}
+
+}  // namespace
+
+extern "C" {
+
 sep_status sep_dispatch(sep_handle *h, const void *x, int64_t hidden, int payload, int scale,
                         void *recv_x, void *recv_scales, int64_t recv_capacity_rows,
                         uint32_t *tile_ready, int64_t tile_ready_len, uint32_t dispatch_seq, void *stream)
@@ -477,31 +616,10 @@ sep_status sep_dispatch(sep_handle *h, const void *x, int64_t hidden, int payloa
         st = check_not_leased(h);
     if (st != SEP_OK)
         return st;
-    if (payload != SEP_PAYLOAD_BF16 && payload != SEP_PAYLOAD_FP8_E4M3)
-        return fail(SEP_ERR_INVALID_ARG, "unknown payload %d", payload);
-    const bool fp8 = payload == SEP_PAYLOAD_FP8_E4M3;
-    if (!fp8 && scale != SEP_SCALE_NONE)
-        return fail(SEP_ERR_INVALID_ARG, "bf16 payload takes SEP_SCALE_NONE");
-    if (fp8 && scale != SEP_SCALE_F32 && scale != SEP_SCALE_UE8M0 && scale != SEP_SCALE_F32_POW2)
-        return fail(SEP_ERR_INVALID_ARG, "FP8 payload needs a scale format (got %d)", scale);
-    if (hidden < 1 || hidden > 65536 || hidden % (fp8 ? 128 : 8) != 0)
-        return fail(SEP_ERR_INVALID_ARG, "hidden must be a multiple of %d in 1..65536 (got %lld)",
-                    fp8 ? 128 : 8, (long long)hidden);
-    if (h->T > 0 && (x == nullptr || recv_x == nullptr))
-        return fail(SEP_ERR_INVALID_ARG, "x or recv_x is NULL");
-    if (!aligned16(x) || !aligned16(recv_x))
-        return fail(SEP_ERR_INVALID_ARG, "x and recv_x must be 16-byte aligned");
-    if (fp8) {
-        if (h->T > 0 && recv_scales == nullptr)
-            return fail(SEP_ERR_INVALID_ARG, "recv_scales is NULL");
-        if (scale != SEP_SCALE_UE8M0 && (reinterpret_cast<uintptr_t>(recv_scales) & 3u))
-            return fail(SEP_ERR_INVALID_ARG, "fp32 recv_scales must be 4-byte aligned");
-    }
     const int64_t need = needed_rows(h);
-    if (recv_capacity_rows < need)
-        return fail(SEP_ERR_CAPACITY, "recv_x holds %lld rows, the layout needs %lld%s",
-                    (long long)recv_capacity_rows, (long long)need,
-                    h->synced ? "" : " (worst case; sync the layout for the exact size)");
+    if ((st = check_payload_args(h->T, x, hidden, payload, scale, recv_x, recv_scales, recv_capacity_rows, need,
+                                 h->synced)) != SEP_OK)
+        return st;
     if (tile_ready != nullptr) {
         if (dispatch_seq == 0)
             return fail(SEP_ERR_INVALID_ARG, "dispatch_seq must be nonzero with tile_ready");
@@ -533,25 +651,47 @@ sep_status sep_dispatch(sep_handle *h, const void *x, int64_t hidden, int payloa
         h->arrivals_used = 1;
     }
 
-    const int num_sms = sep::device_sm_count();
-    sep::DispatchParams p{};
-    p.x = x;
-    p.T = h->T;
-    p.H = (int)hidden;
-    p.k = h->k;
-    p.B = h->B;
-    p.src_pool_row = h->src_pool_row;
-    p.recv = recv_x;
-    p.recv_scales = recv_scales;
-    p.scale = scale;
+    sep::DispatchParams p = dispatch_params(h, x, hidden, scale, recv_x, recv_scales);
     p.tile_ready = tile_ready;
-    p.pool_arrival_count = h->pool_arrival_count;
-    p.pool_arrival_target = h->pool_arrival_target;
     p.seq = dispatch_seq;
-    p.error_epoch = h->timeout_epoch;
-    p.epoch = h->epoch;
-    cudaError_t e = sep::launch_dispatch(p, payload, s, num_sms);
+    cudaError_t e = sep::launch_dispatch(p, payload, s, sep::device_sm_count());
     return e == cudaSuccess ? SEP_OK : cuda_fail(e, "dispatch launch");
+}
+
+sep_status sep_layout_dispatch(const void *topk_idx, int idx_bytes, int64_t num_tokens, int top_k,
+                               int num_experts, int num_owners, int block_m, uint32_t flags, const void *x,
+                               int64_t hidden, int payload, int scale, void *recv_x, void *recv_scales,
+                               int64_t recv_capacity_rows, void *stream, sep_handle **handle)
+{
+    // every check before anything changes: the pool must hold the worst case
+    // for num_tokens, since the exact size is known only after the layout
+    sep_status st = check_dims(num_tokens, top_k, num_experts, num_owners, block_m);
+    if (st != SEP_OK)
+        return st;
+    if ((st = check_payload_args(num_tokens, x, hidden, payload, scale, recv_x, recv_scales, recv_capacity_rows,
+                                 worst_pool_rows(num_tokens * top_k, num_experts, block_m), false)) != SEP_OK)
+        return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    sep::LayoutParams lp{};
+    if ((st = layout_begin(topk_idx, idx_bytes, num_tokens, top_k, num_experts, num_owners, block_m,
+                           flags & ~(uint32_t)SEP_LAYOUT_SYNC_COUNTS, s, handle, &lp)) != SEP_OK)
+        return st;
+    sep_handle *h = *handle;
+    h->flags = flags;
+    const sep::DispatchParams dp = dispatch_params(h, x, hidden, scale, recv_x, recv_scales);
+    bool fused = false;
+    cudaError_t e = sep::try_layout_dispatch(lp, idx_bytes, dp, payload, s, &fused);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "layout + dispatch launch");
+    if (!fused) {
+        if ((e = sep::launch_layout(lp, idx_bytes, s)) != cudaSuccess)
+            return cuda_fail(e, "layout launch");
+        if (h->T > 0 && (e = sep::launch_dispatch(dp, payload, s, sep::device_sm_count())) != cudaSuccess)
+            return cuda_fail(e, "dispatch launch");
+    }
+    if (flags & SEP_LAYOUT_SYNC_COUNTS)
+        return sep_handle_sync(h, stream);
+    return SEP_OK;
 }
 
 namespace {
@@ -1196,6 +1336,184 @@ sep_status sep_ep_mark_padding(int num_local_experts, int block_m, const int32_t
     return e == cudaSuccess ? SEP_OK : cuda_fail(e, "padding launch");
 }
 
+sep_status sep_ep_plan_device(const int32_t *all_counts, int num_ranks, int num_experts, int block_m, int rank,
+                              int32_t *delta, int64_t *owner_rows, int32_t *owner_block_offset,
+                              int32_t *owner_expert_counts, int32_t *expert_rows, int32_t *expert_tile_offset,
+                              uint32_t *error, void *stream)
+{
+    if (all_counts == nullptr || delta == nullptr || error == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "NULL all_counts, delta or error");
+    if (num_ranks < 1 || num_ranks > sep::kEpMaxRanks || num_experts < 1 || num_experts > 1024 ||
+        num_experts % num_ranks != 0)
+        return fail(SEP_ERR_INVALID_ARG, "need 1 <= num_ranks <= %d, num_experts in 1..1024 divisible by num_ranks",
+                    sep::kEpMaxRanks);
+    if (block_m < 1 || block_m > 1024)
+        return fail(SEP_ERR_INVALID_ARG, "block_m must be in 1..1024");
+    if (rank < 0 || rank >= num_ranks)
+        return fail(SEP_ERR_INVALID_ARG, "rank %d outside 0..%d", rank, num_ranks - 1);
+    if (((reinterpret_cast<uintptr_t>(all_counts) | reinterpret_cast<uintptr_t>(delta) |
+          reinterpret_cast<uintptr_t>(owner_block_offset) | reinterpret_cast<uintptr_t>(owner_expert_counts) |
+          reinterpret_cast<uintptr_t>(expert_rows) | reinterpret_cast<uintptr_t>(expert_tile_offset) |
+          reinterpret_cast<uintptr_t>(error)) & 3u) != 0 ||
+        (reinterpret_cast<uintptr_t>(owner_rows) & 7u) != 0)
+        return fail(SEP_ERR_INVALID_ARG, "misaligned array");
+    int dev = -1;
+    sep_status st = current_device(&dev);
+    if (st != SEP_OK || (st = preload_once(dev)) != SEP_OK)
+        return st;
+    sep::EpPlanParams p{};
+    p.all_counts = all_counts;
+    p.R = num_ranks;
+    p.E = num_experts;
+    p.B = block_m;
+    p.rank = rank;
+    p.delta = delta;
+    p.owner_rows = owner_rows;
+    p.owner_block_offset = owner_block_offset;
+    p.owner_expert_counts = owner_expert_counts;
+    p.expert_rows = expert_rows;
+    p.expert_tile_offset = expert_tile_offset;
+    p.error = error;
+    const cudaError_t e = sep::launch_ep_plan(p, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SEP_OK : cuda_fail(e, "expert-parallel plan launch");
+}
+
+sep_status sep_ep_dispatch_publish(const sep_handle *h, uint32_t layout_epoch, const void *x, int64_t hidden,
+                                   int rank, int payload, int scale, const int32_t *delta, void *const *pools,
+                                   void *const *scales, const int64_t *pool_rows, int32_t *const *recv_token,
+                                   int32_t *const *recv_rank, int32_t *const *recv_slot, uint32_t *const *tile_ready,
+                                   uint32_t *const *arrival_count, const int32_t *expert_rows,
+                                   const int32_t *expert_tile_offset, uint32_t dispatch_seq, uint32_t *error,
+                                   void *stream)
+{
+    EpCommon c{};
+    sep_status st = ep_common(h, layout_epoch, hidden, delta, pool_rows, error, &c);
+    if (st != SEP_OK)
+        return st;
+    if (rank < 0 || rank >= h->R)
+        return fail(SEP_ERR_INVALID_ARG, "rank %d outside 0..%d", rank, h->R - 1);
+    const bool fp8 = payload == SEP_PAYLOAD_FP8_E4M3;
+    if (payload != SEP_PAYLOAD_BF16 && !fp8)
+        return fail(SEP_ERR_INVALID_ARG, "unknown payload %d", payload);
+    if (!fp8 && scale != SEP_SCALE_NONE)
+        return fail(SEP_ERR_INVALID_ARG, "bf16 payload takes SEP_SCALE_NONE");
+    if (fp8 && (hidden % 128 != 0 ||
+                (scale != SEP_SCALE_F32 && scale != SEP_SCALE_UE8M0 && scale != SEP_SCALE_F32_POW2)))
+        return fail(SEP_ERR_INVALID_ARG, "the FP8 payload needs hidden % 128 == 0 and an fp32, UE8M0 or "
+                                         "power-of-two fp32 scale");
+    if (pools == nullptr || (fp8 && scales == nullptr) || (h->T > 0 && x == nullptr))
+        return fail(SEP_ERR_INVALID_ARG, "NULL pools, scales or x");
+    if (tile_ready == nullptr || arrival_count == nullptr || expert_rows == nullptr || expert_tile_offset == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "NULL tile_ready, arrival_count, expert_rows or expert_tile_offset");
+    if (dispatch_seq == 0)
+        return fail(SEP_ERR_INVALID_ARG, "dispatch_seq must be nonzero");
+    if (!aligned16(x) || ((reinterpret_cast<uintptr_t>(expert_rows) | reinterpret_cast<uintptr_t>(expert_tile_offset)) &
+                          3u) != 0)
+        return fail(SEP_ERR_INVALID_ARG, "x must be 16-byte aligned, expert_rows / expert_tile_offset 4-byte");
+    sep::EpDispatchParams p{};
+    p.T = c.T;
+    p.H = c.H;
+    p.k = c.k;
+    p.B = c.B;
+    p.E_loc = c.E_loc;
+    p.R = c.R;
+    p.src_pool_row = c.src_pool_row;
+    p.tile_expert = c.tile_expert;
+    p.delta = c.delta;
+    p.error = c.error;
+    memcpy(p.pool_rows, c.pool_rows, sizeof(p.pool_rows));
+    const uintptr_t scale_align = scale == SEP_SCALE_UE8M0 ? 0u : 3u;
+    for (int r = 0; r < h->R; ++r) {
+        if ((pool_rows[r] > 0 && pools[r] == nullptr) || !aligned16(pools[r]))
+            return fail(SEP_ERR_INVALID_ARG, "pools[%d] must be non-NULL (if it has rows) and 16-byte aligned", r);
+        if (fp8 && ((pool_rows[r] > 0 && scales[r] == nullptr) ||
+                    (reinterpret_cast<uintptr_t>(scales[r]) & scale_align) != 0))
+            return fail(SEP_ERR_INVALID_ARG, "scales[%d] must be non-NULL (if it has rows) and scale-size aligned", r);
+        if (tile_ready[r] == nullptr || arrival_count[r] == nullptr ||
+            ((reinterpret_cast<uintptr_t>(tile_ready[r]) | reinterpret_cast<uintptr_t>(arrival_count[r])) & 3u) != 0)
+            return fail(SEP_ERR_INVALID_ARG, "tile_ready[%d] / arrival_count[%d] must be non-NULL, 4-byte aligned", r,
+                        r);
+        p.pools[r] = pools[r];
+        p.scales[r] = fp8 ? scales[r] : nullptr;
+        p.recv_token[r] = recv_token ? recv_token[r] : nullptr;
+        p.recv_rank[r] = recv_rank ? recv_rank[r] : nullptr;
+        p.recv_slot[r] = recv_slot ? recv_slot[r] : nullptr;
+        if (((reinterpret_cast<uintptr_t>(p.recv_token[r]) | reinterpret_cast<uintptr_t>(p.recv_rank[r]) |
+              reinterpret_cast<uintptr_t>(p.recv_slot[r])) & 3u) != 0)
+            return fail(SEP_ERR_INVALID_ARG, "receive maps of rank %d must be 4-byte aligned", r);
+        p.tile_ready[r] = tile_ready[r];
+        p.arrival_count[r] = arrival_count[r];
+    }
+    p.x = x;
+    p.rank = rank;
+    p.scale = scale;
+    p.expert_rows = expert_rows;
+    p.expert_tile_offset = expert_tile_offset;
+    p.seq = dispatch_seq;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = wait_for_release(const_cast<sep_handle *>(h), s, false)) != SEP_OK)
+        return st;
+    if (h->T == 0)
+        return SEP_OK;
+    const_cast<sep_handle *>(h)->last_stream = s;
+    const int sms = sep::device_sm_count();
+    const cudaError_t e = fp8 ? sep::launch_ep_dispatch_fp8(p, s, sms) : sep::launch_ep_dispatch(p, s, sms);
+    return e == cudaSuccess ? SEP_OK : cuda_fail(e, "expert-parallel publishing dispatch launch");
+}
+
+sep_status sep_ep_consume_tiles(int num_local_experts, int block_m, const int32_t *owner_block_offset,
+                                const void *pool, const int32_t *recv_token, int64_t row_bytes, int64_t pool_rows,
+                                const uint32_t *tile_ready, uint32_t *arrival_count, uint32_t dispatch_seq,
+                                void *dst, int num_ctas, uint64_t timeout_ns, uint32_t *status, void *stream)
+{
+    if (num_local_experts < 1 || num_local_experts > 1024 || block_m < 1 || block_m > 1024)
+        return fail(SEP_ERR_INVALID_ARG, "need num_local_experts and block_m in 1..1024");
+    if (pool_rows < 0 || pool_rows > INT32_MAX)
+        return fail(SEP_ERR_INVALID_ARG, "pool_rows outside 0..2^31-1");
+    if (owner_block_offset == nullptr || tile_ready == nullptr || arrival_count == nullptr || status == nullptr ||
+        recv_token == nullptr || (pool_rows > 0 && (pool == nullptr || dst == nullptr)))
+        return fail(SEP_ERR_INVALID_ARG, "NULL owner_block_offset, tile_ready, arrival_count, status, recv_token, "
+                                         "pool or dst");
+    if (row_bytes < 16 || row_bytes % 16 != 0 || row_bytes > (1LL << 20))
+        return fail(SEP_ERR_INVALID_ARG, "row_bytes must be a multiple of 16 in 16..2^20");
+    if (!aligned16(pool) || !aligned16(dst))
+        return fail(SEP_ERR_INVALID_ARG, "pool and dst must be 16-byte aligned");
+    if (((reinterpret_cast<uintptr_t>(owner_block_offset) | reinterpret_cast<uintptr_t>(tile_ready) |
+          reinterpret_cast<uintptr_t>(arrival_count) | reinterpret_cast<uintptr_t>(status) |
+          reinterpret_cast<uintptr_t>(recv_token)) & 3u) != 0)
+        return fail(SEP_ERR_INVALID_ARG, "arrays must be 4-byte aligned");
+    if (dispatch_seq == 0)
+        return fail(SEP_ERR_INVALID_ARG, "dispatch_seq must be nonzero");
+    if (num_ctas < 1 || num_ctas > 1024)
+        return fail(SEP_ERR_INVALID_ARG, "num_ctas must be in 1..1024");
+    int dev = -1;
+    sep_status st = current_device(&dev);
+    if (st != SEP_OK || (st = preload_once(dev)) != SEP_OK)
+        return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(status, 0, 2 * sizeof(uint32_t), s);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaMemsetAsync (status)");
+    sep::ConsumeParams p{};
+    p.src = static_cast<const uint8_t *>(pool);
+    p.dst = static_cast<uint8_t *>(dst);
+    p.row_bytes = row_bytes;
+    p.E = num_local_experts;
+    p.B = block_m;
+    p.expert_pool_block_offset = owner_block_offset;
+    p.pool_recv_token = recv_token;
+    p.tile_ready = tile_ready;
+    p.seq = dispatch_seq;
+    p.timeout_ns = timeout_ns ? timeout_ns : 1000000000ull;
+    p.max_polls = poll_budget(p.timeout_ns);
+    p.status = status;
+    p.abort_flag = status;
+    p.arrival_count = arrival_count;
+    p.max_tiles = pool_rows / block_m;
+    e = sep::launch_consume(p, num_ctas, s);
+    return e == cudaSuccess ? SEP_OK : cuda_fail(e, "expert-parallel consumer launch");
+}
+
 sep_status sep_ep_combine(const sep_handle *h, uint32_t layout_epoch, const void *const *y_pools,
                           const int64_t *pool_rows, int64_t hidden, const int32_t *delta, const float *topk_weight,
                           void *out, uint32_t *error, void *stream)
@@ -1295,12 +1613,19 @@ void sep_handle_free(sep_handle *h)
     const bool switched = cudaGetDevice(&prev) == cudaSuccess && prev != h->device &&
                           cudaSetDevice(h->device) == cudaSuccess;
     // consumers of the last borrowed view still read the row map: the free
-    // waits for the streams its release recorded
-    wait_for_release(h, h->last_stream, true);
+    // waits for the streams its release recorded; if that ordering cannot be
+    // enqueued, the host waits for those consumers instead
+    if (wait_for_release(h, h->last_stream, false) != SEP_OK) {
+        for (int i = 0; i < h->n_release; ++i)
+            cudaEventSynchronize(h->release_events[i]);
+        fail(SEP_ERR_CUDA, "sep_handle_free: could not order the free after the view's consumers on the stream; "
+                           "waited for them on the host");
+    }
+    h->n_release = 0;
     if (h->block != nullptr)
         cudaFreeAsync(h->block, h->last_stream);
     if (h->host_mirror != nullptr)
-        cudaFreeHost(h->host_mirror);
+        mirror_pool().give(h->host_mirror);
     for (int i = 0; i < h->release_events_made; ++i)
         cudaEventDestroy(h->release_events[i]);
     if (switched)

@@ -32,6 +32,11 @@ inline void split_rows(int64_t rows, int64_t units, int64_t want_warps, int64_t 
 // CTA chunks of the assignment stream: CTA c of the count / assign kernels
 // owns assignments [c * 256 * rounds, (c + 1) * 256 * rounds), and its warp w
 // the contiguous run of 32 * rounds entries starting at w * 32 * rounds.
+// Index of the one-launch layout + dispatch's completion counter in
+// barrier_words: 128 bytes from the grid barrier's, so that the dispatch CTAs
+// polling it do not contend for the barrier's cache line.
+constexpr int kDoneWord = 32;
+
 struct LayoutParams {
     const void *topk_idx;
     int64_t T;
@@ -56,7 +61,8 @@ struct LayoutParams {
     int64_t *sizes;                  // [2] = {P, NT}
     uint32_t *bad_epoch;             // last epoch that met an id >= E
     uint32_t *timeout_epoch;         // last epoch whose grid barrier gave up
-    uint32_t *barrier_words;         // [2]: [0] the grid barrier's arrival counter (never reset)
+    uint32_t *barrier_words;         // [64]: [0] the grid barrier's arrival counter, [kDoneWord] the
+                                     // one-launch layout + dispatch's completion counter (never reset)
     uint32_t epoch;
 };
 
@@ -88,6 +94,12 @@ struct DispatchParams {
 };
 
 cudaError_t launch_dispatch(DispatchParams p, int payload, cudaStream_t s, int num_sms);
+
+// Layout and dispatch in one cooperative launch when the routing is small
+// enough for every dispatch item to sit in registers while the layout runs;
+// *launched = false (and nothing enqueued) when it is not.
+cudaError_t try_layout_dispatch(const LayoutParams &p, int idx_bytes, const DispatchParams &d, int payload,
+                                cudaStream_t s, bool *launched);
 
 // -------------------------------------------------------- backward pair
 
@@ -173,7 +185,30 @@ struct EpDispatchParams {
     // FP8 payload (pools hold e4m3 codes): owners' scale arrays [rows][H/128]
     int scale;                       // sep_scale
     void *scales[kEpMaxRanks];
+    // per-tile publication into the owners' memory (tile_ready[0] != nullptr):
+    // a row's arrival on its owner tile, and the arrival that completes the
+    // tile release-stores seq into the owner's tile_ready (system scope)
+    uint32_t *tile_ready[kEpMaxRanks];
+    uint32_t *arrival_count[kEpMaxRanks];
+    const int32_t *expert_rows;       // [E] N_e over all ranks
+    const int32_t *expert_tile_offset;  // [E] first tile of expert e in its owner's pool
+    uint32_t seq;
 };
+
+// Device-side plan of an expert-parallel step (the host sep_ep_plan, on the GPU).
+struct EpPlanParams {
+    const int32_t *all_counts;       // [R][E]
+    int R, E, B, rank;
+    int32_t *delta;                  // [E]
+    int64_t *owner_rows;             // [R] or nullptr
+    int32_t *owner_block_offset;     // [E/R + 1] or nullptr
+    int32_t *owner_expert_counts;    // [E/R] or nullptr
+    int32_t *expert_rows;            // [E] or nullptr
+    int32_t *expert_tile_offset;     // [E] or nullptr
+    uint32_t *error;                 // set to 1 for a negative count or rows beyond 32 bits
+};
+
+cudaError_t launch_ep_plan(const EpPlanParams &p, cudaStream_t s);
 
 struct EpPaddingParams {
     int E_loc, B;
@@ -224,6 +259,11 @@ struct ConsumeParams {
     const int32_t *src_pool_row;     // [T][k]
     int k;
     uint32_t done_seq;
+    // an expert-parallel owner's pool (arrival_count != nullptr): flags are
+    // acquired at system scope, the receive map is read through L2, and each
+    // consumed tile's arrival counter is zeroed for the next step
+    uint32_t *arrival_count;
+    int64_t max_tiles;               // tiles the owner's arrays hold; a tile past them is refused
 };
 
 cudaError_t launch_consume(const ConsumeParams &p, int num_ctas, cudaStream_t s);

@@ -77,6 +77,8 @@ _SIGNATURES = [
     ("sep_dispatch_borrow", _i32, [_P, _P, _i64, _i32, ctypes.POINTER(RecvView)]),
     ("sep_view_release", _i32, [_P, ctypes.POINTER(_P), _i32]),
     ("sep_gather_rows", _i32, [ctypes.POINTER(RecvView), _P, _i64, _P]),
+    ("sep_layout_dispatch", _i32, [_P, _i32, _i64, _i32, _i32, _i32, _i32, _u32, _P, _i64, _i32, _i32, _P, _P, _i64,
+                                   _P, ctypes.POINTER(_P)]),
     ("sep_layout_noalloc", _i32, [_P, _i32, _i64, _i32, _i32, _i32, _i32, ctypes.POINTER(LayoutArrays), _P]),
     ("sep_consume_tiles_stamp", _i32, [_P, _P, _i64, _i64, _P, _i64, _u32, _P, _i32, _u64, _P, _P, _i64, _u32,
                                        _P]),
@@ -89,6 +91,10 @@ _SIGNATURES = [
     ("sep_ep_mark_padding", _i32, [_i32, _i32, _P, _P, _i64, _P, _P, _P, _P]),
     ("sep_ep_dispatch_fp8", _i32, [_P, _u32, _P, _i64, _i32, _i32, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
     ("sep_ep_combine", _i32, [_P, _u32, _P, _P, _i64, _P, _P, _P, _P, _P]),
+    ("sep_ep_plan_device", _i32, [_P, _i32, _i32, _i32, _i32, _P, _P, _P, _P, _P, _P, _P, _P]),
+    ("sep_ep_dispatch_publish", _i32, [_P, _u32, _P, _i64, _i32, _i32, _i32, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                       _P, _P, _u32, _P, _P]),
+    ("sep_ep_consume_tiles", _i32, [_i32, _i32, _P, _P, _P, _i64, _i64, _P, _P, _u32, _P, _i32, _u64, _P, _P]),
     ("sep_ep_buffer_alloc", _i32, [_i64, ctypes.POINTER(_P), _P]),
     ("sep_ep_buffer_open", _i32, [_P, ctypes.POINTER(_P)]),
     ("sep_ep_buffer_close", _i32, [_P, _i32]),
@@ -240,6 +246,27 @@ def sep_dispatch(handle: Handle, x: torch.Tensor, recv_x: torch.Tensor, payload:
                              _stream(stream)), "sep_dispatch")
 
 
+def sep_layout_dispatch(topk_idx: torch.Tensor, x: torch.Tensor, recv_x: torch.Tensor, num_experts: int,
+                        num_owners: int, block_m: int, payload: str = "bf16", scale: str = "none",
+                        recv_scales: torch.Tensor | None = None, flags: int = 0, handle: Handle | None = None,
+                        stream=None) -> Handle:
+    """Layout and dispatch of one routing in one call (one launch when the routing is small)."""
+    if topk_idx.dtype not in (torch.int32, torch.int64) or topk_idx.dim() != 2:
+        raise ValueError("topk_idx must be a [T, k] int32 or int64 tensor")
+    if x.dtype != torch.bfloat16 or x.dim() != 2:
+        raise ValueError("x must be a [T, H] bf16 tensor")
+    T, k = topk_idx.shape
+    h = handle.ptr if handle is not None else ctypes.c_void_p(None)
+    _check(_lib.sep_layout_dispatch(_ptr(topk_idx) if T else ctypes.c_void_p(None), topk_idx.element_size(),
+                                    T, k, num_experts, num_owners, block_m, flags, _ptr(x), x.shape[1],
+                                    PAYLOADS[payload], SCALES[scale], _ptr(recv_x), _ptr(recv_scales),
+                                    recv_x.shape[0], _stream(stream), ctypes.byref(h)), "sep_layout_dispatch")
+    if handle is not None:
+        handle.ptr = h
+        return handle
+    return Handle(h)
+
+
 def sep_combine(handle: Handle, y_pool: torch.Tensor, topk_weight: torch.Tensor, out: torch.Tensor,
                 layout_epoch: int | None = None, stream=None) -> None:
     if y_pool.dtype != torch.bfloat16 or out.dtype != torch.bfloat16 or topk_weight.dtype != torch.float32:
@@ -312,6 +339,72 @@ def sep_ep_dispatch_fp8(handle: Handle, x: torch.Tensor, rank: int, delta: torch
     _check(_lib.sep_ep_dispatch_fp8(handle.ptr, epoch, _ptr(x), x.shape[1], rank, SCALES[scale], _ptr(delta),
                                     _ptr_array(pools), _ptr_array(scales), rows, maps[0], maps[1], maps[2],
                                     _ptr(error), _stream(stream)), "sep_ep_dispatch_fp8")
+
+
+def sep_ep_plan_device(all_counts: torch.Tensor, rank: int, block_m: int, stream=None) -> dict:
+    """sep_ep_plan on the GPU from device counts int32 [R, E]: device tensors delta [E],
+    owner_rows [R] (int64), owner_block_offset [E/R + 1], owner_expert_counts [E/R],
+    expert_rows [E], expert_tile_offset [E] and error [1]."""
+    if all_counts.dtype != torch.int32 or all_counts.dim() != 2 or not all_counts.is_cuda:
+        raise ValueError("all_counts must be a device int32 [R, E] tensor")
+    counts = all_counts.contiguous()
+    R, E = counts.shape
+    El = E // R if R > 0 and E % R == 0 else 1
+    dev = counts.device
+    i32 = dict(dtype=torch.int32, device=dev)
+    out = dict(delta=torch.zeros(E, **i32), owner_rows=torch.zeros(R, dtype=torch.int64, device=dev),
+               owner_block_offset=torch.zeros(El + 1, **i32), owner_expert_counts=torch.zeros(El, **i32),
+               expert_rows=torch.zeros(E, **i32), expert_tile_offset=torch.zeros(E, **i32),
+               error=torch.zeros(1, **i32))
+    _check(_lib.sep_ep_plan_device(_ptr(counts), R, E, block_m, rank, _ptr(out["delta"]), _ptr(out["owner_rows"]),
+                                   _ptr(out["owner_block_offset"]), _ptr(out["owner_expert_counts"]),
+                                   _ptr(out["expert_rows"]), _ptr(out["expert_tile_offset"]), _ptr(out["error"]),
+                                   _stream(stream)), "sep_ep_plan_device")
+    return out
+
+
+def sep_ep_dispatch_publish(handle: Handle, x: torch.Tensor, rank: int, plan: dict, pools, pool_rows,
+                            tile_ready, arrival_count, dispatch_seq: int, error: torch.Tensor, payload: str = "bf16",
+                            scale: str = "none", scales=None, recv_token=None, recv_rank=None, recv_slot=None,
+                            layout_epoch: int | None = None, stream=None) -> None:
+    """This rank's rows into the owners' pools, each owner tile published (tile_ready
+    = dispatch_seq) once complete.  plan: sep_ep_plan_device's tensors."""
+    if x.dtype != torch.bfloat16:
+        raise ValueError("x must be bf16")
+    R = len(pools)
+    B = handle.info().block_m
+    for o in range(R):
+        need = -(-int(pool_rows[o]) // B)
+        if tile_ready[o].numel() < need or arrival_count[o].numel() < need or tile_ready[o].element_size() != 4 \
+                or arrival_count[o].element_size() != 4:
+            raise ValueError(f"tile_ready[{o}] / arrival_count[{o}] must hold {need} 32-bit entries")
+    rows = (ctypes.c_int64 * R)(*[int(r) for r in pool_rows])
+    maps = [None if m is None else _ptr_array(m) for m in (recv_token, recv_rank, recv_slot)]
+    epoch = handle.epoch if layout_epoch is None else layout_epoch
+    _check(_lib.sep_ep_dispatch_publish(handle.ptr, epoch, _ptr(x), x.shape[1], rank, PAYLOADS[payload],
+                                        SCALES[scale], _ptr(plan["delta"]), _ptr_array(pools),
+                                        None if scales is None else _ptr_array(scales), rows, maps[0], maps[1],
+                                        maps[2], _ptr_array(tile_ready), _ptr_array(arrival_count),
+                                        _ptr(plan["expert_rows"]), _ptr(plan["expert_tile_offset"]), dispatch_seq,
+                                        _ptr(error), _stream(stream)), "sep_ep_dispatch_publish")
+
+
+def sep_ep_consume_tiles(owner_block_offset: torch.Tensor, pool: torch.Tensor, recv_token: torch.Tensor,
+                         tile_ready: torch.Tensor, arrival_count: torch.Tensor, dispatch_seq: int, dst: torch.Tensor,
+                         status: torch.Tensor, block_m: int, num_ctas: int = 16, timeout_ns: int = 0,
+                         stream=None) -> None:
+    """Owner side: copy each published tile of pool into dst (valid rows only)."""
+    rows = pool.shape[0]
+    row_bytes = pool.shape[1] * pool.element_size()
+    if dst.shape[0] < rows or dst.shape[1] * dst.element_size() != row_bytes or recv_token.numel() < rows:
+        raise ValueError("dst and recv_token must cover the pool's rows")
+    need = rows // block_m
+    if tile_ready.numel() < need or arrival_count.numel() < need or status.numel() < 2:
+        raise ValueError("tile_ready / arrival_count must cover the pool's tiles and status hold two words")
+    _check(_lib.sep_ep_consume_tiles(owner_block_offset.numel() - 1, block_m, _ptr(owner_block_offset), _ptr(pool),
+                                     _ptr(recv_token), row_bytes, rows, _ptr(tile_ready), _ptr(arrival_count),
+                                     dispatch_seq, _ptr(dst), num_ctas, timeout_ns, _ptr(status), _stream(stream)),
+           "sep_ep_consume_tiles")
 
 
 def sep_ep_mark_padding(owner_block_offset: torch.Tensor, owner_expert_counts: torch.Tensor, block_m: int,
@@ -467,6 +560,27 @@ def sep_layout_noalloc(topk_idx: torch.Tensor, num_experts: int, num_owners: int
     if topk_idx.dtype not in (torch.int32, torch.int64) or topk_idx.dim() != 2:
         raise ValueError("topk_idx must be a [T, k] int32 or int64 tensor")
     T, k = topk_idx.shape
+    E, R = int(num_experts), int(num_owners)
+    # the C ABI sees only pointers, so every array's type and length is checked
+    # here: a short or mistyped array would be written past its end on the device
+    least = {"expert_counts": E, "owner_counts": R, "expert_pool_block_offset": E + 1,
+             "owner_pool_row_offset": R + 1, "src_pool_row": T * k, "sizes": 2, "status": 2}
+    for name, _ in LayoutArrays._fields_[:11]:
+        if name not in arrays or arrays[name] is None:
+            raise ValueError(f"sep_layout_noalloc: arrays[{name!r}] is missing")
+        a = arrays[name]
+        want = torch.int64 if name == "sizes" else torch.int32
+        if a.dtype != want:
+            raise ValueError(f"sep_layout_noalloc: {name} must be {want} (got {a.dtype})")
+        if name in least and a.numel() < least[name]:
+            raise ValueError(f"sep_layout_noalloc: {name} must hold at least {least[name]} elements "
+                             f"(got {a.numel()})")
+    for name, _ in LayoutArrays._fields_[:11]:
+        a = arrays[name]
+        if not a.is_cuda or (T and topk_idx.is_cuda and a.device != topk_idx.device):
+            raise ValueError(f"sep_layout_noalloc: {name} must be on the device of topk_idx")
+    if T and (not topk_idx.is_cuda or topk_idx.device.index != torch.cuda.current_device()):
+        raise ValueError("sep_layout_noalloc: topk_idx must be on the current CUDA device")
     la = LayoutArrays()
     for name, _ in LayoutArrays._fields_[:11]:
         setattr(la, name, _ptr(arrays[name]).value)

@@ -147,7 +147,8 @@ typedef struct sep_layout_info {
  *               num_experts, num_owners and block_m match and T fits its
  *               capacity; otherwise SEP_ERR_HANDLE_MISMATCH and nothing changes.
  * The handle's device memory is allocated stream-ordered on `stream` when it is
- * created; later layouts into it allocate nothing.  Creating the first handle
+ * created, and its pinned host words come from a process-wide pool (no
+ * cudaMallocHost per handle); later layouts into it allocate nothing.  Creating the first handle
  * on a device also loads all of the library's kernels on it (CUDA otherwise
  * loads kernels lazily, and a load may wait for running kernels, which would
  * stall a dispatch behind a consumer that is waiting for it).
@@ -212,6 +213,35 @@ SEP_API sep_status sep_dispatch(sep_handle *handle, const void *x, int64_t hidde
                         int scale, void *recv_x, void *recv_scales,
                         int64_t recv_capacity_rows, uint32_t *tile_ready,
                         int64_t tile_ready_len, uint32_t dispatch_seq, void *stream);
+
+/*
+ * sep_layout_dispatch — the layout and the dispatch of one routing in one call.
+ *
+ * The dispatch of the pages' problem statement takes the router's top-k
+ * output and the hidden states together ("DeepEP MoE dispatch/combine" blog,
+ * "一轮 DeepEP 数据流": count by destination/expert, compute the layout and
+ * offsets, move the hidden states; the low-latency article's
+ * low_latency_dispatch takes x and topk_idx in one call).  This call computes
+ * exactly what sep_layout followed by sep_dispatch (no tile_ready) computes,
+ * into the same handle, with the same arguments and errors, except:
+ *  - recv_capacity_rows must cover the worst case for num_tokens (the exact
+ *    pool size is known only after the layout), else SEP_ERR_CAPACITY and
+ *    nothing changes;
+ *  - when the routing is small enough (every dispatch item of x held in
+ *    registers by the CTAs the GPU can keep resident beside the layout's), the
+ *    two run as ONE cooperative launch: the dispatch CTAs load, and for FP8
+ *    quantise, their slices of x while the layout runs, wait for it (bounded;
+ *    a wait that gives up is reported by sep_handle_sync as SEP_ERR_TIMEOUT),
+ *    then store to the pool rows.  Otherwise the two kernels are launched one
+ *    after the other, as by the two calls.
+ * SEP_LAYOUT_SYNC_COUNTS waits for both, then reads the exact pool size.
+ * sep_launch_count tells the two cases apart (one launch or two).
+ */
+SEP_API sep_status sep_layout_dispatch(const void *topk_idx, int idx_bytes, int64_t num_tokens, int top_k,
+                               int num_experts, int num_owners, int block_m, uint32_t flags,
+                               const void *x, int64_t hidden, int payload, int scale, void *recv_x,
+                               void *recv_scales, int64_t recv_capacity_rows, void *stream,
+                               sep_handle **handle);
 
 /*
  * sep_combine — weighted top-k reduction back into token order.
@@ -521,6 +551,83 @@ SEP_API sep_status sep_ep_mark_padding(int num_local_experts, int block_m, const
                                        int32_t *recv_rank, int32_t *recv_slot, void *stream);
 
 /*
+ * sep_ep_plan_device — sep_ep_plan on the GPU: the same outputs from the same
+ * exchanged counts, computed by one kernel on `stream`, so a step needs no
+ * copy to the host (the counts can be all-gathered device to device).
+ *
+ *  all_counts           device int32 [num_ranks, num_experts], as for sep_ep_plan.
+ *  delta, owner_rows (int64 [num_ranks]), owner_block_offset, owner_expert_counts:
+ *                       device outputs as for sep_ep_plan (the last three may be NULL).
+ *  expert_rows          device int32 [num_experts] or NULL, out: N_e, every rank's
+ *                       assignments of expert e (the owner's valid rows of e).
+ *  expert_tile_offset   device int32 [num_experts] or NULL, out: the first tile of
+ *                       expert e in its owner's pool.  With expert_rows, what a
+ *                       publishing dispatch needs to know when a tile is complete.
+ *  error                device uint32, set to 1 (never cleared) for a negative
+ *                       count or a pool beyond 32-bit rows; the outputs are then
+ *                       not to be used.
+ * num_ranks <= 64 (the expert-parallel kernels' limit), num_experts <= 1024.
+ */
+SEP_API sep_status sep_ep_plan_device(const int32_t *all_counts, int num_ranks, int num_experts, int block_m,
+                                      int rank, int32_t *delta, int64_t *owner_rows, int32_t *owner_block_offset,
+                                      int32_t *owner_expert_counts, int32_t *expert_rows,
+                                      int32_t *expert_tile_offset, uint32_t *error, void *stream);
+
+/*
+ * sep_ep_dispatch_publish — sep_ep_dispatch (payload SEP_PAYLOAD_BF16, scale
+ * SEP_SCALE_NONE, scales NULL) or sep_ep_dispatch_fp8 (SEP_PAYLOAD_FP8_E4M3),
+ * that also publishes every owner tile as soon as it is complete (StreamEP
+ * README, "Streaming dispatch in one paragraph": arrivals counted per tile on
+ * the receiver, dispatch_seq release-stored at system scope by the arrival
+ * that completes the tile).  A warp writes whole rows; after its stores it
+ * fences at system scope and adds one arrival per row to
+ * arrival_count[owner][tile] (atom.add.acq_rel.sys); the arrival that reaches
+ * the tile's valid rows (from expert_rows and expert_tile_offset of
+ * sep_ep_plan_device) stores dispatch_seq into tile_ready[owner][tile]
+ * (st.release.sys).  No load with multicast, no TMA: plain peer stores and
+ * atomics.
+ *
+ *  tile_ready, arrival_count  host arrays [R] of device uint32 arrays in the
+ *                       owners' memory (peer pointers), each of at least
+ *                       ceil(pool_rows[o] / block_m) entries.  Every counter
+ *                       must be zero when the group's dispatches start:
+ *                       allocate them zeroed; sep_ep_consume_tiles zeroes each
+ *                       tile it consumes.
+ *  dispatch_seq         nonzero, advancing (mod 2^32) per step of the group.
+ * Other arguments and errors as sep_ep_dispatch / sep_ep_dispatch_fp8.
+ */
+SEP_API sep_status sep_ep_dispatch_publish(const sep_handle *handle, uint32_t layout_epoch, const void *x,
+                                           int64_t hidden, int rank, int payload, int scale, const int32_t *delta,
+                                           void *const *pools, void *const *scales, const int64_t *pool_rows,
+                                           int32_t *const *recv_token, int32_t *const *recv_rank,
+                                           int32_t *const *recv_slot, uint32_t *const *tile_ready,
+                                           uint32_t *const *arrival_count, const int32_t *expert_rows,
+                                           const int32_t *expert_tile_offset, uint32_t dispatch_seq,
+                                           uint32_t *error, void *stream);
+
+/*
+ * sep_ep_consume_tiles — owner side: the reference consumer of a publishing
+ * dispatch (a stand-in for the owner's expert compute).  Persistent CTAs walk
+ * the owner's tiles (from owner_block_offset of sep_ep_plan_device, device
+ * [E_loc + 1]); thread 0 acquire-loads tile_ready[tile] at system scope
+ * until it reaches dispatch_seq, bounded by timeout_ns (0: 1 s) and a poll
+ * budget; the CTA then copies the tile's valid rows (recv_token >= 0, read
+ * through L2) from pool to dst and zeroes arrival_count[tile] for the next
+ * step.  status (device uint32 [2]) = {SEP_OK or SEP_ERR_TIMEOUT, tiles not
+ * copied}; a tile beyond pool_rows / block_m (a plan larger than the owner's
+ * arrays) is not touched and gives SEP_ERR_CAPACITY.  After a timeout the
+ * group must zero the arrival counters before its next step.  Launch it after
+ * the dispatches it waits for are enqueued on their GPUs, or before them on
+ * another GPU; never wait on a dispatch that another process launches on the
+ * same GPU (nothing guarantees the two kernels run at the same time).
+ */
+SEP_API sep_status sep_ep_consume_tiles(int num_local_experts, int block_m, const int32_t *owner_block_offset,
+                                        const void *pool, const int32_t *recv_token, int64_t row_bytes,
+                                        int64_t pool_rows, const uint32_t *tile_ready, uint32_t *arrival_count,
+                                        uint32_t dispatch_seq, void *dst, int num_ctas, uint64_t timeout_ns,
+                                        uint32_t *status, void *stream);
+
+/*
  * sep_ep_combine — out[t] = bf16( sum over valid j, ascending, of
  * topk_weight[t, j] * y_pools[owner][row(t, j)] ) with fp32 products and sums:
  * sep_combine over the owners' expert-output pools (host array [R] of device
@@ -554,8 +661,14 @@ SEP_API sep_status sep_ep_buffer_close(void *ptr, int opened);
 /* Frees the handle.  Its device memory is released stream-ordered on the
  * stream of the last call that used it, after the streams the last
  * sep_view_release named; the caller must have ordered every other stream
- * that used the handle before that point.  NULL is a no-op; a handle with an
- * active borrowed view is not freed (release the view first). */
+ * that used the handle before that point.  The call does not wait for the
+ * device: its pinned host words go back to a process-wide pool (no
+ * cudaFreeHost), so a free between a consumer's launch and the dispatch it
+ * waits for does not stall.  If the wait on the view's consumers cannot be
+ * enqueued, the host waits for them instead and sep_last_error says so.
+ * NULL is a no-op; a handle with an active borrowed view is not freed
+ * (release the view first).  Handles may be created and freed from several
+ * host threads at once. */
 SEP_API void sep_handle_free(sep_handle *handle);
 
 /* Message for the calling thread's last failed call ("" if none). */

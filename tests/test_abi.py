@@ -23,7 +23,7 @@ def test_library_is_built_for_sm100a_and_in_tree():
 
 def test_exports_match_header():
     declared = sep.declared_entry_points(HEADER)
-    assert len(declared) == 29
+    assert len(declared) == 33
     out = subprocess.run(["nm", "-D", "--defined-only", sep.library_path()], capture_output=True,
                          text=True, check=True).stdout
     exported = sorted(set(re.findall(r"\sT\s+(sep_\w+)$", out, flags=re.M)))
@@ -131,3 +131,25 @@ def test_host_tensors_are_refused_not_computed():
         sep.sep_dispatch(h, x, pool)
     with pytest.raises(ValueError, match="device tensors"):
         sep.sep_combine(h, pool, torch.zeros(4, 2), torch.zeros(4, 16, dtype=torch.bfloat16), layout_epoch=1)
+
+
+def test_layout_dispatch_rejects_bad_arguments_before_any_cuda_call():
+    """Every check of sep_layout_dispatch comes before the handle is created or
+    changed: the capacity against the worst case for num_tokens (4 tokens x 2
+    over 8 experts with BLOCK_M 16 need 8 + 8 * 15 = 128 rows), the payload,
+    the hidden size and the alignment."""
+    lib = sep.library()
+    h = ctypes.c_void_p(None)
+
+    def call(cap, payload=0, scale=0, hidden=16, x=16, recv=16, k=2):
+        return lib.sep_layout_dispatch(ctypes.c_void_p(16), 4, 4, k, 8, 2, 16, 0, ctypes.c_void_p(x), hidden,
+                                       payload, scale, ctypes.c_void_p(recv), None, cap, None, ctypes.byref(h))
+
+    assert call(127) == sep.SEP_ERR_CAPACITY
+    assert "128" in lib.sep_last_error().decode()
+    assert call(1 << 20, payload=5) == sep.SEP_ERR_INVALID_ARG
+    assert call(1 << 20, payload=1, scale=0) == sep.SEP_ERR_INVALID_ARG
+    assert call(1 << 20, hidden=12) == sep.SEP_ERR_INVALID_ARG
+    assert call(1 << 20, x=8) == sep.SEP_ERR_INVALID_ARG
+    assert call(1 << 20, k=0) == sep.SEP_ERR_INVALID_ARG
+    assert not h.value
