@@ -68,8 +68,8 @@ def parse_args(argv=None):
     ap.add_argument("--extras", default="borrowed,backward,gate,scatter,ep",
                     help="comma list of the measurements taken after the timed region")
     ap.add_argument("--profile-case", default=None,
-                    choices=["layout", "layout_dispatch", "dispatch", "combine", "consumer", "gated", "gather",
-                             "scatter", "backward", "ep"],
+                    choices=["layout", "layout_dispatch", "one_launch", "dispatch", "combine", "consumer", "gated",
+                             "gather", "scatter", "backward", "ep"],
                     help="run one kernel family a few times, its producers finished first (for ncu); no timing")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the borrowed-receive, backward-pair, combine-gate and scatter-combine measurements")
@@ -1102,9 +1102,10 @@ def profile_case(args) -> int:
         for _ in range(n):
             if case == "layout":
                 sep.sep_layout(idx, w.E, w.R, w.B, handle=h)
-            elif case == "layout_dispatch":
+            elif case in ("layout_dispatch", "one_launch"):
                 sep.sep_layout_dispatch(idx, x, recv, w.E, w.R, w.B, payload=w.payload, scale=w.scale,
-                                        recv_scales=scales, handle=h)
+                                        recv_scales=scales, handle=h,
+                                        flags=sep.SEP_LAYOUT_ONE_LAUNCH if case == "one_launch" else 0)
             elif case == "dispatch":
                 sep.sep_dispatch(h, x, recv, payload=w.payload, scale=w.scale, recv_scales=scales)
             elif case == "combine":

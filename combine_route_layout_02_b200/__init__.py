@@ -14,5 +14,5 @@ from .sep import (  # noqa: F401
     sep_ep_plan_device, sep_ep_dispatch_publish, sep_ep_consume_tiles,
     SharedBuffer, sep_ep_buffer_alloc, sep_ep_buffer_open, sep_consume_tiles_stamp, sep_dispatch_grads,
     SEP_OK, SEP_ERR_INVALID_ARG, SEP_ERR_CAPACITY, SEP_ERR_BAD_EXPERT_ID, SEP_ERR_HANDLE_MISMATCH,
-    SEP_ERR_TIMEOUT, SEP_ERR_CUDA, SEP_LAYOUT_SYNC_COUNTS, SEP_LAYOUT_TOKEN_IN_OWNER,
+    SEP_ERR_TIMEOUT, SEP_ERR_CUDA, SEP_LAYOUT_SYNC_COUNTS, SEP_LAYOUT_TOKEN_IN_OWNER, SEP_LAYOUT_ONE_LAUNCH,
 )

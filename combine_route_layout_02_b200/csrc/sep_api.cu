@@ -672,6 +672,8 @@ sep_status sep_layout_dispatch(const void *topk_idx, int idx_bytes, int64_t num_
                                  worst_pool_rows(num_tokens * top_k, num_experts, block_m), false)) != SEP_OK)
         return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool one_launch = (flags & SEP_LAYOUT_ONE_LAUNCH) != 0;
+    flags &= ~(uint32_t)SEP_LAYOUT_ONE_LAUNCH;
     sep::LayoutParams lp{};
     if ((st = layout_begin(topk_idx, idx_bytes, num_tokens, top_k, num_experts, num_owners, block_m,
                            flags & ~(uint32_t)SEP_LAYOUT_SYNC_COUNTS, s, handle, &lp)) != SEP_OK)
@@ -680,7 +682,7 @@ sep_status sep_layout_dispatch(const void *topk_idx, int idx_bytes, int64_t num_
     h->flags = flags;
     const sep::DispatchParams dp = dispatch_params(h, x, hidden, scale, recv_x, recv_scales);
     bool fused = false;
-    cudaError_t e = sep::try_layout_dispatch(lp, idx_bytes, dp, payload, s, &fused);
+    cudaError_t e = one_launch ? sep::try_layout_dispatch(lp, idx_bytes, dp, payload, s, &fused) : cudaSuccess;
     if (e != cudaSuccess)
         return cuda_fail(e, "layout + dispatch launch");
     if (!fused) {

@@ -20,7 +20,7 @@ SEP_OK, SEP_ERR_INVALID_ARG, SEP_ERR_CAPACITY, SEP_ERR_BAD_EXPERT_ID = 0, 1, 2, 
 SEP_ERR_HANDLE_MISMATCH, SEP_ERR_TIMEOUT, SEP_ERR_CUDA = 4, 5, 6
 SEP_PAYLOAD_BF16, SEP_PAYLOAD_FP8_E4M3 = 0, 1
 SEP_SCALE_NONE, SEP_SCALE_F32, SEP_SCALE_UE8M0, SEP_SCALE_F32_POW2 = 0, 1, 2, 3
-SEP_LAYOUT_SYNC_COUNTS, SEP_LAYOUT_TOKEN_IN_OWNER = 0x1, 0x2
+SEP_LAYOUT_SYNC_COUNTS, SEP_LAYOUT_TOKEN_IN_OWNER, SEP_LAYOUT_ONE_LAUNCH = 0x1, 0x2, 0x4
 
 PAYLOADS = {"bf16": SEP_PAYLOAD_BF16, "fp8": SEP_PAYLOAD_FP8_E4M3}
 SCALES = {"none": SEP_SCALE_NONE, "f32": SEP_SCALE_F32, "ue8m0": SEP_SCALE_UE8M0,
@@ -250,7 +250,8 @@ def sep_layout_dispatch(topk_idx: torch.Tensor, x: torch.Tensor, recv_x: torch.T
                         num_owners: int, block_m: int, payload: str = "bf16", scale: str = "none",
                         recv_scales: torch.Tensor | None = None, flags: int = 0, handle: Handle | None = None,
                         stream=None) -> Handle:
-    """Layout and dispatch of one routing in one call (one launch when the routing is small)."""
+    """Layout and dispatch of one routing in one call (flags SEP_LAYOUT_ONE_LAUNCH: one
+    cooperative launch when the routing is small; by default the two kernels)."""
     if topk_idx.dtype not in (torch.int32, torch.int64) or topk_idx.dim() != 2:
         raise ValueError("topk_idx must be a [T, k] int32 or int64 tensor")
     if x.dtype != torch.bfloat16 or x.dim() != 2:

@@ -90,6 +90,8 @@ typedef enum sep_scale {
                                           of PR #769) instead of the worst case */
 #define SEP_LAYOUT_TOKEN_IN_OWNER 0x2u /* also write is_token_in_rank [T, R] and
                                           owner_token_counts [R] */
+#define SEP_LAYOUT_ONE_LAUNCH    0x4u  /* sep_layout_dispatch only: run a small routing's
+                                          layout and dispatch as one cooperative launch */
 
 /* Opaque routing layout ("EPHandle" in the blog): valid only for the routing
  * that produced it (blog, "EPHandle": the handle is valid only for the routing
@@ -227,13 +229,18 @@ SEP_API sep_status sep_dispatch(sep_handle *handle, const void *x, int64_t hidde
  *  - recv_capacity_rows must cover the worst case for num_tokens (the exact
  *    pool size is known only after the layout), else SEP_ERR_CAPACITY and
  *    nothing changes;
- *  - when the routing is small enough (every dispatch item of x held in
- *    registers by the CTAs the GPU can keep resident beside the layout's), the
- *    two run as ONE cooperative launch: the dispatch CTAs load, and for FP8
- *    quantise, their slices of x while the layout runs, wait for it (bounded;
- *    a wait that gives up is reported by sep_handle_sync as SEP_ERR_TIMEOUT),
- *    then store to the pool rows.  Otherwise the two kernels are launched one
- *    after the other, as by the two calls.
+ *  - with SEP_LAYOUT_ONE_LAUNCH, when the routing is small enough (every
+ *    dispatch item of x held in registers by the CTAs the GPU can keep
+ *    resident beside the layout's), the two run as ONE cooperative launch:
+ *    the dispatch CTAs load, and for FP8 quantise, their slices of x while
+ *    the layout runs, wait for it (bounded; a wait that gives up is reported
+ *    by sep_handle_sync as SEP_ERR_TIMEOUT), then store to the pool rows.
+ *    Otherwise, and by default, the layout and dispatch kernels are launched
+ *    one after the other, as by the two calls (the dispatch with programmatic
+ *    dependent launch, resident while the layout drains).  Measured on one
+ *    B200 the one launch is not faster: decode step 27.6 us against 27.0,
+ *    graph replay 30.2 against 28.6; tiny 13.5 against 15.3 eager, 16.4
+ *    against 15.6 replayed.
  * SEP_LAYOUT_SYNC_COUNTS waits for both, then reads the exact pool size.
  * sep_launch_count tells the two cases apart (one launch or two).
  */
@@ -579,12 +586,13 @@ SEP_API sep_status sep_ep_plan_device(const int32_t *all_counts, int num_ranks, 
  * that also publishes every owner tile as soon as it is complete (StreamEP
  * README, "Streaming dispatch in one paragraph": arrivals counted per tile on
  * the receiver, dispatch_seq release-stored at system scope by the arrival
- * that completes the tile).  A warp writes whole rows; after its stores it
- * fences at system scope and adds one arrival per row to
- * arrival_count[owner][tile] (atom.add.acq_rel.sys); the arrival that reaches
- * the tile's valid rows (from expert_rows and expert_tile_offset of
- * sep_ep_plan_device) stores dispatch_seq into tile_ready[owner][tile]
- * (st.release.sys).  No load with multicast, no TMA: plain peer stores and
+ * that completes the tile).  Rows are cut into segments by the hidden size
+ * alone (2 KB bf16 steps, 512-channel FP8 steps), so every rank counts alike;
+ * after its stores a warp fences at system scope and adds one arrival per row
+ * to arrival_count[owner][tile] (atom.add.acq_rel.sys); the arrival that
+ * reaches the tile's valid rows times the segments per row (the valid rows
+ * from expert_rows and expert_tile_offset of sep_ep_plan_device) stores
+ * dispatch_seq into tile_ready[owner][tile] (st.release.sys).  No load with multicast, no TMA: plain peer stores and
  * atomics.
  *
  *  tile_ready, arrival_count  host arrays [R] of device uint32 arrays in the

@@ -3,9 +3,9 @@
 The call must compute exactly what sep_layout followed by sep_dispatch
 computes ("DeepEP MoE dispatch/combine" blog, "一轮 DeepEP 数据流": count by
 expert, lay out, move the hidden states; the low-latency article's dispatch
-takes x and topk_idx together).  Small routings run as one cooperative launch
-(layout CTAs beside dispatch CTAs that wait for them); larger ones as the two
-kernels.  Every case is compared with the oracle: the layout arrays and the
+takes x and topk_idx together).  With SEP_LAYOUT_ONE_LAUNCH small routings
+run as one cooperative launch (layout CTAs beside dispatch CTAs that wait for
+them); larger ones, and every routing by default, as the two kernels.  Every case is compared with the oracle: the layout arrays and the
 pool rows (bf16 bits, or FP8 codes and scales) bit for bit, padding rows
 untouched, and which path ran is read from sep_launch_count.
 """
@@ -55,7 +55,10 @@ def _check_pool(lay, x, recv, sc, payload, scale):
     assert (codes[P:] == POISON_U8).all()
 
 
-def _run(idx, x, E, R, B, payload="bf16", scale="none", handle=None, idx_dtype=torch.int32):
+ONE = sep.SEP_LAYOUT_ONE_LAUNCH
+
+
+def _run(idx, x, E, R, B, payload="bf16", scale="none", handle=None, idx_dtype=torch.int32, flags=ONE):
     T, k = idx.shape
     H = x.shape[1]
     worst = oracle.capacity_rows(T * k, E, B)
@@ -65,7 +68,7 @@ def _run(idx, x, E, R, B, payload="bf16", scale="none", handle=None, idx_dtype=t
     torch.cuda.synchronize()
     n0 = sep.sep_launch_count()
     h = sep.sep_layout_dispatch(idx_d, x_d, recv, E, R, B, payload=payload, scale=scale, recv_scales=sc,
-                                handle=handle)
+                                handle=handle, flags=flags)
     launches = sep.sep_launch_count() - n0
     torch.cuda.synchronize()
     lay = oracle.layout(idx.numpy(), E, R, B)
@@ -126,6 +129,21 @@ def test_duplicate_experts_and_many_experts():
     h, lay, launches, _ = _run(torch.from_numpy(idx), x, 1024, 8, 16, "bf16", "none")
     sep.sep_handle_free(h)
     assert launches == 1
+
+
+@pytest.mark.parametrize("name,payload,scale", [("decode", "fp8", "ue8m0"), ("tiny", "bf16", "none")])
+def test_two_launches_by_default(name, payload, scale):
+    w = W.WORKLOADS[name]
+    d = W.make_inputs(w)
+    h, lay, launches, _ = _run(d["topk_idx"], d["x"], w.E, w.R, w.B, payload, scale, flags=0)
+    sep.sep_handle_free(h)
+    assert launches == 2
+
+
+def test_the_one_launch_flag_is_refused_by_sep_layout():
+    idx = torch.zeros(4, 2, dtype=torch.int32, device="cuda")
+    with pytest.raises(sep.SepError, match="SEP_ERR_INVALID_ARG"):
+        sep.sep_layout(idx, 8, 2, 16, flags=sep.SEP_LAYOUT_ONE_LAUNCH)
 
 
 def test_large_routing_falls_back_to_two_launches():
@@ -204,7 +222,7 @@ def test_one_launch_step_replays_from_a_cuda_graph(name, payload, scale):
 
         def step():
             sep.sep_layout_dispatch(idx, x, recv, w.E, w.R, w.B, payload=payload, scale=scale, recv_scales=sc,
-                                    handle=h)
+                                    handle=h, flags=ONE)
             sep.sep_combine(h, y, wt, out)
 
         with torch.cuda.stream(s):
