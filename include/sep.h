@@ -586,13 +586,12 @@ SEP_API sep_status sep_ep_plan_device(const int32_t *all_counts, int num_ranks, 
  * that also publishes every owner tile as soon as it is complete (StreamEP
  * README, "Streaming dispatch in one paragraph": arrivals counted per tile on
  * the receiver, dispatch_seq release-stored at system scope by the arrival
- * that completes the tile).  Rows are cut into segments by the hidden size
- * alone (2 KB bf16 steps, 512-channel FP8 steps), so every rank counts alike;
- * after its stores a warp fences at system scope and adds one arrival per row
- * to arrival_count[owner][tile] (atom.add.acq_rel.sys); the arrival that
- * reaches the tile's valid rows times the segments per row (the valid rows
- * from expert_rows and expert_tile_offset of sep_ep_plan_device) stores
- * dispatch_seq into tile_ready[owner][tile] (st.release.sys).  No load with multicast, no TMA: plain peer stores and
+ * that completes the tile).  A warp writes whole rows; after its stores it
+ * fences at system scope and adds one arrival per row to
+ * arrival_count[owner][tile] (atom.add.acq_rel.sys); the arrival that reaches
+ * the tile's valid rows (from expert_rows and expert_tile_offset of
+ * sep_ep_plan_device) stores dispatch_seq into tile_ready[owner][tile]
+ * (st.release.sys).  No load with multicast, no TMA: plain peer stores and
  * atomics.
  *
  *  tile_ready, arrival_count  host arrays [R] of device uint32 arrays in the
