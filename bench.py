@@ -656,7 +656,11 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
            if w.streaming else {}),
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "peak_source": peaks["source"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": traffic},
+                     "traffic": traffic,
+                     # the whole step's algorithmic bytes over its time: lines a kernel leaves dirty in L2
+                     # are written back during the next one, so the step's figure is the one that
+                     # charges every byte to the time it took
+                     "step_frac": step_gbs / peaks["hbm_gbs"]},
         "e2e": {"value": world * T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "mode": e2e_mode,
                 "copies_only_ms_per_step": copies_ms or None,
