@@ -204,6 +204,8 @@ class EPGroup:
         y_is_pool the received rows themselves are the outputs (identity experts)."""
         self._barrier()                                  # every owner's outputs are written
         ys = self.pools if y_is_pool else self.ys
+        if self.signals and int(self.plan["error"].item()) != 0:
+            raise RuntimeError("the exchanged counts hold a negative count or exceed 32-bit pool rows")
         if self.signals and int(self.status[0].item()) != 0:
             raise RuntimeError(f"an owner's consumer reported {self.status.cpu().tolist()}")
         _sep.sep_ep_combine(self.handle, ys, self.rows, self.delta, topk_weight, out, self.error)
