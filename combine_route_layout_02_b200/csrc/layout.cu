@@ -417,15 +417,15 @@ constexpr int kRedInts = 1024;               // per reduction table: row groups 
 // Chunk c of the G = p.num_wchunks chunks of the layout, run by one CTA
 // (phases A to D above).  sm: the dynamic shared memory of
 // layout_smem_bytes(); false if its grid barrier gave up.
-template <typename IdxT>
+template <typename IdxT, int WARPS = kWarps>
 __device__ bool layout_chunk(const LayoutParams &p, const int c, const int G, int32_t *sm, int &s_flag,
                              int *s_part)
 {
     const int E = p.E, nc = p.num_wchunks;
     const int hs = (E + 3) & ~3;                         // padded row stride of the chunk table
     int32_t *s_red = sm;                                 // [2][kRedInts], read and written as int4: first
-    int32_t *s_cnt = s_red + 2 * kRedInts;               // [kWarps][E]
-    int32_t *s_off = s_cnt + kWarps * E;                 // [E+1]
+    int32_t *s_cnt = s_red + 2 * kRedInts;               // [WARPS][E]
+    int32_t *s_off = s_cnt + WARPS * E;                 // [E+1]
     int32_t *s_tot = s_off + E + 1;                      // [E]
     int32_t *s_pre = s_tot + E;                          // [E]
     int32_t *s_own = s_pre + E;                          // [R]
@@ -437,10 +437,10 @@ __device__ bool layout_chunk(const LayoutParams &p, const int c, const int G, in
             p.owner_token_counts[r] = 0;
 
     // A. count
-    for (int i = tid; i < kWarps * E; i += blockDim.x)
+    for (int i = tid; i < WARPS * E; i += blockDim.x)
         s_cnt[i] = 0;
     __syncthreads();
-    const int64_t a0 = ((int64_t)c * kWarps + warp) * 32 * p.rounds;
+    const int64_t a0 = ((int64_t)c * WARPS + warp) * 32 * p.rounds;
     bool bad = false;
     count_warp_run(p, idx, a0, s_cnt + warp * E, lane, bad);
     if (__any_sync(kFullMask, bad) && lane == 0)
@@ -451,7 +451,7 @@ __device__ bool layout_chunk(const LayoutParams &p, const int c, const int G, in
         for (int e = tid; e < E; e += blockDim.x) {
             int sum = 0;
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w)
+            for (int w = 0; w < WARPS; ++w)
                 sum += s_cnt[w * E + e];
             s_tot[e] = sum;
             s_pre[e] = 0;
@@ -462,7 +462,7 @@ __device__ bool layout_chunk(const LayoutParams &p, const int c, const int G, in
         int sum = 0;
         if (e < E) {
 #pragma unroll
-            for (int w = 0; w < kWarps; ++w)
+            for (int w = 0; w < WARPS; ++w)
                 sum += s_cnt[w * E + e];
         }
         p.wchunk_hist[(int64_t)c * hs + e] = sum;
@@ -473,10 +473,10 @@ __device__ bool layout_chunk(const LayoutParams &p, const int c, const int G, in
     // B. totals and this chunk's prefix, from the whole table
     {
         const int cols = hs / 4;                         // int4 columns per row
-        const int groups = kFusedThreads / cols > 0 ? kFusedThreads / cols : 1;
-        for (int q0 = 0; q0 < cols; q0 += kFusedThreads) {   // more than 1024 experts never happens
-            const int q = q0 + tid % min(cols, kFusedThreads);
-            const int g = tid / min(cols, kFusedThreads);
+        const int groups = (WARPS * 32) / cols > 0 ? (WARPS * 32) / cols : 1;
+        for (int q0 = 0; q0 < cols; q0 += (WARPS * 32)) {   // more than 1024 experts never happens
+            const int q = q0 + tid % min(cols, (WARPS * 32));
+            const int g = tid / min(cols, (WARPS * 32));
             int4 tot = make_int4(0, 0, 0, 0), pre = make_int4(0, 0, 0, 0);
             if (g < groups && q < cols) {
                 const int4 *col = reinterpret_cast<const int4 *>(p.wchunk_hist) + q;
@@ -505,13 +505,13 @@ __device__ bool layout_chunk(const LayoutParams &p, const int c, const int G, in
                 reinterpret_cast<int4 *>(s_red + kRedInts)[g * cols + q - q0] = pre;
             }
             __syncthreads();
-            for (int e = tid; e < min(4 * (cols - q0), 4 * kFusedThreads); e += blockDim.x) {
+            for (int e = tid; e < min(4 * (cols - q0), 4 * (WARPS * 32)); e += blockDim.x) {
                 const int ee = 4 * q0 + e;
                 if (ee < E) {
                     int t = 0, b = 0;
                     for (int gg = 0; gg < groups; ++gg) {
-                        t += s_red[gg * 4 * min(cols, kFusedThreads) + e];
-                        b += s_red[kRedInts + gg * 4 * min(cols, kFusedThreads) + e];
+                        t += s_red[gg * 4 * min(cols, (WARPS * 32)) + e];
+                        b += s_red[kRedInts + gg * 4 * min(cols, (WARPS * 32)) + e];
                     }
                     s_tot[ee] = t;
                     s_pre[ee] = b;
@@ -533,9 +533,9 @@ __device__ bool layout_chunk(const LayoutParams &p, const int c, const int G, in
         s_part[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-        const int v = lane < kWarps ? s_part[lane] : 0;
+        const int v = lane < WARPS ? s_part[lane] : 0;
         const int inc2 = warp_inclusive_scan(v, lane);
-        if (lane < kWarps)
+        if (lane < WARPS)
             s_part[lane] = inc2 - v;
     }
     __syncthreads();
@@ -573,7 +573,7 @@ __device__ bool layout_chunk(const LayoutParams &p, const int c, const int G, in
     for (int e = tid; e < E; e += blockDim.x) {
         int cur = s_off[e] * p.B + s_pre[e];
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
+        for (int w = 0; w < WARPS; ++w) {
             const int n = s_cnt[w * E + e];
             s_cnt[w * E + e] = cur;
             cur += n;
@@ -616,7 +616,7 @@ __device__ bool layout_chunk(const LayoutParams &p, const int c, const int G, in
 
     // D. tile tables and padding rows; one warp per expert, experts spread over
     // the warps of all CTAs
-    for (int e = c * kWarps + warp; e < E; e += G * kWarps) {
+    for (int e = c * WARPS + warp; e < E; e += G * WARPS) {
         const int t0 = s_off[e], t1 = s_off[e + 1];
         const int n = s_tot[e];
         for (int i = lane; i < t1 - t0; i += 32) {
@@ -657,20 +657,29 @@ __device__ bool layout_chunk(const LayoutParams &p, const int c, const int G, in
     return true;
 }
 
-size_t layout_smem_bytes(const LayoutParams &p)
+size_t layout_smem_bytes(const LayoutParams &p, int warps = kWarps)
 {
-    return (size_t)(kWarps * p.E + 3 * p.E + 1 + 2 * kRedInts + p.R) * sizeof(int32_t);
+    return (size_t)(warps * p.E + 3 * p.E + 1 + 2 * kRedInts + p.R) * sizeof(int32_t);
 }
 
-template <typename IdxT>
-__global__ void __launch_bounds__(kFusedThreads) layout_fused_kernel(LayoutParams p)
+template <typename IdxT, int WARPS = kWarps>
+__global__ void __launch_bounds__(WARPS * 32) layout_fused_kernel(LayoutParams p)
 {
     extern __shared__ __align__(16) int32_t sm[];
     __shared__ int s_flag;
-    __shared__ int s_part[kWarps];
+    __shared__ int s_part[WARPS];
     allow_dependents();
-    layout_chunk<IdxT>(p, blockIdx.x, gridDim.x, sm, s_flag, s_part);
+    layout_chunk<IdxT, WARPS>(p, blockIdx.x, gridDim.x, sm, s_flag, s_part);
 }
+
+// Routings of 1025 to 4096 assignments (a decode step) in narrower chunks:
+// kNarrowWarps warps per CTA, one 32-entry round per warp, so more CTAs (and
+// SMs) share the layout's latency-bound phases (decode: 16 CTAs of 4 warps,
+// 26.9 against 27.6 us per step, graph replay 28.1 against 28.6).  Smaller
+// routings keep one CTA of 8 warps, which needs no grid barrier.
+constexpr int kNarrowWarps = 4;
+constexpr int64_t kNarrowMinNa = 1025;
+constexpr int64_t kNarrowMaxNa = 4096;
 
 // ------------------------------------------- layout and dispatch, one launch
 //
@@ -898,6 +907,35 @@ cudaError_t try_layout_dispatch_idx(const LayoutParams &p, const DispatchParams 
 template <typename IdxT>
 cudaError_t launch_layout_t(const LayoutParams &p, cudaStream_t s)
 {
+    if (p.Na >= kNarrowMinNa && p.Na <= kNarrowMaxNa && p.E <= 1024) {
+        // one chunk per 32 * kNarrowWarps assignments, one cooperative launch, one grid barrier
+        LayoutParams q = p;
+        q.rounds = 1;
+        q.num_wchunks = (int)((p.Na + 32LL * kNarrowWarps - 1) / (32LL * kNarrowWarps));
+        const size_t smem = layout_smem_bytes(q, kNarrowWarps);
+        static std::atomic<bool> narrow_attr[64] = {};
+        int dev = 0, sms = 0, per_sm = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+            return cudaErrorInvalidDevice;
+        if (!narrow_attr[dev].load(std::memory_order_acquire)) {
+            const cudaError_t e = cudaFuncSetAttribute(layout_fused_kernel<IdxT, kNarrowWarps>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+            if (e != cudaSuccess)
+                return e;
+            narrow_attr[dev].store(true, std::memory_order_release);
+        }
+        if (q.num_wchunks <= p.num_wchunks * 64 && q.num_wchunks < (int)kBarrierWindow &&
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, layout_fused_kernel<IdxT, kNarrowWarps>,
+                                                          kNarrowWarps * 32, smem) == cudaSuccess &&
+            q.num_wchunks <= per_sm * sms) {
+            void *args[] = {&q};
+            count_launch();
+            return cudaLaunchCooperativeKernel(
+                reinterpret_cast<const void *>(layout_fused_kernel<IdxT, kNarrowWarps>), dim3(q.num_wchunks),
+                dim3(kNarrowWarps * 32), args, smem, s);
+        }
+    }
     const int chunks = p.num_wchunks;
     const size_t smem_count = (size_t)kWarps * p.E * sizeof(int32_t);
     const size_t smem_fused = layout_smem_bytes(p);
@@ -997,6 +1035,8 @@ cudaError_t preload_layout_kernels()
                        reinterpret_cast<const void *>(layout_dispatch_kernel<long long, SEP_SCALE_F32_POW2>),
                        reinterpret_cast<const void *>(layout_fused_kernel<int>),
                        reinterpret_cast<const void *>(layout_fused_kernel<long long>),
+                       reinterpret_cast<const void *>(layout_fused_kernel<int, kNarrowWarps>),
+                       reinterpret_cast<const void *>(layout_fused_kernel<long long, kNarrowWarps>),
                        reinterpret_cast<const void *>(layout_count_kernel<int>),
                        reinterpret_cast<const void *>(layout_count_kernel<long long>),
                        reinterpret_cast<const void *>(layout_scan_kernel),

@@ -130,6 +130,9 @@ class EPGroup:
         self.rows = [self.rows_cap] * self.world         # capacities: the kernels refuse rows past them
         _sep.sep_ep_mark_padding(plan["owner_block_offset"], plan["owner_expert_counts"], self.B, self.rows_cap,
                                  self.recv_token[self.rank], self.recv_rank[self.rank], self.recv_slot[self.rank])
+        # this owner's arrival counters start the step at zero even if the last
+        # step's tiles were not all consumed (the consumer zeroes only what it copies)
+        self.arrival[self.rank].zero_()
         self._barrier()                                  # every owner ready, the last step's readers done
         self.seq = (self.seq + 1) & 0x7FFFFFFF or 1
         maps = dict(recv_token=self.recv_token, recv_rank=self.recv_rank, recv_slot=self.recv_slot)
