@@ -20,10 +20,12 @@ group's backend is gloo), so the host never waits for a count; every owner
 tile is published once complete (``sep_ep_dispatch_publish``: per-tile
 arrivals and a system-scope release of the step's sequence number in the
 owner's memory), and the owner's reference consumer (``consume``) copies each
-tile as it is published.  The barriers stay by default; ``concurrent=True``
-drops the one between the dispatches and the owners' consumers, for groups
-whose ranks are on different GPUs (never for ranks sharing a GPU, whose
-kernels are not guaranteed to run at the same time).
+tile as it is published.  A step then holds two or three barriers instead
+of four: the one after the combine goes (the next step's barrier before its
+dispatches follows every rank's synchronised combine), and
+``concurrent=True`` drops the one between the dispatches and the owners'
+consumers, for groups whose ranks are on different GPUs (never for ranks
+sharing a GPU, whose kernels are not guaranteed to run at the same time).
 
 The dispatch may carry the bf16 rows or the FP8 e4m3 payload with its
 per-128-channel scales.  The pools, y buffers, scales and receive maps are
@@ -212,7 +214,10 @@ class EPGroup:
         if self.signals and int(self.status[0].item()) != 0:
             raise RuntimeError(f"an owner's consumer reported {self.status.cpu().tolist()}")
         _sep.sep_ep_combine(self.handle, ys, self.rows, self.delta, topk_weight, out, self.error)
-        self._barrier()                                  # before the next step reuses the buffers
+        if not self.signals:
+            self._barrier()                              # before the next step reuses the buffers
+        # with signals the next step's pre-dispatch barrier follows every rank's
+        # synchronised combine before any pool, y buffer or counter is written again
         if int(self.error.item()) != 0:
             raise RuntimeError("a row fell outside its owner's pool")
 
