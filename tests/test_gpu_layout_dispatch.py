@@ -250,3 +250,26 @@ def test_one_launch_step_replays_from_a_cuda_graph(name, payload, scale):
         del g
     finally:
         sep.sep_handle_free(h)
+
+
+@pytest.mark.parametrize("flags", [sep.SEP_LAYOUT_SYNC_COUNTS | sep.SEP_LAYOUT_TOKEN_IN_OWNER,
+                                   sep.SEP_LAYOUT_SYNC_COUNTS | sep.SEP_LAYOUT_TOKEN_IN_OWNER | ONE])
+def test_layout_flags_pass_through(flags):
+    """SEP_LAYOUT_SYNC_COUNTS makes the exact pool size known on return and
+    SEP_LAYOUT_TOKEN_IN_OWNER fills is_token_in_rank and the per-owner token
+    counts, as with sep_layout."""
+    w = W.WORKLOADS["decode"]
+    d = W.make_inputs(w)
+    lay = oracle.layout(d["topk_idx"].numpy(), w.E, w.R, w.B)
+    h = sep.sep_handle_create(w.T, w.k, w.E, w.R, w.B, flags=sep.SEP_LAYOUT_TOKEN_IN_OWNER)
+    try:
+        rows = h.info().max_pool_rows
+        recv, sc = _pool(rows, w.H, "fp8", "ue8m0")
+        sep.sep_layout_dispatch(d["topk_idx"].cuda(), d["x"].cuda(), recv, w.E, w.R, w.B, payload="fp8",
+                                scale="ue8m0", recv_scales=sc, handle=h, flags=flags)
+        info = h.info()
+        assert info.num_pool_rows == lay.num_pool_rows and info.num_tiles == lay.num_tiles
+        check_layout(h, lay, token_in_owner=True)
+        _check_pool(lay, d["x"], recv, sc, "fp8", "ue8m0")
+    finally:
+        sep.sep_handle_free(h)
