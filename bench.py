@@ -65,7 +65,7 @@ def parse_args(argv=None):
                     help="CTAs of the gated combine in the combine_gate measurement (0: one per SM)")
     ap.add_argument("--no-graph", action="store_true",
                     help="skip timing the step replayed from a CUDA graph (non-streaming workloads)")
-    ap.add_argument("--extras", default="borrowed,backward,gate,scatter,ep",
+    ap.add_argument("--extras", default="borrowed,backward,gate,scatter,ep,budget",
                     help="comma list of the measurements taken after the timed region")
     ap.add_argument("--profile-case", default=None,
                     choices=["layout", "layout_dispatch", "one_launch", "dispatch", "combine", "consumer", "gated",
@@ -606,6 +606,8 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
                if want("scatter") else None)
     ep = (ep_compare(w, dev, None if flush is None else flush.zero_, peaks["hbm_gbs"])
           if w.payload == "bf16" and not w.streaming and want("ep") and w.T % w.R == 0 else None)
+    budget = (budget_compare(w, h, x, idx, recv, scales, y, wt, None if flush is None else flush.zero_, peaks["hbm_gbs"])
+              if not w.streaming and want("budget") else None)
     sep.sep_handle_free(h)
 
     ab = algorithmic_bytes(w)
@@ -674,6 +676,7 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
         **({"combine_gate": gate} if gate else {}),
         **({"combine_scatter": scatter} if scatter else {}),
         **({"ep_emulated": ep} if ep else {}),
+        **({"sm_budget": budget} if budget else {}),
         "clocks": sampler.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -780,6 +783,33 @@ def scatter_compare(w, h, idx, wt, y, flush, peak_gbs, steps=100):
             "delta_pct": 100.0 * (scatter_us - gather_us) / gather_us,
             "note": "same combine bytes for both (the scatter also writes out's zeros first); "
                     "L2 flushed before every call"}
+
+
+def budget_compare(w, h, x, idx, recv, scales, y, wt, flush, peak_gbs, steps=50):
+    """The dispatch and the combine alone (L2 flushed before every call) with a
+    CTA budget: how much of the copy bandwidth a fraction of the SMs reaches
+    (the DeepEP vibeleaderboard entry, "Why it's ranked here": peak bandwidth
+    with up to 4x fewer SMs).  0 is the default grid (one CTA per 8 items)."""
+    import torch
+    import combine_route_layout_02_b200 as sep
+    out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=x.device)
+    sep.sep_layout(idx, w.E, w.R, w.B, handle=h)
+    ab = algorithmic_bytes(w)
+    sms = torch.cuda.get_device_properties(x.device).multi_processor_count
+    res = []
+    for ctas in (sms // 8, sms // 4, sms // 2, sms, 2 * sms, 0):
+        sep.sep_handle_set_max_ctas(h, ctas)
+        d_us = _time_arm(lambda: sep.sep_dispatch(h, x, recv, payload=w.payload, scale=w.scale, recv_scales=scales),
+                         steps, flush)
+        c_us = _time_arm(lambda: sep.sep_combine(h, y, wt, out), steps, flush)
+        res.append({"max_ctas": ctas, "dispatch_us": d_us, "combine_us": c_us,
+                    "dispatch_frac": ab["dispatch"] / (d_us * 1e-6) / 1e9 / peak_gbs,
+                    "combine_frac": ab["combine"] / (c_us * 1e-6) / 1e9 / peak_gbs})
+    sep.sep_handle_set_max_ctas(h, 0)
+    return {"sms": sms, "budgets": res,
+            "note": "each kernel alone on the bench workload's layout, L2 flushed before every call; max_ctas 0 is "
+                    "the default grid; 8-warp CTAs, so max_ctas = SMs means about one CTA per SM"}
+
 
 
 def ep_compare(w, dev, flush, peak_gbs, steps=100):

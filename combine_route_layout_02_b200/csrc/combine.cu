@@ -223,7 +223,8 @@ cudaError_t launch_combine(CombineParams p, cudaStream_t s, int num_sms, int num
         const int64_t n = want < num_ctas ? want : num_ctas;
         return launch_kernel(combine_kernel<true>, dim3((int)n), dim3(kWarps * 32), 0, s, p);
     }
-    return launch_kernel(combine_kernel<false>, dim3((int)want), dim3(kWarps * 32), 0, s, p);
+    const int64_t ctas = p.max_ctas > 0 && want > p.max_ctas ? p.max_ctas : want;
+    return launch_kernel(combine_kernel<false>, dim3((int)ctas), dim3(kWarps * 32), 0, s, p);
 }
 
 cudaError_t preload_combine_kernels()

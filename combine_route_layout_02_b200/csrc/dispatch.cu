@@ -256,16 +256,19 @@ bool staged_dispatch_selected()
 
 // One warp per work item and no cap at the resident CTA count: CTAs that
 // finish early make room for the rest, which balances the tail across SMs.
+// A caller's CTA budget (max_ctas) caps the grid instead; the kernels walk
+// their items with a grid stride, so any grid size covers them.
 template <typename K>
-int blocks_for(K, int64_t items, int)
+int blocks_for(K, int64_t items, int max_ctas)
 {
-    return (int)((items + kWarps - 1) / kWarps);
+    const int64_t b = (items + kWarps - 1) / kWarps;
+    return (int)(max_ctas > 0 && b > max_ctas ? max_ctas : b);
 }
 
 template <bool PUBLISH>
 cudaError_t launch_fp8(const DispatchParams &p, cudaStream_t s, int num_sms)
 {
-    const dim3 grid(blocks_for(0, p.T * p.segs, num_sms)), block(kWarps * 32);
+    const dim3 grid(blocks_for(0, p.T * p.segs, p.max_ctas)), block(kWarps * 32);
     switch (p.scale) {
     case SEP_SCALE_F32:
         return launch_kernel(dispatch_fp8_kernel<SEP_SCALE_F32, PUBLISH>, grid, block, 0, s, p);
@@ -302,12 +305,12 @@ cudaError_t launch_dispatch(DispatchParams p, int payload, cudaStream_t s, int n
     const int64_t items = p.T * p.segs;
     if (payload == SEP_PAYLOAD_BF16) {
         if (p.tile_ready == nullptr && p.seg_len % kStageVecs == 0 && staged_dispatch_selected())
-            return launch_kernel(dispatch_bf16_staged_kernel, dim3(blocks_for(0, items, num_sms)),
+            return launch_kernel(dispatch_bf16_staged_kernel, dim3(blocks_for(0, items, p.max_ctas)),
                                  dim3(kWarps * 32), 0, s, p);
         if (p.tile_ready != nullptr)
-            return launch_kernel(dispatch_bf16_kernel<4, true>, dim3(blocks_for(0, items, num_sms)),
+            return launch_kernel(dispatch_bf16_kernel<4, true>, dim3(blocks_for(0, items, p.max_ctas)),
                                  dim3(kWarps * 32), 0, s, p);
-        return launch_kernel(dispatch_bf16_kernel<4, false>, dim3(blocks_for(0, items, num_sms)),
+        return launch_kernel(dispatch_bf16_kernel<4, false>, dim3(blocks_for(0, items, p.max_ctas)),
                              dim3(kWarps * 32), 0, s, p);
     }
     return p.tile_ready != nullptr ? launch_fp8<true>(p, s, num_sms) : launch_fp8<false>(p, s, num_sms);

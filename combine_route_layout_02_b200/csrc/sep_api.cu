@@ -520,6 +520,16 @@ sep_status sep_handle_info(const sep_handle *h, sep_layout_info *info)
     return SEP_OK;
 }
 
+sep_status sep_handle_set_max_ctas(sep_handle *h, int max_ctas)
+{
+    if (h == nullptr)
+        return fail(SEP_ERR_INVALID_ARG, "NULL handle");
+    if (max_ctas < 0)
+        return fail(SEP_ERR_INVALID_ARG, "max_ctas must be >= 0 (got %d)", max_ctas);
+    h->max_ctas = max_ctas;
+    return SEP_OK;
+}
+
 sep_status sep_handle_sync(sep_handle *h, void *stream)
 {
     if (h == nullptr)
@@ -598,6 +608,7 @@ sep::DispatchParams dispatch_params(const sep_handle *h, const void *x, int64_t 
     p.pool_arrival_target = h->pool_arrival_target;
     p.error_epoch = h->timeout_epoch;
     p.epoch = h->epoch;
+    p.max_ctas = h->max_ctas;
     return p;
 }
 
@@ -745,6 +756,7 @@ sep_status prepare_combine(const sep_handle *h, uint32_t layout_epoch, const voi
     p->src_pool_row = h->src_pool_row;
     p->w = weighted ? w : nullptr;
     p->out = out;
+    p->max_ctas = h->max_ctas;
     p->error_epoch = h->timeout_epoch;
     p->epoch = h->epoch;
     return SEP_OK;

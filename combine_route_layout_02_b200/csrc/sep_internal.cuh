@@ -83,6 +83,7 @@ struct DispatchParams {
     int scale;                       // sep_scale
     int segs;                        // warps sharing one token row (set by launch_dispatch)
     int seg_len;                     // per warp: 16-byte vectors (bf16) or 512-channel steps (fp8)
+    int max_ctas;                    // > 0: at most this many CTAs (the grid walks the items)
     // streaming publication (tile_ready != nullptr)
     uint32_t *tile_ready;
     uint32_t *pool_arrival_count;
@@ -130,6 +131,7 @@ struct CombineParams {
     void *out;                       // bf16 [T][H]
     int segs;                        // warps sharing one token row
     int seg_len;                     // 16-byte vectors per warp
+    int max_ctas;                    // > 0: at most this many CTAs (ungated; the grid walks the items)
     uint32_t *error_epoch;           // a bounded wait that gave up records the epoch
     uint32_t epoch;
     // per-token gate (y_done != nullptr): token t is reduced once y_done[t] >= done_seq
@@ -374,6 +376,8 @@ struct sep_handle {
     uint32_t *timeout_epoch;         // a bounded wait gave up during this epoch
     uint32_t *barrier_words;         // grid-barrier counter of the single-launch layout
     uint32_t *token_arrivals;        // [T_cap] per-token row counters of the stamping consumer
+    // CTA budget of the dispatch and combine launches (0: one warp per work item)
+    int max_ctas;
     // borrowed-view lease and the consumer events its release recorded
     int leased;
     int n_release;

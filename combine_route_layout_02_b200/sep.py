@@ -66,6 +66,7 @@ _SIGNATURES = [
     ("sep_handle_create", _i32, [_i64, _i32, _i32, _i32, _i32, _u32, _P, ctypes.POINTER(_P)]),
     ("sep_handle_info", _i32, [_P, ctypes.POINTER(LayoutInfo)]),
     ("sep_handle_sync", _i32, [_P, _P]),
+    ("sep_handle_set_max_ctas", _i32, [_P, _i32]),
     ("sep_dispatch", _i32, [_P, _P, _i64, _i32, _i32, _P, _P, _i64, _P, _i64, _u32, _P]),
     ("sep_combine", _i32, [_P, _u32, _P, _i64, _i64, _P, _P, _P]),
     ("sep_consume_tiles", _i32, [_P, _P, _i64, _i64, _P, _i64, _u32, _P, _i32, _u64, _P, _P]),
@@ -233,6 +234,11 @@ def sep_layout(topk_idx: torch.Tensor, num_experts: int, num_owners: int, block_
 
 def sep_handle_sync(handle: Handle, stream=None) -> None:
     _check(_lib.sep_handle_sync(handle.ptr, _stream(stream)), "sep_handle_sync")
+
+
+def sep_handle_set_max_ctas(handle: Handle, max_ctas: int) -> None:
+    """CTA budget of the handle's dispatch and combine launches (0: unbounded)."""
+    _check(_lib.sep_handle_set_max_ctas(handle.ptr, int(max_ctas)), "sep_handle_set_max_ctas")
 
 
 def sep_dispatch(handle: Handle, x: torch.Tensor, recv_x: torch.Tensor, payload: str = "bf16",

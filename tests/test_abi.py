@@ -23,7 +23,7 @@ def test_library_is_built_for_sm100a_and_in_tree():
 
 def test_exports_match_header():
     declared = sep.declared_entry_points(HEADER)
-    assert len(declared) == 33
+    assert len(declared) == 34
     out = subprocess.run(["nm", "-D", "--defined-only", sep.library_path()], capture_output=True,
                          text=True, check=True).stdout
     exported = sorted(set(re.findall(r"\sT\s+(sep_\w+)$", out, flags=re.M)))
@@ -153,3 +153,8 @@ def test_layout_dispatch_rejects_bad_arguments_before_any_cuda_call():
     assert call(1 << 20, x=8) == sep.SEP_ERR_INVALID_ARG
     assert call(1 << 20, k=0) == sep.SEP_ERR_INVALID_ARG
     assert not h.value
+
+
+def test_cta_budget_rejects_bad_arguments_before_any_cuda_call():
+    lib = sep.library()
+    assert lib.sep_handle_set_max_ctas(None, 4) == sep.SEP_ERR_INVALID_ARG

@@ -631,3 +631,34 @@ def test_borrowed_view_delayed_cross_stream_reader():
         check_layout(h, oracle.layout(other.numpy(), w.E, w.R, w.B))
     finally:
         sep.sep_handle_free(h)
+
+
+@pytest.mark.parametrize("max_ctas", [1, 3, 37])
+def test_cta_budget_keeps_every_result(max_ctas):
+    """With a CTA budget the dispatch and combine grids walk all their work
+    items with fewer CTAs: pool rows (bf16 and FP8), codes, scales and the
+    combine equal the oracle bit for bit."""
+    w, d = _inputs(W.WORKLOADS["train8k"], 700)
+    lay = oracle.layout(d["topk_idx"].numpy(), w.E, w.R, w.B)
+    h = sep.sep_layout(d["topk_idx"].cuda(), w.E, w.R, w.B, flags=sep.SEP_LAYOUT_SYNC_COUNTS)
+    try:
+        sep.sep_handle_set_max_ctas(h, max_ctas)
+        P = lay.num_pool_rows
+        valid = lay.pool_recv_token >= 0
+        recv = poisoned_bf16(P, w.H)
+        sep.sep_dispatch(h, d["x"].cuda(), recv)
+        want = oracle.dispatch_bf16(d["x"], lay)
+        got = bf16_bits(recv)
+        np.testing.assert_array_equal(got[valid], want[valid])
+        assert (got[~valid] == POISON_BF16).all()
+        out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device="cuda")
+        sep.sep_combine(h, recv, d["topk_weight"].cuda(), out)
+        check_combine(bf16_bits(out), oracle.combine(want, d["topk_weight"].numpy(), lay))
+        codes = torch.full((P, w.H), POISON_U8, dtype=torch.uint8, device="cuda")
+        scales = torch.zeros(P, w.H // 128, dtype=torch.uint8, device="cuda")
+        sep.sep_dispatch(h, d["x"].cuda(), codes, payload="fp8", scale="ue8m0", recv_scales=scales)
+        want_c, want_s = oracle.dispatch_fp8(d["x"], lay, "ue8m0")
+        np.testing.assert_array_equal(codes.cpu().numpy()[valid], want_c[valid])
+        np.testing.assert_array_equal(scales.cpu().numpy()[valid], want_s[valid])
+    finally:
+        sep.sep_handle_free(h)
