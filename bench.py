@@ -65,7 +65,7 @@ def parse_args(argv=None):
                     help="CTAs of the gated combine in the combine_gate measurement (0: one per SM)")
     ap.add_argument("--no-graph", action="store_true",
                     help="skip timing the step replayed from a CUDA graph (non-streaming workloads)")
-    ap.add_argument("--extras", default="borrowed,backward,gate,scatter,ep,budget",
+    ap.add_argument("--extras", default="borrowed,backward,gate,scatter,ep,budget,overlap",
                     help="comma list of the measurements taken after the timed region")
     ap.add_argument("--profile-case", default=None,
                     choices=["layout", "layout_dispatch", "one_launch", "dispatch", "combine", "consumer", "gated",
@@ -608,6 +608,8 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
           if w.payload == "bf16" and not w.streaming and want("ep") and w.T % w.R == 0 else None)
     budget = (budget_compare(w, h, x, idx, recv, scales, y, wt, None if flush is None else flush.zero_, peaks["hbm_gbs"])
               if not w.streaming and want("budget") else None)
+    overlap = (overlap_compare(w, h, x, idx, recv, y, wt, None if flush is None else flush.zero_)
+               if w.payload == "bf16" and not w.streaming and want("overlap") else None)
     sep.sep_handle_free(h)
 
     ab = algorithmic_bytes(w)
@@ -677,6 +679,7 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
         **({"combine_scatter": scatter} if scatter else {}),
         **({"ep_emulated": ep} if ep else {}),
         **({"sm_budget": budget} if budget else {}),
+        **({"gemm_overlap": overlap} if overlap else {}),
         "clocks": sampler.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -810,6 +813,59 @@ def budget_compare(w, h, x, idx, recv, scales, y, wt, flush, peak_gbs, steps=50)
             "note": "each kernel alone on the bench workload's layout, L2 flushed before every call; max_ctas 0 is "
                     "the default grid; 8-warp CTAs, so max_ctas = SMs means about one CTA per SM"}
 
+
+
+def overlap_compare(w, h, x, idx, recv, y, wt, flush, steps=30):
+    """What the CTA budget is for: the dispatch and combine on one stream beside
+    a dense bf16 GEMM on another (cuBLAS through torch, [T, H] x [H, 4096],
+    standing in for an expert GEMM of another micro-batch).  Per budget: the
+    GEMM alone, dispatch + combine alone, the two one after the other, and the
+    two concurrently (fork on the main stream, join back; L2 flushed before
+    each)."""
+    import torch
+    import combine_route_layout_02_b200 as sep
+    dev = x.device
+    main = torch.cuda.current_stream()
+    side = torch.cuda.Stream()
+    g = torch.Generator(device="cpu").manual_seed(5)
+    a = torch.randn(w.T, w.H, generator=g).to(dev, torch.bfloat16)
+    b = torch.randn(w.H, 4096, generator=g).to(dev, torch.bfloat16)
+    c = torch.empty(w.T, 4096, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
+    sep.sep_layout(idx, w.E, w.R, w.B, handle=h)
+
+    def gemm():
+        torch.matmul(a, b, out=c)
+
+    def comm():
+        sep.sep_dispatch(h, x, recv)
+        sep.sep_combine(h, y, wt, out)
+
+    def serial():
+        gemm()
+        comm()
+
+    def concurrent():
+        side.wait_stream(main)
+        with torch.cuda.stream(side):
+            gemm()
+        comm()
+        main.wait_stream(side)
+
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    gemm_us = _time_arm(gemm, steps, flush)
+    res = []
+    for ctas in (0, sms // 4, sms // 2, 3 * sms // 4):
+        sep.sep_handle_set_max_ctas(h, ctas)
+        comm_us = _time_arm(comm, steps, flush)
+        serial_us = _time_arm(serial, steps, flush)
+        conc_us = _time_arm(concurrent, steps, flush)
+        res.append({"max_ctas": ctas, "comm_us": comm_us, "serial_us": serial_us, "concurrent_us": conc_us,
+                    "saved_pct": 100.0 * (serial_us - conc_us) / serial_us})
+    sep.sep_handle_set_max_ctas(h, 0)
+    return {"gemm_us": gemm_us, "gemm_tflops": 2.0 * w.T * w.H * 4096 / (gemm_us * 1e-6) / 1e12, "budgets": res,
+            "note": "bf16 GEMM [T,H]x[H,4096] on a side stream beside the budgeted dispatch + combine; max_ctas 0 is "
+                    "the default grid; L2 flushed before every call"}
 
 
 def ep_compare(w, dev, flush, peak_gbs, steps=100):

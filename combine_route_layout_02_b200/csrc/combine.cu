@@ -115,8 +115,8 @@ __device__ __forceinline__ uint4 pack_out(const float *acc)
                       pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
 }
 
-template <bool GATED>
-__global__ void __launch_bounds__(kWarps * 32) combine_kernel(CombineParams p)
+template <bool GATED, int WARPS = kWarps>
+__global__ void __launch_bounds__(WARPS * 32) combine_kernel(CombineParams p)
 {
     grid_dependency_wait();
     allow_dependents();
@@ -223,8 +223,14 @@ cudaError_t launch_combine(CombineParams p, cudaStream_t s, int num_sms, int num
         const int64_t n = want < num_ctas ? want : num_ctas;
         return launch_kernel(combine_kernel<true>, dim3((int)n), dim3(kWarps * 32), 0, s, p);
     }
-    const int64_t ctas = p.max_ctas > 0 && want > p.max_ctas ? p.max_ctas : want;
-    return launch_kernel(combine_kernel<false>, dim3((int)ctas), dim3(kWarps * 32), 0, s, p);
+    if (p.max_ctas > 0 && want > p.max_ctas) {
+        // a CTA budget below the default grid: at most max_ctas CTAs of kBudgetWarps warps (about one per
+        // SM; a small grid of 8-warp CTAs keeps too few row loads in flight per SM)
+        const int64_t b = (items + kBudgetWarps - 1) / kBudgetWarps;
+        return launch_kernel(combine_kernel<false, kBudgetWarps>, dim3((int)(b < p.max_ctas ? b : p.max_ctas)),
+                             dim3(kBudgetWarps * 32), 0, s, p);
+    }
+    return launch_kernel(combine_kernel<false>, dim3((int)want), dim3(kWarps * 32), 0, s, p);
 }
 
 cudaError_t preload_combine_kernels()
@@ -233,6 +239,8 @@ cudaError_t preload_combine_kernels()
     cudaError_t e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(combine_kernel<false>));
     if (e == cudaSuccess)
         e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(combine_kernel<true>));
+    if (e == cudaSuccess)
+        e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(combine_kernel<false, kBudgetWarps>));
     return e;
 }
 

@@ -77,8 +77,8 @@ __device__ __forceinline__ void publish_rows(const DispatchParams &p, int my_row
 }
 
 // bf16: a work item is (token, segment of seg_len 16-byte vectors).
-template <int UNROLL, bool PUBLISH>
-__global__ void __launch_bounds__(kWarps * 32) dispatch_bf16_kernel(DispatchParams p)
+template <int UNROLL, bool PUBLISH, int WARPS = kWarps>
+__global__ void __launch_bounds__(WARPS * 32) dispatch_bf16_kernel(DispatchParams p)
 {
     grid_dependency_wait();
     allow_dependents();
@@ -119,8 +119,8 @@ __global__ void __launch_bounds__(kWarps * 32) dispatch_bf16_kernel(DispatchPara
 }
 
 // fp8: a work item is (token, segment of seg_len 512-channel iterations).
-template <int SCALE, bool PUBLISH>
-__global__ void __launch_bounds__(kWarps * 32) dispatch_fp8_kernel(DispatchParams p)
+template <int SCALE, bool PUBLISH, int WARPS = kWarps>
+__global__ void __launch_bounds__(WARPS * 32) dispatch_fp8_kernel(DispatchParams p)
 {
     grid_dependency_wait();
     allow_dependents();
@@ -256,26 +256,32 @@ bool staged_dispatch_selected()
 
 // One warp per work item and no cap at the resident CTA count: CTAs that
 // finish early make room for the rest, which balances the tail across SMs.
-// A caller's CTA budget (max_ctas) caps the grid instead; the kernels walk
-// their items with a grid stride, so any grid size covers them.
-template <typename K>
-int blocks_for(K, int64_t items, int max_ctas)
+// A caller's CTA budget (max_ctas) below that grid launches at most max_ctas
+// CTAs of kBudgetWarps warps instead (about one per SM: a small grid of
+// 8-warp CTAs keeps too few loads in flight per SM); the kernels walk their
+// items with a grid stride, so any grid covers them.
+int64_t default_blocks(int64_t items)
 {
-    const int64_t b = (items + kWarps - 1) / kWarps;
-    return (int)(max_ctas > 0 && b > max_ctas ? max_ctas : b);
+    return (items + kWarps - 1) / kWarps;
 }
 
-template <bool PUBLISH>
-cudaError_t launch_fp8(const DispatchParams &p, cudaStream_t s, int num_sms)
+int budget_blocks(int64_t items, int max_ctas)
 {
-    const dim3 grid(blocks_for(0, p.T * p.segs, p.max_ctas)), block(kWarps * 32);
+    const int64_t b = (items + kBudgetWarps - 1) / kBudgetWarps;
+    return (int)(b > max_ctas ? max_ctas : b);
+}
+
+template <bool PUBLISH, int WARPS>
+cudaError_t launch_fp8(const DispatchParams &p, cudaStream_t s, dim3 grid)
+{
+    const dim3 block(WARPS * 32);
     switch (p.scale) {
     case SEP_SCALE_F32:
-        return launch_kernel(dispatch_fp8_kernel<SEP_SCALE_F32, PUBLISH>, grid, block, 0, s, p);
+        return launch_kernel(dispatch_fp8_kernel<SEP_SCALE_F32, PUBLISH, WARPS>, grid, block, 0, s, p);
     case SEP_SCALE_UE8M0:
-        return launch_kernel(dispatch_fp8_kernel<SEP_SCALE_UE8M0, PUBLISH>, grid, block, 0, s, p);
+        return launch_kernel(dispatch_fp8_kernel<SEP_SCALE_UE8M0, PUBLISH, WARPS>, grid, block, 0, s, p);
     default:
-        return launch_kernel(dispatch_fp8_kernel<SEP_SCALE_F32_POW2, PUBLISH>, grid, block, 0, s, p);
+        return launch_kernel(dispatch_fp8_kernel<SEP_SCALE_F32_POW2, PUBLISH, WARPS>, grid, block, 0, s, p);
     }
 }
 
@@ -303,17 +309,24 @@ cudaError_t launch_dispatch(DispatchParams p, int payload, cudaStream_t s, int n
                &p.segs, &steps);
     p.seg_len = (int)(fp8 ? steps : steps * kStepVecs);
     const int64_t items = p.T * p.segs;
+    if (p.max_ctas > 0 && p.max_ctas < default_blocks(items)) {
+        const dim3 grid(budget_blocks(items, p.max_ctas)), block(kBudgetWarps * 32);
+        if (payload == SEP_PAYLOAD_BF16)
+            return p.tile_ready != nullptr
+                       ? launch_kernel(dispatch_bf16_kernel<4, true, kBudgetWarps>, grid, block, 0, s, p)
+                       : launch_kernel(dispatch_bf16_kernel<4, false, kBudgetWarps>, grid, block, 0, s, p);
+        return p.tile_ready != nullptr ? launch_fp8<true, kBudgetWarps>(p, s, grid)
+                                       : launch_fp8<false, kBudgetWarps>(p, s, grid);
+    }
+    const dim3 grid((int)default_blocks(items)), block(kWarps * 32);
     if (payload == SEP_PAYLOAD_BF16) {
         if (p.tile_ready == nullptr && p.seg_len % kStageVecs == 0 && staged_dispatch_selected())
-            return launch_kernel(dispatch_bf16_staged_kernel, dim3(blocks_for(0, items, p.max_ctas)),
-                                 dim3(kWarps * 32), 0, s, p);
+            return launch_kernel(dispatch_bf16_staged_kernel, grid, block, 0, s, p);
         if (p.tile_ready != nullptr)
-            return launch_kernel(dispatch_bf16_kernel<4, true>, dim3(blocks_for(0, items, p.max_ctas)),
-                                 dim3(kWarps * 32), 0, s, p);
-        return launch_kernel(dispatch_bf16_kernel<4, false>, dim3(blocks_for(0, items, p.max_ctas)),
-                             dim3(kWarps * 32), 0, s, p);
+            return launch_kernel(dispatch_bf16_kernel<4, true>, grid, block, 0, s, p);
+        return launch_kernel(dispatch_bf16_kernel<4, false>, grid, block, 0, s, p);
     }
-    return p.tile_ready != nullptr ? launch_fp8<true>(p, s, num_sms) : launch_fp8<false>(p, s, num_sms);
+    return p.tile_ready != nullptr ? launch_fp8<true, kWarps>(p, s, grid) : launch_fp8<false, kWarps>(p, s, grid);
 }
 
 cudaError_t preload_dispatch_kernels()
@@ -327,7 +340,15 @@ cudaError_t preload_dispatch_kernels()
         reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_UE8M0, false>),
         reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_UE8M0, true>),
         reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_F32_POW2, false>),
-        reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_F32_POW2, true>)};
+        reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_F32_POW2, true>),
+        reinterpret_cast<const void *>(dispatch_bf16_kernel<4, false, kBudgetWarps>),
+        reinterpret_cast<const void *>(dispatch_bf16_kernel<4, true, kBudgetWarps>),
+        reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_F32, false, kBudgetWarps>),
+        reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_F32, true, kBudgetWarps>),
+        reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_UE8M0, false, kBudgetWarps>),
+        reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_UE8M0, true, kBudgetWarps>),
+        reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_F32_POW2, false, kBudgetWarps>),
+        reinterpret_cast<const void *>(dispatch_fp8_kernel<SEP_SCALE_F32_POW2, true, kBudgetWarps>)};
     cudaFuncAttributes a;
     for (const void *f : k) {
         const cudaError_t e = cudaFuncGetAttributes(&a, f);

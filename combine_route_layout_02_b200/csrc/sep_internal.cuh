@@ -73,6 +73,10 @@ cudaError_t launch_layout(const LayoutParams &p, int idx_bytes, cudaStream_t s);
 
 // --------------------------------------------------------------- dispatch
 
+// Warps per CTA of a dispatch or combine launched under a CTA budget below
+// its default grid: a whole SM's worth, so max_ctas CTAs cover about as many SMs.
+constexpr int kBudgetWarps = 32;
+
 struct DispatchParams {
     const void *x;                   // bf16 [T][H]
     int64_t T;

@@ -177,13 +177,15 @@ SEP_API sep_status sep_handle_sync(sep_handle *handle, void *stream);
 
 /*
  * sep_handle_set_max_ctas — the CTA budget of this handle's dispatch and
- * combine launches (sep_dispatch without tile_ready, the dispatch launch of
- * sep_layout_dispatch, sep_combine, sep_combine_grads).  0 (the default): one 8-warp CTA per eight
- * work items, every SM used.  n > 0: at most n CTAs, which walk all the work
- * items, so the kernels leave the other SMs to a concurrent kernel (an expert
- * GEMM) at the cost of bandwidth (the DeepEP vibeleaderboard entry, "Why it's
- * ranked here": peak bandwidth with a fraction of the SMs).  Host-only; takes
- * effect at the next launch; SEP_ERR_INVALID_ARG for n < 0.
+ * combine launches (sep_dispatch, bf16 or FP8, with or without tile_ready; the
+ * dispatch launch of sep_layout_dispatch; sep_combine; sep_combine_grads).
+ * 0 (the default): one 8-warp CTA per eight work items, every SM used.  n > 0
+ * below that grid: at most n CTAs of 32 warps (about one per SM), which walk
+ * all the work items, so the kernels leave the other SMs to a concurrent
+ * kernel (an expert GEMM) at the cost of bandwidth (the DeepEP vibeleaderboard
+ * entry, "Why it's ranked here": peak bandwidth with a fraction of the SMs).
+ * Results are identical under any budget.  Host-only; takes effect at the next
+ * launch; SEP_ERR_INVALID_ARG for n < 0.
  */
 SEP_API sep_status sep_handle_set_max_ctas(sep_handle *handle, int max_ctas);
 

@@ -43,7 +43,7 @@ def test_traffic_is_reported_only_for_the_profiled_sources(tmp_path, monkeypatch
 
 def test_argument_defaults():
     a = bench.parse_args([])
-    assert a.extras.split(",") == ["borrowed", "backward", "gate", "scatter", "ep", "budget"]
+    assert a.extras.split(",") == ["borrowed", "backward", "gate", "scatter", "ep", "budget", "overlap"]
     assert not a.no_graph and not a.no_extras and a.gate_ctas == 0 and a.consumer_ctas == 64
 
 

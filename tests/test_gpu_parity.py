@@ -662,3 +662,44 @@ def test_cta_budget_keeps_every_result(max_ctas):
         np.testing.assert_array_equal(scales.cpu().numpy()[valid], want_s[valid])
     finally:
         sep.sep_handle_free(h)
+
+
+@pytest.mark.parametrize("kind,T,k,H,max_ctas", [
+    ("uniform", 1000, 8, 3072, 37),
+    ("masked", 777, 4, 264, 5),         # a ragged 528-byte row; masked assignments
+    ("skew", 300, 8, 7168, 2),
+    ("one_expert", 129, 2, 8, 1),       # 16-byte rows, duplicate experts, one CTA
+    ("uniform", 64, 8, 16384, 100),     # long rows split over several warps
+    ("uniform", 257, 32, 64, 3),        # k = 32
+])
+def test_budget_grids_match_the_oracle(kind, T, k, H, max_ctas):
+    """A CTA budget below the default grid launches at most max_ctas CTAs of
+    32 warps that walk every item: pool rows, the combine and the unit-weight
+    combine of the backward equal the oracle bit for bit, and padding rows
+    stay unwritten."""
+    E, R, B = 64, 8, 16
+    idx = W.edge_routing(kind, T, k, E, R, seed=T + k)
+    x = W.random_x(T, H, seed=T)
+    wt = W.random_weights(T, k, seed=k)
+    lay = oracle.layout(idx.numpy(), E, R, B)
+    h = sep.sep_layout(idx.cuda(), E, R, B, flags=sep.SEP_LAYOUT_SYNC_COUNTS)
+    try:
+        sep.sep_handle_set_max_ctas(h, max_ctas)
+        P = lay.num_pool_rows
+        valid = lay.pool_recv_token >= 0
+        recv = poisoned_bf16(P + 2, H)
+        sep.sep_dispatch(h, x.cuda(), recv)
+        want = oracle.dispatch_bf16(x, lay)
+        got = bf16_bits(recv)
+        np.testing.assert_array_equal(got[:P][valid], want[valid])
+        assert (got[:P][~valid] == POISON_BF16).all(), "a padding row was written"
+        assert (got[P:] == POISON_BF16).all(), "a row past the pool was written"
+        out = poisoned_bf16(T, H)
+        sep.sep_combine(h, recv, wt.cuda(), out)
+        check_combine(bf16_bits(out), oracle.combine(want, wt.numpy(), lay))
+        grad_x = poisoned_bf16(T, H)
+        sep.sep_combine_grads(h, recv, grad_x)
+        np.testing.assert_array_equal(bf16_bits(grad_x), oracle.combine_grads(want, lay))
+        sep.sep_handle_sync(h)
+    finally:
+        sep.sep_handle_free(h)
