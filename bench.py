@@ -71,6 +71,8 @@ def parse_args(argv=None):
                     choices=["layout", "layout_dispatch", "one_launch", "dispatch", "combine", "consumer", "gated",
                              "gather", "scatter", "backward", "ep"],
                     help="run one kernel family a few times, its producers finished first (for ncu); no timing")
+    ap.add_argument("--max-ctas", type=int, default=0,
+                    help="with --profile-case: the handle's CTA budget (sep_handle_set_max_ctas; 0 = default grid)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the borrowed-receive, backward-pair, combine-gate and scatter-combine measurements")
     return ap.parse_args(argv)
@@ -921,6 +923,18 @@ def ep_compare(w, dev, flush, peak_gbs, steps=100):
         for st in streams:
             main.wait_stream(st)
 
+    def ep_concurrent_phase(combine):
+        main = torch.cuda.current_stream()
+        for st in streams:
+            st.wait_stream(main)
+        for r in range(R):
+            if combine:
+                sep.sep_ep_combine(hs[r], pools, rows, deltas[r], ws[r], outs[r], err, stream=streams[r])
+            else:
+                sep.sep_ep_dispatch(hs[r], xs[r], r, deltas[r], pools, rows, err, stream=streams[r])
+        for st in streams:
+            main.wait_stream(st)
+
     idx_cat = torch.cat([sd["topk_idx"] for sd in shards]).to(dev)
     x_cat = torch.cat([sd["x"] for sd in shards]).to(dev)
     w_cat = torch.cat([sd["topk_weight"] for sd in shards]).to(dev)
@@ -932,10 +946,26 @@ def ep_compare(w, dev, flush, peak_gbs, steps=100):
         sep.sep_dispatch(h1, x_cat, pool1)
         sep.sep_combine(h1, pool1, w_cat, out1)
 
+    def graph_of(fn):
+        """fn captured once (side streams fork from and join back to the capture stream)."""
+        cap = torch.cuda.Stream(device=dev)
+        cap.wait_stream(torch.cuda.current_stream())
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            fn()
+        torch.cuda.synchronize()
+        return g
+
     ep_us = _time_arm(ep_step, steps, flush)
     ep_conc_us = _time_arm(ep_concurrent_step, steps, flush)
     single_us = _time_arm(single_step, steps, flush)
+    phase_us = [_time_arm(lambda c=c: ep_concurrent_phase(c), steps, flush) for c in (False, True)]
+    single_phase_us = [_time_arm(lambda: sep.sep_dispatch(h1, x_cat, pool1), steps, flush),
+                       _time_arm(lambda: sep.sep_combine(h1, pool1, w_cat, out1), steps, flush)]
+    graphs = [graph_of(f) for f in (ep_step, ep_concurrent_step, single_step)]
+    ep_g_us, ep_conc_g_us, single_g_us = (_time_arm(g.replay, steps, flush) for g in graphs)
     assert int(err.item()) == 0, "a row fell outside its owner's pool"
+    del graphs
     for h in hs + [h1]:
         sep.sep_handle_free(h)
     b = algorithmic_bytes(replace(w, T=R * Tr))
@@ -944,6 +974,12 @@ def ep_compare(w, dev, flush, peak_gbs, steps=100):
             "single_gpu_us": single_us,
             "ep_gbs": moved / (ep_us * 1e-6) / 1e9, "ep_frac": moved / (ep_us * 1e-6) / 1e9 / peak_gbs,
             "ep_concurrent_frac": moved / (ep_conc_us * 1e-6) / 1e9 / peak_gbs,
+            "phases_us": {"ep_concurrent_dispatch": phase_us[0], "ep_concurrent_combine": phase_us[1],
+                          "single_gpu_dispatch": single_phase_us[0], "single_gpu_combine": single_phase_us[1]},
+            "graph_replay": {"ep_us": ep_g_us, "ep_concurrent_us": ep_conc_g_us, "single_gpu_us": single_g_us,
+                             "ep_concurrent_frac": moved / (ep_conc_g_us * 1e-6) / 1e9 / peak_gbs,
+                             "note": "each arm captured once in a CUDA graph and replayed: the same kernels "
+                                     "without the host's per-launch cost (16 library calls per EP step)"},
             "note": "R ranks emulated on one GPU (2R launches: every rank's dispatch, then every rank's combine, "
                     "into / from the owners' pools); ep_us runs them one after another on one stream, "
                     "ep_concurrent_us runs each rank on its own stream with a join between the dispatches and "
@@ -1123,6 +1159,7 @@ def profile_case(args) -> int:
     d = W.make_inputs(w)
     x, idx, wt = d["x"].to(dev), d["topk_idx"].to(dev), d["topk_weight"].to(dev)
     h = sep.sep_layout(idx, w.E, w.R, w.B, flags=sep.SEP_LAYOUT_SYNC_COUNTS)
+    sep.sep_handle_set_max_ctas(h, args.max_ctas)
     info = h.info()
     rows = info.max_pool_rows
     recv, scales = sep.alloc_pool(h, w.H, w.payload, w.scale, rows=rows)

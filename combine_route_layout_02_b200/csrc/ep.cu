@@ -49,6 +49,7 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kUnroll = 4;
 constexpr int kRowBatch = 4;
+constexpr int kKMax = 8;             // combine: row pointers and weights held in registers
 
 __device__ __forceinline__ uint4 ld_stream(const uint4 *ptr)
 {
@@ -113,11 +114,22 @@ __device__ __forceinline__ void ep_publish_rows(const EpDispatchParams &p, int64
 }
 
 // bf16 dispatch into the owners' pools: a work item is (token, segment).
+// STAGED (no publication): each 2 KB step of x[t] goes through one of two
+// shared-memory stages of the warp and lane 0 issues one bulk store
+// (cp.async.bulk, no multicast) of the stage per destination row, as the
+// single-GPU dispatch does; a stage is rewritten once the bulk group that read
+// it two steps earlier has finished reading.  Otherwise the lanes store from
+// registers.
+constexpr int kStageVecs = 32 * kUnroll;         // one 2 KB step
+
+template <bool STAGED>
 __global__ void __launch_bounds__(kWarps * 32) ep_dispatch_kernel(EpDispatchParams p)
 {
+    __shared__ __align__(128) uint4 s_stage[STAGED ? kWarps : 1][2][STAGED ? kStageVecs : 1];
     grid_dependency_wait();
     allow_dependents();
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int stage = 0;
     const int V = p.H / 8;
     const int64_t items = p.T * p.segs;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -145,6 +157,30 @@ __global__ void __launch_bounds__(kWarps * 32) ep_dispatch_kernel(EpDispatchPara
                 const int v = v0 + u * 32 + lane;
                 buf[u] = v < v_end ? ld_stream(src + v) : make_uint4(0, 0, 0, 0);
             }
+            if (STAGED) {
+                const int n = min(kStageVecs, v_end - v0);
+                if (lane == 0)                               // the stage's previous bulk reads are done
+                    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                __syncwarp();
+                uint4 *st = s_stage[STAGED ? warp : 0][stage];
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u)
+                    st[u * 32 + lane] = buf[u];
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                const uint32_t saddr = static_cast<uint32_t>(__cvta_generic_to_shared(st));
+                for (int j = 0; j < p.k; ++j) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(
+                        __shfl_sync(kFullMask, reinterpret_cast<unsigned long long>(my_dst), j));
+                    if (dst != nullptr && lane == 0)
+                        asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                                     ::"l"(dst + v0), "r"(saddr), "r"(n * 16) : "memory");
+                }
+                if (lane == 0)
+                    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                stage ^= 1;
+                continue;
+            }
             for (int j = 0; j < p.k; ++j) {
                 uint4 *dst = reinterpret_cast<uint4 *>(
                     __shfl_sync(kFullMask, reinterpret_cast<unsigned long long>(my_dst), j));
@@ -158,9 +194,11 @@ __global__ void __launch_bounds__(kWarps * 32) ep_dispatch_kernel(EpDispatchPara
                 }
             }
         }
-        if (p.tile_ready[0] != nullptr)                  // publication
+        if (!STAGED && p.tile_ready[0] != nullptr)       // publication
             ep_publish_rows(p, t * p.k + lane, my_row, my_owner, lane);
     }
+    if (STAGED && lane == 0)
+        asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // FP8 dispatch into the owners' pools: a work item is (token, segment of
@@ -372,8 +410,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 }
 
 // Combine from the owners' expert outputs: a warp owns (token, segment); the
-// k row pointers and weights are broadcast into registers once; fp32 sums in
-// ascending j, as the single-GPU combine.
+// k row pointers and weights are broadcast into registers once (k <= 8) or
+// per batch of rows; fp32 sums in ascending j, as the single-GPU combine.
+// Tokens are visited in descending order, as there: a dispatch that ran just
+// before wrote the highest tokens' rows last.
 __global__ void __launch_bounds__(kWarps * 32) ep_combine_kernel(EpCombineParams p)
 {
     grid_dependency_wait();
@@ -383,8 +423,9 @@ __global__ void __launch_bounds__(kWarps * 32) ep_combine_kernel(EpCombineParams
     const int64_t items = p.T * p.segs;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     for (int64_t it = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; it < items; it += nwarps) {
-        const int64_t t = it / p.segs;
-        const int s = (int)(it - t * p.segs);
+        const int64_t q = it / p.segs;
+        const int64_t t = p.T - 1 - q;
+        const int s = (int)(it - q * p.segs);
         const int v_begin = s * p.seg_len;
         const int v_end = min(V, v_begin + p.seg_len);
         int my_owner = 0;
@@ -392,6 +433,37 @@ __global__ void __launch_bounds__(kWarps * 32) ep_combine_kernel(EpCombineParams
         const uint4 *my_src = my_row >= 0 ? static_cast<const uint4 *>(p.y_pools[my_owner]) + my_row * V : nullptr;
         const float my_w = lane < p.k ? __ldg(p.w + t * p.k + lane) : 0.f;
         uint4 *out = static_cast<uint4 *>(p.out) + t * V;
+        if (p.k <= kKMax) {
+            const uint4 *srcs[kKMax];
+            float ws[kKMax];
+#pragma unroll
+            for (int j = 0; j < kKMax; ++j) {
+                srcs[j] = reinterpret_cast<const uint4 *>(
+                    __shfl_sync(kFullMask, reinterpret_cast<unsigned long long>(my_src), j));
+                ws[j] = __shfl_sync(kFullMask, my_w, j);
+            }
+            for (int v = v_begin + lane; v < v_end; v += 32) {
+                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int j0 = 0; j0 < kKMax; j0 += kRowBatch) {
+                    uint4 buf[kRowBatch];
+#pragma unroll
+                    for (int u = 0; u < kRowBatch; ++u)
+                        buf[u] = srcs[j0 + u] != nullptr ? ld_stream(srcs[j0 + u] + v) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                    for (int u = 0; u < kRowBatch; ++u)
+                        if (srcs[j0 + u] != nullptr) {
+                            accumulate_word(acc[0], acc[1], buf[u].x, ws[j0 + u]);
+                            accumulate_word(acc[2], acc[3], buf[u].y, ws[j0 + u]);
+                            accumulate_word(acc[4], acc[5], buf[u].z, ws[j0 + u]);
+                            accumulate_word(acc[6], acc[7], buf[u].w, ws[j0 + u]);
+                        }
+                }
+                out[v] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                    pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+            }
+            continue;
+        }
         for (int v0 = v_begin; v0 < v_end; v0 += 32) {
             const int v = v0 + lane;
             const bool act = v < v_end;
@@ -445,7 +517,10 @@ cudaError_t launch_ep_dispatch(EpDispatchParams p, cudaStream_t s, int num_sms)
         p.seg_len = p.H / 8;
     }
     const int64_t items = p.T * p.segs;
-    return launch_kernel(ep_dispatch_kernel, dim3((int)((items + kWarps - 1) / kWarps)), dim3(kWarps * 32), 0, s, p);
+    const dim3 grid((int)((items + kWarps - 1) / kWarps)), block(kWarps * 32);
+    if (p.tile_ready[0] == nullptr && p.seg_len % kStageVecs == 0)
+        return launch_kernel(ep_dispatch_kernel<true>, grid, block, 0, s, p);
+    return launch_kernel(ep_dispatch_kernel<false>, grid, block, 0, s, p);
 }
 
 cudaError_t launch_ep_dispatch_fp8(EpDispatchParams p, cudaStream_t s, int num_sms)
@@ -494,7 +569,9 @@ cudaError_t launch_ep_combine(EpCombineParams p, cudaStream_t s, int num_sms)
 cudaError_t preload_ep_kernels()
 {
     cudaFuncAttributes a;
-    cudaError_t e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(ep_dispatch_kernel));
+    cudaError_t e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(ep_dispatch_kernel<false>));
+    if (e == cudaSuccess)
+        e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(ep_dispatch_kernel<true>));
     if (e == cudaSuccess)
         e = cudaFuncGetAttributes(&a, reinterpret_cast<const void *>(ep_plan_kernel));
     if (e == cudaSuccess)
