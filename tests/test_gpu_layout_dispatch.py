@@ -273,3 +273,23 @@ def test_layout_flags_pass_through(flags):
         _check_pool(lay, d["x"], recv, sc, "fp8", "ue8m0")
     finally:
         sep.sep_handle_free(h)
+
+
+@pytest.mark.parametrize("payload,scale", [("bf16", "none"), ("fp8", "ue8m0")])
+def test_cta_budget_on_the_two_launches(payload, scale):
+    """A CTA budget on the handle bounds the dispatch launch of
+    sep_layout_dispatch: the same two launches and the same pool."""
+    w = W.scaled(W.WORKLOADS["train8k"], 900)
+    d = W.make_inputs(w)
+    h = sep.sep_handle_create(w.T, w.k, w.E, w.R, w.B)
+    try:
+        sep.sep_handle_set_max_ctas(h, 5)
+        _, lay, launches, recv = _run(d["topk_idx"], d["x"], w.E, w.R, w.B, payload, scale, handle=h, flags=0)
+        assert launches == 2
+        if payload == "bf16":
+            out = torch.empty(w.T, w.H, dtype=torch.bfloat16, device="cuda")
+            sep.sep_combine(h, recv, d["topk_weight"].cuda(), out)
+            want = oracle.combine(oracle.dispatch_bf16(d["x"], lay), d["topk_weight"].numpy(), lay)
+            check_combine(bf16_bits(out), want)
+    finally:
+        sep.sep_handle_free(h)

@@ -703,3 +703,43 @@ def test_budget_grids_match_the_oracle(kind, T, k, H, max_ctas):
         sep.sep_handle_sync(h)
     finally:
         sep.sep_handle_free(h)
+
+
+def test_cta_budget_with_publication_and_an_empty_routing():
+    """Under a CTA budget the publishing dispatch still publishes every tile
+    once its rows have landed (the reference consumer, launched first on
+    another stream, copies them all), and a routing of no tokens launches
+    nothing."""
+    w, d = _inputs(W.WORKLOADS["streaming"], 4096, 512)
+    lay = oracle.layout(d["topk_idx"].numpy(), w.E, w.R, w.B)
+    h = sep.sep_layout(d["topk_idx"].cuda(), w.E, w.R, w.B)
+    try:
+        sep.sep_handle_set_max_ctas(h, 6)
+        info = h.info()
+        rows, NT = info.max_pool_rows, lay.num_tiles
+        want = oracle.dispatch_bf16(d["x"], lay)
+        valid = lay.pool_recv_token >= 0
+        tile_ready = torch.zeros(info.max_tiles, dtype=torch.int32, device="cuda")
+        status = torch.zeros(2, dtype=torch.int32, device="cuda")
+        recv, dst = poisoned_bf16(rows, w.H), poisoned_bf16(rows, w.H)
+        _streaming_round(h, lay, d["x"].cuda(), recv, tile_ready, 5, dst, status, consumer_first=True)
+        assert status.cpu().tolist() == [0, 0]
+        assert (tile_ready.cpu().numpy()[:NT] == 5).all()
+        got = bf16_bits(dst)[:lay.num_pool_rows]
+        np.testing.assert_array_equal(got[valid], want[valid])
+        assert (got[~valid] == POISON_BF16).all()
+    finally:
+        sep.sep_handle_free(h)
+    h = sep.sep_layout(torch.zeros(0, 4, dtype=torch.int32, device="cuda"), 16, 4, 16, flags=sep.SEP_LAYOUT_SYNC_COUNTS)
+    try:
+        sep.sep_handle_set_max_ctas(h, 1)
+        recv = poisoned_bf16(1, 64)
+        n0 = sep.sep_launch_count()
+        sep.sep_dispatch(h, torch.zeros(0, 64, dtype=torch.bfloat16, device="cuda"), recv)
+        sep.sep_combine(h, recv, torch.zeros(0, 4, device="cuda"), torch.empty(0, 64, dtype=torch.bfloat16,
+                                                                                device="cuda"))
+        assert sep.sep_launch_count() == n0
+        torch.cuda.synchronize()
+        assert (bf16_bits(recv) == POISON_BF16).all()
+    finally:
+        sep.sep_handle_free(h)
