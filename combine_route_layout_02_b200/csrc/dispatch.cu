@@ -119,8 +119,12 @@ __global__ void __launch_bounds__(WARPS * 32) dispatch_bf16_kernel(DispatchParam
 }
 
 // fp8: a work item is (token, segment of seg_len 512-channel iterations).
+// The default grid's 8-warp CTAs are held to 40 registers, so 6 of them fit
+// an SM (42 registers, allocated as 48, allowed 5): more warps waiting on x
+// at once (prefill_skew dispatch 193.6 against 194.0 us, decode step 26.2
+// against 26.8 us).
 template <int SCALE, bool PUBLISH, int WARPS = kWarps>
-__global__ void __launch_bounds__(WARPS * 32) dispatch_fp8_kernel(DispatchParams p)
+__global__ void __launch_bounds__(WARPS * 32, WARPS == kWarps ? 6 : 1) dispatch_fp8_kernel(DispatchParams p)
 {
     grid_dependency_wait();
     allow_dependents();
@@ -292,11 +296,13 @@ cudaError_t launch_fp8(const DispatchParams &p, cudaStream_t s, dim3 grid)
 // item, so the items divide finely over the waves of CTAs (measured faster
 // than whole rows per warp).  With tile publication a row stays on one warp
 // where possible, since every item pays a fence and one arrival per row.  FP8
-// steps are 512 channels, and a row splits over up to 7 warps.
+// steps are 512 channels, and a row splits over up to 14 warps (prefill_skew,
+// H = 7168: one step per warp, so no warp waits on a second load of x after
+// its first step's stores; dispatch 194.0 against 206.3 us with up to 7).
 constexpr int64_t kStepVecs = 128;
 constexpr int64_t kMinSegs = 1 << 20;
 constexpr int64_t kPublishMinSegs = 1;
-constexpr int64_t kFp8MinSegs = 7;
+constexpr int64_t kFp8MinSegs = 14;
 
 cudaError_t launch_dispatch(DispatchParams p, int payload, cudaStream_t s, int num_sms)
 {
