@@ -607,7 +607,8 @@ def run_ours(args, rank: int, world: int, local: int) -> dict | None:
     scatter = (scatter_compare(w, h, idx, wt, y, None if flush is None else flush.zero_, peaks["hbm_gbs"])
                if want("scatter") else None)
     ep = (ep_compare(w, dev, None if flush is None else flush.zero_, peaks["hbm_gbs"])
-          if w.payload == "bf16" and not w.streaming and want("ep") and w.T % w.R == 0 else None)
+          if not w.streaming and want("ep") and w.T % w.R == 0 and (w.payload == "bf16" or w.T // w.R >= 128)
+          else None)
     budget = (budget_compare(w, h, x, idx, recv, scales, y, wt, None if flush is None else flush.zero_, peaks["hbm_gbs"])
               if not w.streaming and want("budget") else None)
     overlap = (overlap_compare(w, h, x, idx, recv, y, wt, None if flush is None else flush.zero_)
@@ -885,23 +886,43 @@ def ep_compare(w, dev, flush, peak_gbs, steps=100):
     import torch
     import combine_route_layout_02_b200 as sep
     R, Tr = w.R, w.T // w.R
+    fp8 = w.payload != "bf16"
     shards = [W.make_inputs(replace(w, T=Tr, seed=w.seed + 7919 * (r + 1))) for r in range(R)]
     hs = [sep.sep_layout(sd["topk_idx"].to(dev), w.E, R, w.B, flags=sep.SEP_LAYOUT_SYNC_COUNTS) for sd in shards]
     counts = np.stack([h.view("expert_counts").cpu().numpy() for h in hs]).astype(np.int32)
     plans = [sep.sep_ep_plan(counts, r, w.B) for r in range(R)]
     rows = [int(v) for v in plans[0]["owner_rows"]]
-    pools = [torch.empty(max(n, 1), w.H, dtype=torch.bfloat16, device=dev) for n in rows]
+    y_src = W.random_x(61, w.H, seed=w.seed + 7).to(dev) if fp8 else None
+
+    def y_rows(n):
+        """An FP8 workload's expert outputs: a seeded bf16 pool of n rows."""
+        return y_src[torch.arange(max(n, 1), device=dev) % 61].contiguous()
+
+    pools = [torch.empty(max(n, 1), w.H, dtype=torch.uint8 if fp8 else torch.bfloat16, device=dev) for n in rows]
+    sdt = torch.uint8 if w.scale == "ue8m0" else torch.float32
+    scale_pools = [torch.empty(max(n, 1), w.H // 128, dtype=sdt, device=dev) for n in rows] if fp8 else None
+    y_pools = [y_rows(n) for n in rows] if fp8 else pools
     deltas = [torch.from_numpy(p["delta"]).to(dev) for p in plans]
     xs = [sd["x"].to(dev) for sd in shards]
     ws = [sd["topk_weight"].to(dev) for sd in shards]
     outs = [torch.empty(Tr, w.H, dtype=torch.bfloat16, device=dev) for _ in range(R)]
     err = torch.zeros(1, dtype=torch.int32, device=dev)
 
+    def ep_dispatch(r, stream=None):
+        if fp8:
+            sep.sep_ep_dispatch_fp8(hs[r], xs[r], r, deltas[r], pools, scale_pools, rows, err, scale=w.scale,
+                                    stream=stream)
+        else:
+            sep.sep_ep_dispatch(hs[r], xs[r], r, deltas[r], pools, rows, err, stream=stream)
+
+    def ep_combine(r, stream=None):
+        sep.sep_ep_combine(hs[r], y_pools, rows, deltas[r], ws[r], outs[r], err, stream=stream)
+
     def ep_step():
         for r in range(R):
-            sep.sep_ep_dispatch(hs[r], xs[r], r, deltas[r], pools, rows, err)
+            ep_dispatch(r)
         for r in range(R):
-            sep.sep_ep_combine(hs[r], pools, rows, deltas[r], ws[r], outs[r], err)
+            ep_combine(r)
 
     streams = [torch.cuda.Stream(device=dev) for _ in range(R)]
 
@@ -916,10 +937,10 @@ def ep_compare(w, dev, flush, peak_gbs, steps=100):
         for st in streams:
             st.wait_stream(main)
         for r in range(R):
-            sep.sep_ep_dispatch(hs[r], xs[r], r, deltas[r], pools, rows, err, stream=streams[r])
+            ep_dispatch(r, streams[r])
         join(main)
         for r in range(R):
-            sep.sep_ep_combine(hs[r], pools, rows, deltas[r], ws[r], outs[r], err, stream=streams[r])
+            ep_combine(r, streams[r])
         for st in streams:
             main.wait_stream(st)
 
@@ -929,9 +950,9 @@ def ep_compare(w, dev, flush, peak_gbs, steps=100):
             st.wait_stream(main)
         for r in range(R):
             if combine:
-                sep.sep_ep_combine(hs[r], pools, rows, deltas[r], ws[r], outs[r], err, stream=streams[r])
+                ep_combine(r, streams[r])
             else:
-                sep.sep_ep_dispatch(hs[r], xs[r], r, deltas[r], pools, rows, err, stream=streams[r])
+                ep_dispatch(r, streams[r])
         for st in streams:
             main.wait_stream(st)
 
@@ -939,12 +960,20 @@ def ep_compare(w, dev, flush, peak_gbs, steps=100):
     x_cat = torch.cat([sd["x"] for sd in shards]).to(dev)
     w_cat = torch.cat([sd["topk_weight"] for sd in shards]).to(dev)
     h1 = sep.sep_layout(idx_cat, w.E, R, w.B, flags=sep.SEP_LAYOUT_SYNC_COUNTS)
-    pool1 = torch.empty(h1.info().num_pool_rows, w.H, dtype=torch.bfloat16, device=dev)
+    P1 = h1.info().num_pool_rows
+    pool1, scales1 = sep.alloc_pool(h1, w.H, w.payload, w.scale, rows=max(P1, 1))
+    y1 = y_rows(P1) if fp8 else pool1
     out1 = torch.empty(R * Tr, w.H, dtype=torch.bfloat16, device=dev)
 
+    def single_dispatch():
+        sep.sep_dispatch(h1, x_cat, pool1, payload=w.payload, scale=w.scale, recv_scales=scales1)
+
+    def single_combine():
+        sep.sep_combine(h1, y1, w_cat, out1)
+
     def single_step():
-        sep.sep_dispatch(h1, x_cat, pool1)
-        sep.sep_combine(h1, pool1, w_cat, out1)
+        single_dispatch()
+        single_combine()
 
     def graph_of(fn):
         """fn captured once (side streams fork from and join back to the capture stream)."""
@@ -960,8 +989,7 @@ def ep_compare(w, dev, flush, peak_gbs, steps=100):
     ep_conc_us = _time_arm(ep_concurrent_step, steps, flush)
     single_us = _time_arm(single_step, steps, flush)
     phase_us = [_time_arm(lambda c=c: ep_concurrent_phase(c), steps, flush) for c in (False, True)]
-    single_phase_us = [_time_arm(lambda: sep.sep_dispatch(h1, x_cat, pool1), steps, flush),
-                       _time_arm(lambda: sep.sep_combine(h1, pool1, w_cat, out1), steps, flush)]
+    single_phase_us = [_time_arm(single_dispatch, steps, flush), _time_arm(single_combine, steps, flush)]
     graphs = [graph_of(f) for f in (ep_step, ep_concurrent_step, single_step)]
     ep_g_us, ep_conc_g_us, single_g_us = (_time_arm(g.replay, steps, flush) for g in graphs)
     assert int(err.item()) == 0, "a row fell outside its owner's pool"

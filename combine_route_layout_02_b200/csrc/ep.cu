@@ -157,12 +157,12 @@ __global__ void __launch_bounds__(kWarps * 32) ep_dispatch_kernel(EpDispatchPara
                 const int v = v0 + u * 32 + lane;
                 buf[u] = v < v_end ? ld_stream(src + v) : make_uint4(0, 0, 0, 0);
             }
-            if (STAGED) {
+            if constexpr (STAGED) {
                 const int n = min(kStageVecs, v_end - v0);
                 if (lane == 0)                               // the stage's previous bulk reads are done
                     asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
                 __syncwarp();
-                uint4 *st = s_stage[STAGED ? warp : 0][stage];
+                uint4 *st = s_stage[warp][stage];
 #pragma unroll
                 for (int u = 0; u < kUnroll; ++u)
                     st[u * 32 + lane] = buf[u];
@@ -179,18 +179,18 @@ __global__ void __launch_bounds__(kWarps * 32) ep_dispatch_kernel(EpDispatchPara
                 if (lane == 0)
                     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
                 stage ^= 1;
-                continue;
-            }
-            for (int j = 0; j < p.k; ++j) {
-                uint4 *dst = reinterpret_cast<uint4 *>(
-                    __shfl_sync(kFullMask, reinterpret_cast<unsigned long long>(my_dst), j));
-                if (dst == nullptr)
-                    continue;                            // warp-uniform
+            } else {
+                for (int j = 0; j < p.k; ++j) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(
+                        __shfl_sync(kFullMask, reinterpret_cast<unsigned long long>(my_dst), j));
+                    if (dst == nullptr)
+                        continue;                        // warp-uniform
 #pragma unroll
-                for (int u = 0; u < kUnroll; ++u) {
-                    const int v = v0 + u * 32 + lane;
-                    if (v < v_end)
-                        dst[v] = buf[u];
+                    for (int u = 0; u < kUnroll; ++u) {
+                        const int v = v0 + u * 32 + lane;
+                        if (v < v_end)
+                            dst[v] = buf[u];
+                    }
                 }
             }
         }
@@ -204,6 +204,10 @@ __global__ void __launch_bounds__(kWarps * 32) ep_dispatch_kernel(EpDispatchPara
 // FP8 dispatch into the owners' pools: a work item is (token, segment of
 // 512-channel iterations); each token is quantised once (the single-GPU
 // kernel's arithmetic) and its codes and scales stored to the k owners' rows.
+// Rows split over up to 7 warps: unlike the single-GPU kernel, every item
+// resolves its rows' owners through three dependent loads, and splitting
+// over up to 14 warps with 6 CTAs per SM measured slower here (8 emulated
+// prefill_skew ranks on their own streams: dispatches 221.6 against 212.0 us).
 template <int SCALE>
 __global__ void __launch_bounds__(kWarps * 32) ep_dispatch_fp8_kernel(EpDispatchParams p)
 {
