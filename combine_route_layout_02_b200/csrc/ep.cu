@@ -20,9 +20,11 @@
 // computed on the host from the exchanged counts (sep_ep_plan).
 //
 // The dispatch writes each token row straight into the owner's pool through
-// the owner's pointer (a peer pointer on another GPU, plain stores over
-// NVLink; no TMA, no multicast) together with the owner's receive map
-// (token, rank, slot); the owner marks its own padding rows.
+// the owner's pointer (a peer pointer on another GPU: stores over NVLink;
+// bf16 rows without publication go as untiled bulk stores from shared
+// memory, everything else from registers; no tensor map, no multicast)
+// together with the owner's receive map (token, rank, slot); the owner marks
+// its own padding rows.
 //
 // The plan can also be computed on the GPU from the exchanged counts
 // (ep_plan_kernel), so a step needs no copy to the host.  With publication

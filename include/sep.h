@@ -496,8 +496,11 @@ SEP_API sep_status sep_gather_rows(const sep_recv_view *view, void *dst, int64_t
  * the rows are ordered by (source rank, token, slot): exactly owner o's segment
  * of the single-GPU layout of all ranks' tokens concatenated in rank order.
  * A pool is any device memory of this or a peer GPU (a peer pointer from CUDA
- * IPC or symmetric memory); rows are written and read with plain stores and
- * loads (no TMA, no multicast).  Between the dispatches of all ranks and the
+ * IPC or symmetric memory); rows are written by stores from registers, or
+ * (sep_ep_dispatch, which publishes nothing) by untiled bulk stores from
+ * shared memory, and read with plain loads: no tensor map, no multicast.
+ * Only the one-GPU emulation has run here: bulk stores to a peer's pool are
+ * not tested across GPUs.  Between the dispatches of all ranks and the
  * owners' expert compute, and between that and the combines, the caller
  * synchronises the ranks (a barrier or a collective).
  */
