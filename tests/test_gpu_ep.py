@@ -83,6 +83,7 @@ def _oracle(idx, xs, ws, E, R, B, k):
     (2, 8, 128, 2, 3072, [1000, 1000], 0.0),
     (3, 6, 8, 3, 24, [5, 1, 9], 0.5),
     (2, 8, 16, 2, 65536, [20, 13], 0.1),
+    (4, 32, 16, 12, 136, [50, 20, 0, 33], 0.1),   # k > 8: the combine's batched-pointer path
 ])
 def test_ep_dispatch_and_combine_match_the_concatenated_oracle(R, E, B, k, H, Ts, masked):
     idx, xs, ws, rows, pools, maps, outs, err = _run(R, E, B, k, H, Ts, seed=R * 1000 + H, masked=masked)
