@@ -31,8 +31,6 @@
 #include <atomic>
 #include <mutex>
 
-#include <cooperative_groups.h>
-
 #include "fp8_quant.cuh"
 #include "sep_internal.cuh"
 
@@ -425,14 +423,7 @@ constexpr bool kTable16 = true;
 // Chunk c of the G = p.num_wchunks chunks of the layout, run by one CTA
 // (phases A to D above).  sm: the dynamic shared memory of
 // layout_smem_bytes(); false if its grid barrier gave up.
-// CLUSTER: the G CTAs are one thread-block cluster.  Each keeps its chunk's
-// per-expert counts in its own shared memory, and after one cluster barrier
-// every CTA sums all G rows through distributed shared memory (its totals and
-// its prefix over earlier chunks); a second cluster barrier keeps every CTA
-// (and its row) alive until all have read.  No chunk table in global memory
-// and no grid barrier: the exchange costs two hardware barriers and G
-// shared-memory loads per expert.  Every thread reaches both barriers.
-template <typename IdxT, int WARPS = kWarps, bool CLUSTER = false>
+template <typename IdxT, int WARPS = kWarps>
 __device__ bool layout_chunk(const LayoutParams &p, const int c, const int G, int32_t *sm, int &s_flag,
                              int *s_part)
 {
@@ -472,29 +463,6 @@ __device__ bool layout_chunk(const LayoutParams &p, const int c, const int G, in
             s_pre[e] = 0;
         }
         __syncthreads();
-    } else if (CLUSTER) {
-        int32_t *s_row = s_red;                          // this chunk's counts, read by the whole cluster
-        for (int e = tid; e < E; e += blockDim.x) {
-            int sum = 0;
-#pragma unroll
-            for (int w = 0; w < WARPS; ++w)
-                sum += s_cnt[w * E + e];
-            s_row[e] = sum;
-        }
-        cooperative_groups::cluster_group cluster = cooperative_groups::this_cluster();
-        cluster.sync();
-        for (int e = tid; e < E; e += blockDim.x) {
-            int t = 0, b = 0;
-            for (int r = 0; r < G; ++r) {
-                const int v = cluster.map_shared_rank(s_row, r)[e];
-                t += v;
-                if (r < c)
-                    b += v;
-            }
-            s_tot[e] = t;
-            s_pre[e] = b;
-        }
-        cluster.sync();
     } else {
     if (kTable16 && WARPS >= 8) {
         // 16-bit entries (a chunk holds at most 16 384 assignments): half the bytes
@@ -793,25 +761,10 @@ __global__ void __launch_bounds__(WARPS * 32) layout_fused_kernel(LayoutParams p
     extern __shared__ __align__(16) int32_t sm[];
     __shared__ int s_flag;
     __shared__ int s_part[WARPS];
-    allow_dependents();
+    grid_dependency_wait();                              // launched dependent (one CTA): the previous kernel's
+    allow_dependents();                                  // writes first; a no-op for a cooperative launch
     layout_chunk<IdxT, WARPS>(p, blockIdx.x, gridDim.x, sm, s_flag, s_part);
 }
-
-// The narrow layout as one thread-block cluster (at most 16 CTAs): the chunk
-// counts are exchanged through distributed shared memory (layout_chunk,
-// CLUSTER).  The cluster's CTAs are co-scheduled by the hardware, so no
-// cooperative launch is needed.
-template <typename IdxT, int WARPS>
-__global__ void __launch_bounds__(WARPS * 32) layout_cluster_kernel(LayoutParams p)
-{
-    extern __shared__ __align__(16) int32_t sm[];
-    __shared__ int s_flag;
-    __shared__ int s_part[WARPS];
-    allow_dependents();
-    layout_chunk<IdxT, WARPS, true>(p, (int)cooperative_groups::this_cluster().block_rank(), gridDim.x, sm, s_flag,
-                                    s_part);
-}
-constexpr int kMaxClusterChunks = 16;
 
 // Routings of 1025 to 4096 assignments (a decode step) in narrower chunks:
 // kNarrowWarps warps per CTA, one 32-entry round per warp, so more CTAs (and
@@ -1097,55 +1050,6 @@ cudaError_t launch_layout_t(const LayoutParams &p, cudaStream_t s)
                 return e;
             narrow_attr[dev].store(true, std::memory_order_release);
         }
-        cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
-        if (cudaStreamIsCapturing(s, &capture) != cudaSuccess)
-            return cudaGetLastError();
-        if (capture == cudaStreamCaptureStatusActive && q.num_wchunks <= kMaxClusterChunks) {
-            // while a CUDA graph is captured: one cluster of num_wchunks CTAs, when the GPU can host it
-            // (else the cooperative launch below).  Replayed from a graph, the cooperative layout costs
-            // about 1.5 us more than launched on a stream and the cluster form does not (decode graph
-            // replay 26.5 against 27.9 us); launched on a stream the cooperative form is the faster
-            // (decode step 26.2 against 26.6 us), so streams keep it.
-            using K = void (*)(LayoutParams);
-            const K kernel = layout_cluster_kernel<IdxT, kNarrowWarps>;
-            static std::atomic<bool> cluster_attr[64] = {};
-            if (!cluster_attr[dev].load(std::memory_order_acquire)) {
-                cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
-                if (e == cudaSuccess)
-                    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-                if (e != cudaSuccess)
-                    return e;
-                cluster_attr[dev].store(true, std::memory_order_release);
-            }
-            cudaLaunchConfig_t cfg = {};
-            cfg.gridDim = dim3(q.num_wchunks);
-            cfg.blockDim = dim3(kNarrowWarps * 32);
-            cfg.dynamicSmemBytes = smem;
-            cfg.stream = s;
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = (unsigned)q.num_wchunks;
-            attr[0].val.clusterDim.y = 1;
-            attr[0].val.clusterDim.z = 1;
-            cfg.attrs = attr;
-            cfg.numAttrs = 1;
-            // whether the GPU can host a cluster of this size: asked once per device and size (the query
-            // costs host time on every launch otherwise); 0 unknown, 1 yes, 2 no
-            static std::atomic<int> hostable[64][kMaxClusterChunks + 1] = {};
-            int ok = hostable[dev][q.num_wchunks].load(std::memory_order_acquire);
-            if (ok == 0) {
-                int clusters = 0;
-                const cudaError_t qe = cudaOccupancyMaxActiveClusters(&clusters, kernel, &cfg);
-                if (qe != cudaSuccess)
-                    (void)cudaGetLastError();            // this query's own error: the launch falls back
-                ok = qe == cudaSuccess && clusters >= 1 ? 1 : 2;
-                hostable[dev][q.num_wchunks].store(ok, std::memory_order_release);
-            }
-            if (ok == 1) {
-                count_launch();
-                return cudaLaunchKernelEx(&cfg, kernel, q);
-            }
-        }
         sms = device_sm_count();
         per_sm = layout_blocks_per_sm(dev, reinterpret_cast<const void *>(layout_fused_kernel<IdxT, kNarrowWarps>),
                                       kNarrowWarps * 32, smem);
@@ -1175,6 +1079,8 @@ cudaError_t launch_layout_t(const LayoutParams &p, cudaStream_t s)
                 return e;
             attr_set[dev].store(true, std::memory_order_release);
         }
+        if (chunks == 1)                                 // one CTA: no grid barrier, so an ordinary dependent launch
+            return launch_kernel(layout_fused_kernel<IdxT>, dim3(1), dim3(kFusedThreads), smem_fused, s, p);
         sms = device_sm_count();
         per_sm = layout_blocks_per_sm(dev, reinterpret_cast<const void *>(layout_fused_kernel<IdxT>), kFusedThreads,
                                       smem_fused);
@@ -1258,8 +1164,6 @@ cudaError_t preload_layout_kernels()
                        reinterpret_cast<const void *>(layout_fused_kernel<long long>),
                        reinterpret_cast<const void *>(layout_fused_kernel<int, kNarrowWarps>),
                        reinterpret_cast<const void *>(layout_fused_kernel<long long, kNarrowWarps>),
-                       reinterpret_cast<const void *>(layout_cluster_kernel<int, kNarrowWarps>),
-                       reinterpret_cast<const void *>(layout_cluster_kernel<long long, kNarrowWarps>),
                        reinterpret_cast<const void *>(layout_count_kernel<int>),
                        reinterpret_cast<const void *>(layout_count_kernel<long long>),
                        reinterpret_cast<const void *>(layout_scan_kernel),

@@ -5,10 +5,9 @@ new routings, activations and weights copied into the captured input buffers
 between replays.  Nothing on the device may depend on host state that a replay
 does not refresh: the single-launch layout's grid barrier advances its counter
 by a fixed window per launch instead of by the host's epoch, so replays (which
-repeat the captured epoch) still synchronise.  Captured, a decode-size layout
-of at most 16 chunks runs as one thread-block cluster instead of a cooperative
-launch.  Every replay's layout arrays and output are checked against the
-oracle bit for bit.
+repeat the captured epoch) still synchronise; a one-chunk layout (tiny) is an
+ordinary dependent launch.  Every replay's layout arrays and output are checked
+against the oracle bit for bit.
 """
 import numpy as np
 import pytest
@@ -23,8 +22,8 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("name,T", [("tiny", None), ("train8k", 2000), ("decode", None),
-                                    ("decode", 150),   # 1200 assignments: a cluster of 10 CTAs
-                                    ("decode", 400)])  # 3200: 25 chunks, more than a cluster holds
+                                    ("decode", 150),   # 1200 assignments: 10 narrow chunks
+                                    ("decode", 400)])  # 3200 assignments: 25 narrow chunks
 def test_forward_step_replays_from_a_cuda_graph(name, T):
     w = W.WORKLOADS[name]
     w = W.scaled(w, T) if T else w
