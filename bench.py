@@ -69,7 +69,7 @@ def parse_args(argv=None):
                     help="comma list of the measurements taken after the timed region")
     ap.add_argument("--profile-case", default=None,
                     choices=["layout", "layout_dispatch", "one_launch", "dispatch", "combine", "consumer", "gated",
-                             "gather", "scatter", "backward", "ep"],
+                             "gather", "scatter", "backward", "ep", "ep_plain"],
                     help="run one kernel family a few times, its producers finished first (for ncu); no timing")
     ap.add_argument("--max-ctas", type=int, default=0,
                     help="with --profile-case: the handle's CTA budget (sep_handle_set_max_ctas; 0 = default grid)")
@@ -1250,6 +1250,39 @@ def profile_case(args) -> int:
                 sep.sep_ep_combine(hs[r], dsts, cap, plans[r]["delta"], ws[r], outs[r], err)
             torch.cuda.synchronize()
             assert status.cpu().tolist() == [0, 0] and int(err.item()) == 0
+        for hh in hs:
+            sep.sep_handle_free(hh)
+    elif case == "ep_plain":
+        # the expert-parallel dispatch without publication (bf16: staged bulk stores; FP8: codes and scales) and
+        # the combine from the owners' pools (an FP8 workload's combine reads seeded bf16 expert outputs)
+        import numpy as np
+        R, Tr = w.R, w.T // w.R
+        fp8 = w.payload != "bf16"
+        shards = [W.make_inputs(replace(w, T=Tr, seed=w.seed + 7919 * (r + 1))) for r in range(R)]
+        hs = [sep.sep_layout(sd["topk_idx"].to(dev), w.E, R, w.B, flags=sep.SEP_LAYOUT_SYNC_COUNTS) for sd in shards]
+        counts = np.stack([hh.view("expert_counts").cpu().numpy() for hh in hs]).astype(np.int32)
+        plans = [sep.sep_ep_plan(counts, r, w.B) for r in range(R)]
+        prow = [max(int(v), 1) for v in plans[0]["owner_rows"]]
+        pools = [torch.empty(n, w.H, dtype=torch.uint8 if fp8 else torch.bfloat16, device=dev) for n in prow]
+        sdt = torch.uint8 if w.scale == "ue8m0" else torch.float32
+        scale_pools = [torch.empty(n, w.H // 128, dtype=sdt, device=dev) for n in prow] if fp8 else None
+        y_src = W.random_x(61, w.H, seed=w.seed + 7).to(dev) if fp8 else None
+        y_pools = ([y_src[torch.arange(n, device=dev) % 61].contiguous() for n in prow] if fp8 else pools)
+        deltas = [torch.from_numpy(pl["delta"]).to(dev) for pl in plans]
+        xs = [sd["x"].to(dev) for sd in shards]
+        ws = [sd["topk_weight"].to(dev) for sd in shards]
+        outs = [torch.empty(Tr, w.H, dtype=torch.bfloat16, device=dev) for _ in range(R)]
+        err = torch.zeros(1, dtype=torch.int32, device=dev)
+        for _ in range(n):
+            for r in range(R):
+                if fp8:
+                    sep.sep_ep_dispatch_fp8(hs[r], xs[r], r, deltas[r], pools, scale_pools, prow, err, scale=w.scale)
+                else:
+                    sep.sep_ep_dispatch(hs[r], xs[r], r, deltas[r], pools, prow, err)
+            for r in range(R):
+                sep.sep_ep_combine(hs[r], y_pools, prow, deltas[r], ws[r], outs[r], err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
         for hh in hs:
             sep.sep_handle_free(hh)
     else:
